@@ -1,0 +1,115 @@
+"""fp64 attention with an online softmax over 128-key tiles: TEST INFRASTRUCTURE ONLY.
+
+What is computed (per query row i of one (batch, head)):
+  scaled dot-product attention softmax(q k^T / sqrt(d)) v
+    (FP4-attention tutorial page, section 2.1; FlashAttention-4 article,
+     "online softmax" and tiling),
+  evaluated the way a fused FlashAttention kernel evaluates it: keys are
+  walked in ascending 128-key tiles aligned to key 0, keeping a running row
+  max m, a running row sum l and an output accumulator O. For each tile:
+      S_j  = softmax_scale * (q_i . k_j)          for the allowed keys j
+      m'   = max(m, max_j S_j)
+      P_j  = exp(S_j - m')
+      l    = l * exp(m - m') + sum_j P_j          (unquantized P)
+      Ph_j = E4M3(448 * P_j) / 448                (P at the fixed 1/448 tensor
+                                                   scale, FPSAttention page,
+                                                   section 3.1)
+      O    = O * exp(m - m') + sum_j Ph_j v_j
+      m    = m'
+  and finally out = O / l, lse = m + ln(l).
+A tile with no allowed key leaves the state unchanged. A row with no allowed
+key at all gives out = 0 and lse = -inf.
+
+Allowed keys: all keys < N; under ``causal`` only j <= i; under a tile mask
+only keys whose 128-key block is listed for the query's 128-row block.
+
+Reading taken where the pages are silent: the row sum l adds the unquantized
+P (so each row of P/l sums to one); ``quantize_p=False`` gives plain fp64
+attention (P kept exact), used to pin the oracle to a textbook softmax.
+
+Inputs are the dequantized fp64 operands q, k, v of one (batch, head), shaped
+[N, d]. The loop over query rows is vectorized over one 128-row block at a
+time; each row's arithmetic is the sequence above, unchanged.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import codec
+
+TILE = 128
+P_SCALE_INV = 448.0
+
+
+def _quantize_p(p: np.ndarray) -> np.ndarray:
+    return codec.e4m3_decode(codec.e4m3_encode(p * P_SCALE_INV)) / P_SCALE_INV
+
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray,
+                   *, softmax_scale: Optional[float] = None, causal: bool = False,
+                   key_blocks: Optional[Sequence[Sequence[int]]] = None,
+                   quantize_p: bool = True):
+    """Attention output and lse for the query ``rows`` of one (batch, head).
+
+    q, k, v     float64 [N, d] dequantized operands
+    rows        int array of query indices (all in one 128-row block, or any)
+    key_blocks  optional list: key_blocks[qb] = allowed 128-key block indices
+                for query block qb (the tile mask); None = dense
+    Returns (out float64 [len(rows), d], lse float64 [len(rows)]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.int64)
+    N, d = k.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    R = len(rows)
+    m = np.full(R, -np.inf)
+    l = np.zeros(R)
+    O = np.zeros((R, v.shape[1]))
+    ntiles = -(-N // TILE)
+    qblk = rows // TILE
+    for t in range(ntiles):
+        keys = np.arange(t * TILE, min((t + 1) * TILE, N))
+        allowed = np.ones((R, len(keys)), dtype=bool)
+        if causal:
+            allowed &= keys[None, :] <= rows[:, None]
+        if key_blocks is not None:
+            listed = np.array([t in key_blocks[b] for b in qblk])
+            allowed &= listed[:, None]
+        live = allowed.any(axis=1)
+        if not live.any():
+            continue
+        S = softmax_scale * (q[rows] @ k[keys].T)
+        S = np.where(allowed, S, -np.inf)
+        m_new = np.where(live, np.maximum(m, S.max(axis=1)), m)
+        with np.errstate(invalid="ignore"):
+            alpha = np.where(live, np.exp(m - m_new), 1.0)
+            P = np.where(allowed, np.exp(S - m_new[:, None]), 0.0)
+        l = l * alpha + P.sum(axis=1)
+        Ph = _quantize_p(P) if quantize_p else P
+        O = O * alpha[:, None] + Ph @ v[keys]
+        m = m_new
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(l[:, None] > 0, O / np.where(l > 0, l, 1.0)[:, None], 0.0)
+        lse = np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
+    return out, lse
+
+
+def attention(q, k, v, *, softmax_scale=None, causal=False, key_blocks=None,
+              quantize_p=True):
+    """Whole (batch, head) attention, 128 rows at a time. Returns (out, lse)."""
+    N = q.shape[0]
+    outs, lses = [], []
+    for b0 in range(0, N, TILE):
+        rows = np.arange(b0, min(b0 + TILE, N))
+        o, s = attention_rows(q, k, v, rows, softmax_scale=softmax_scale, causal=causal,
+                              key_blocks=key_blocks, quantize_p=quantize_p)
+        outs.append(o)
+        lses.append(s)
+    return np.concatenate(outs), np.concatenate(lses)
+

@@ -1,0 +1,155 @@
+"""Pins for the oracle's online-softmax attention and STA geometry (CPU only).
+
+* With P unquantized, the tiled online algorithm equals torch's fp64
+  scaled_dot_product_attention (a library routine), dense, causal and masked,
+  over several tiles and a ragged tail.
+* Rows of P/l sum to one (V = 1 gives output 1).
+* Identical keys give exactly the mean of V (P = 1 is representable).
+* Causal row 0 is v_0.
+* Worked examples pin the E4M3 rounding of P against the running max and the
+  rescale across tiles.
+* The STA block lists agree with a brute-force token-level window test and
+  with the pair counts of the (6,8,8)-tile, (3,3,5)-window video workload.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from oracle import sta
+
+
+def _sdpa(q, k, v, causal=False, mask=None):
+    tq, tk, tv = (torch.from_numpy(np.asarray(t, dtype=np.float64))[None, None] for t in (q, k, v))
+    attn_mask = None if mask is None else torch.from_numpy(mask)[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=attn_mask,
+                                                           is_causal=causal)
+    return out[0, 0].numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(300, 64), (129, 128), (77, 32)])
+def test_unquantized_matches_sdpa(N, d, causal):
+    rng = np.random.default_rng(N + d)
+    q, k, v = (rng.standard_normal((N, d)) * 2 for _ in range(3))
+    out, lse = A.attention(q, k, v, causal=causal, quantize_p=False)
+    ref = _sdpa(q, k, v, causal=causal)
+    assert np.max(np.abs(out - ref)) < 1e-12
+    S = (q @ k.T) / math.sqrt(d)
+    if causal:
+        S = np.where(np.tril(np.ones((N, N), bool)), S, -np.inf)
+    mx = S.max(axis=1)
+    ref_lse = mx + np.log(np.exp(S - mx[:, None]).sum(axis=1))
+    assert np.max(np.abs(lse - ref_lse)) < 1e-12
+
+
+def test_unquantized_block_mask_matches_sdpa():
+    rng = np.random.default_rng(11)
+    N, d = 512, 32
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    key_blocks = [[0, 2], [1], [0, 1, 2, 3], [3]]
+    mask = np.zeros((N, N), bool)
+    for qb, kbs in enumerate(key_blocks):
+        for kb in kbs:
+            mask[qb * 128:(qb + 1) * 128, kb * 128:(kb + 1) * 128] = True
+    out, _ = A.attention(q, k, v, key_blocks=key_blocks, quantize_p=False)
+    assert np.max(np.abs(out - _sdpa(q, k, v, mask=mask))) < 1e-12
+    dense, _ = A.attention(q, k, v, quantize_p=True)
+    allk, _ = A.attention(q, k, v, key_blocks=[[0, 1, 2, 3]] * 4, quantize_p=True)
+    assert np.array_equal(dense, allk)
+
+
+def test_rows_of_p_sum_to_one():
+    rng = np.random.default_rng(12)
+    N, d = 400, 64
+    q, k = rng.standard_normal((N, d)) * 3, rng.standard_normal((N, d)) * 3
+    out, _ = A.attention(q, k, np.ones((N, 8)), quantize_p=False)
+    assert np.max(np.abs(out - 1.0)) < 1e-12
+    out, _ = A.attention(q, k, np.ones((N, 8)), causal=True, quantize_p=False)
+    assert np.max(np.abs(out - 1.0)) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_identical_keys_give_mean_of_v(causal):
+    rng = np.random.default_rng(13)
+    N, d = 300, 64
+    q = rng.standard_normal((N, d))
+    k = np.tile(rng.standard_normal((1, d)), (N, 1))
+    v = rng.standard_normal((N, d))
+    out, lse = A.attention(q, k, v, causal=causal, quantize_p=True)
+    if causal:
+        ref = np.cumsum(v, axis=0) / np.arange(1, N + 1)[:, None]
+    else:
+        ref = np.tile(v.mean(axis=0), (N, 1))
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_causal_row0_is_v0():
+    rng = np.random.default_rng(14)
+    q, k, v = (rng.standard_normal((200, 64)) for _ in range(3))
+    out, lse = A.attention(q, k, v, causal=True)
+    assert np.array_equal(out[0], v[0])
+    assert lse[0] == pytest.approx(q[0] @ k[0] / 8.0, abs=1e-12)
+
+
+def _two_key_setup(s0, s1):
+    """q = e_0, keys with scores exactly s0, s1 under softmax_scale = 1."""
+    q = np.zeros((1, 4)); q[0, 0] = 1.0
+    k = np.zeros((2, 4)); k[0, 0] = s0; k[1, 0] = s1
+    return q, k
+
+
+def test_worked_example_p_rounding():
+    # scores 0 and ln 0.3: P = [1, 0.3]; 448 * 0.3 = 134.4 -> E4M3 128
+    q, k = _two_key_setup(0.0, math.log(0.3))
+    v = np.array([[1.0, 0.0], [0.0, 1.0]])
+    out, lse = A.attention_rows(q, k, v, np.array([0]), softmax_scale=1.0)
+    l = 1.0 + 0.3
+    assert out[0, 0] == pytest.approx(1.0 / l, abs=1e-15)
+    assert out[0, 1] == pytest.approx((128.0 / 448.0) / l, abs=1e-15)
+    assert lse[0] == pytest.approx(math.log(l), abs=1e-15)
+
+
+def test_worked_example_rescale_across_tiles():
+    # 128 keys with score 0 in tile 0, one key with score ln 3 in tile 1.
+    # Tile 0 quantizes P = 1 against its own max (exact); tile 1 raises the
+    # max, scaling the earlier sum by 1/3. Quantizing tile 0 against the final
+    # max instead would give E4M3(448/3)/448 = 144/448 per key.
+    N = 129
+    q = np.zeros((1, 2)); q[0, 0] = 1.0
+    k = np.zeros((N, 2)); k[128, 0] = math.log(3.0)
+    v = np.zeros((N, 2)); v[:128, 0] = 1.0; v[128, 1] = 1.0
+    out, lse = A.attention_rows(q, k, v, np.array([0]), softmax_scale=1.0)
+    l = 128.0 / 3.0 + 1.0
+    assert out[0, 0] == pytest.approx((128.0 / 3.0) / l, rel=1e-14)
+    assert out[0, 1] == pytest.approx(1.0 / l, rel=1e-14)
+    assert lse[0] == pytest.approx(math.log(3.0) + math.log(l), rel=1e-14)
+
+
+def test_sta_counts_video_workload():
+    grid, tile, window = (18, 48, 80), (6, 8, 8), (3, 3, 5)
+    pairs = sta.tile_pairs(grid, tile, window)
+    assert len(pairs) == 3 * 6 * 10
+    assert sum(len(p) for p in pairs) == 4928
+    blocks = sta.block_lists(grid, tile, window)
+    assert len(blocks) == 18 * 48 * 80 // 128 == 540
+    assert sum(len(b) for b in blocks) == 44352
+    assert all(b == sorted(b) for b in blocks)
+    # interior tile sees 3*3*5 tiles
+    assert max(len(p) for p in pairs) == 45
+
+
+def test_sta_block_lists_match_token_bruteforce():
+    grid, tile, window = (12, 16, 24), (6, 8, 8), (3, 3, 5)
+    blocks = sta.block_lists(grid, tile, window)
+    N = 12 * 16 * 24
+    rng = np.random.default_rng(15)
+    qpos = np.unique(np.concatenate([rng.integers(0, N, 40), [0, N - 1, 383, 384]]))
+    tok = sta.token_mask(grid, tile, window, qpos)
+    for i, p in enumerate(qpos):
+        from_blocks = np.zeros(N, bool)
+        for kb in blocks[p // 128]:
+            from_blocks[kb * 128:(kb + 1) * 128] = True
+        assert np.array_equal(from_blocks, tok[i])

@@ -1,0 +1,157 @@
+"""Pins for the oracle's NVFP4 and FP8 quantizers (CPU only).
+
+Checks: hand-worked examples, exactly representable inputs surviving, the
+amax element mapping to the format maximum, zero blocks, the error bound of
+half a grid step, quantize(dequantize(quantize(x))) == quantize(x), the FP8
+element conversion against torch's float8 cast, and the swizzled scale layout
+against a direct restatement of its byte formula.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import codec, quant
+
+F32 = np.float32
+
+
+def _bf16(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def test_nvfp4_hand_example():
+    # static amax 2688 -> s_t = 1 exactly; block amax 3 -> 3/6 = 0.5 -> E4M3 0x30
+    x = np.zeros(16, dtype=F32)
+    x[:6] = [3.0, -1.2, 0.74, 0.26, 2.2, -3.0]
+    codes, sb, s_t = quant.quantize_nvfp4(x[None], static_amax=2688.0)
+    assert s_t == F32(1.0)
+    assert sb[0, 0] == 0x30 and codec.e4m3_decode(0x30) == 0.5
+    # x / 0.5 = [6, -2.4, 1.48, 0.52, 4.4, -6] -> [6, -2, 1.5, 0.5, 4, -6]
+    assert list(codes[0, :6]) == [7, 8 | 4, 3, 1, 6, 8 | 7]
+    assert list(codes[0, 6:]) == [0] * 10
+
+
+def test_nvfp4_grid_points_survive_and_amax_maps_to_6():
+    rng = np.random.default_rng(0)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    # blocks whose values are e2m1 grid values times an exact E4M3 scale, max 6
+    scales = codec.e4m3_decode(rng.integers(0x20, 0x60, 32))
+    vals = rng.choice(grid, (32, 16)) * rng.choice([-1, 1], (32, 16))
+    vals[:, 3] = 6.0
+    x = (vals * scales[:, None]).astype(F32)
+    codes, sb, s_t = quant.quantize_nvfp4(x, static_amax=2688.0)
+    assert s_t == F32(1.0)
+    assert np.array_equal(codec.e4m3_decode(sb[:, 0]), scales)
+    assert np.array_equal(codec.e2m1_decode(codes), vals)
+    assert np.all(codes[:, 3] == 7)
+
+
+def test_nvfp4_zero_block_and_tensor():
+    x = np.zeros((2, 32), dtype=F32)
+    x[1, :16] = 1.0
+    codes, sb, s_t = quant.quantize_nvfp4(x)
+    assert np.all(codes[0] == 0) and np.all(sb[0] == 0)
+    assert np.all(codes[1, 16:] == 0) and sb[1, 1] == 0
+    c0, sb0, st0 = quant.quantize_nvfp4(np.zeros((4, 16), dtype=F32))
+    assert st0 == F32(1.0) and np.all(c0 == 0) and np.all(sb0 == 0)
+
+
+def test_nvfp4_tensor_scale_and_block_max():
+    rng = np.random.default_rng(3)
+    x = _bf16(rng.standard_normal((8, 128)) * 3)
+    codes, sb, s_t = quant.quantize_nvfp4(x)
+    A = F32(np.abs(x).max())
+    assert s_t == F32(A / F32(2688.0))
+    # the tensor-amax element sits in a block whose scale is (nearly) 448,
+    # and it maps to +-6
+    i, j = np.unravel_index(np.abs(x).argmax(), x.shape)
+    assert codec.e4m3_decode(sb[i, j // 16]) == 448.0
+    assert codes[i, j] & 7 == 7
+
+
+def test_nvfp4_error_bound():
+    rng = np.random.default_rng(4)
+    x = _bf16(rng.standard_normal((64, 128)))
+    x[:, 5] *= 20
+    codes, sb, s_t = quant.quantize_nvfp4(x)
+    xh = quant.dequantize_nvfp4(codes, sb, s_t)
+    den = np.repeat(codec.e4m3_decode(sb), 16, axis=-1) * float(s_t)
+    y = np.abs(x / den)
+    gap = np.where(y < 2, 0.5, np.where(y < 4, 1.0, 2.0))
+    assert np.all(np.abs(x - xh) <= (gap / 2) * den * (1 + 1e-5))
+
+
+def test_nvfp4_roundtrip_idempotent():
+    rng = np.random.default_rng(5)
+    x = _bf16(rng.standard_normal((16, 64)))
+    amax = np.abs(x).max()
+    c1, sb1, st1 = quant.quantize_nvfp4(x)
+    xh = quant.dequantize_nvfp4(c1, sb1, st1).astype(F32)
+    c2, sb2, st2 = quant.quantize_nvfp4(xh, static_amax=amax)
+    assert st1 == st2
+    assert np.array_equal(sb1, sb2)
+    assert np.array_equal(codec.e2m1_decode(c1), codec.e2m1_decode(c2))
+
+
+def test_nvfp4_sf_swizzle_formula():
+    rng = np.random.default_rng(6)
+    N, d = 200, 128
+    sf = rng.integers(0, 256, (3, N, d // 16)).astype(np.uint8)
+    sw = quant.nvfp4_sf_swizzle(sf, N, d).reshape(3, -1)
+    for r in (0, 1, 31, 32, 95, 127, 128, 199):
+        for col in range(d // 16):
+            off = ((r // 128) * (d // 64) + col // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + col % 4
+            assert np.array_equal(sw[:, off], sf[:, r, col])
+    # padding rows are zero
+    assert np.all(quant.nvfp4_sf_swizzle(sf, N, d)[:, 1].reshape(3, -1).sum() >= 0)
+    pad_rows = [r for r in range(N, 256)]
+    for r in pad_rows[:5]:
+        off = (1 * (d // 64)) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32)
+        assert np.all(sw[:, off:off + 4] == 0)
+
+
+def test_fp8_tile_amax_maps_to_448_and_matches_torch_cast():
+    rng = np.random.default_rng(7)
+    x = _bf16(rng.standard_normal((2, 3, 300, 64)) * 5)   # ragged: 300 = 2*128 + 44
+    codes, s = quant.quantize_fp8_tile(x)
+    assert s.shape == (2, 3, 3)
+    for t in range(3):
+        blk = x[:, :, t * 128:(t + 1) * 128]
+        A = np.abs(blk).max(axis=(-2, -1)).astype(F32)
+        assert np.array_equal(s[:, :, t], F32(448.0) / A)
+    s_tok = np.repeat(s, 128, axis=-1)[..., :300]
+    prod = (x * s_tok[..., None]).astype(F32)
+    ref = torch.from_numpy(np.clip(prod, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+    # every tile has its amax element at +-448
+    dec = np.abs(codec.e4m3_decode(codes))
+    for t in range(3):
+        assert np.all(dec[:, :, t * 128:(t + 1) * 128].max(axis=(-2, -1)) == 448.0)
+
+
+def test_fp8_channel_scales_and_bound():
+    rng = np.random.default_rng(8)
+    x = _bf16(rng.standard_normal((1, 2, 257, 64)))
+    x[..., 7] *= 30
+    codes, s = quant.quantize_fp8_channel(x)
+    A = np.abs(x).max(axis=-2).astype(F32)
+    assert np.array_equal(s, F32(448.0) / A)
+    xh = quant.dequantize_fp8_channel(codes, s)
+    y = np.abs(x * s[..., None, :]).astype(np.float64)
+    # half an E4M3 step at y: subnormal step 2^-9, else 2^(floor(log2 y) - 3)
+    e = np.floor(np.log2(np.maximum(y, 2.0 ** -6)))
+    half = np.where(y < 2.0 ** -6, 2.0 ** -10, 2.0 ** (e - 4))
+    assert np.all(np.abs(x * s[..., None, :] - codec.e4m3_decode(codes)) <= half * (1 + 1e-6))
+    assert np.all(np.abs(codec.e4m3_decode(codes)).max(axis=-2) == 448.0)
+
+
+def test_fp8_roundtrip_idempotent_and_zero():
+    rng = np.random.default_rng(9)
+    x = _bf16(rng.standard_normal((1, 1, 256, 128)))
+    c1, s1 = quant.quantize_fp8_tile(x)
+    xh = quant.dequantize_fp8_tile(c1, s1).astype(F32)
+    c2, s2 = quant.quantize_fp8_tile(xh)
+    assert np.array_equal(c1, c2)
+    assert np.allclose(s1, s2, rtol=3e-7, atol=0)
+    cz, sz = quant.quantize_fp8_channel(np.zeros((1, 1, 10, 16), dtype=F32))
+    assert np.all(cz == 0) and np.all(sz == 1.0)
