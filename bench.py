@@ -1,0 +1,338 @@
+"""Benchmark of the quantized attention hot path on B200.
+
+One step = the whole path on one batch of synthetic input already resident
+in HBM: NVFP4 quantization of Q and K, per-channel FP8 quantization of V, and
+the fused attention forward (LLM prefill workload: B=4, H=32, N=4096, d=128,
+causal; QK^T in NVFP4, PV in FP8). W untimed warm-up steps, then exactly K
+timed steps bracketed by a barrier and a device synchronize, timed with CUDA
+events on the launching stream; multi-GPU runs take the max over ranks. Rank 0
+prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+``--impl reference`` times the CPU oracle (the only other implementation of
+this path) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "quantized attention fwd TFLOPS & % of B200 FP4/FP8 peak; quantize HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal dense ratios to bf16 (B200: bf16 2.25, fp8 4.5, fp4 9 PFLOP/s)
+FP8_RATIO, FP4_RATIO = 2.0, 4.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def executed_block_pairs(w: workloads.Workload) -> int:
+    """128x128 (query block, key block) pairs the kernel computes per head."""
+    nblk = (w.N + 127) // 128
+    if w.sparse:
+        import precision_attention_nvfp4_b200 as fp
+        tg = tuple(a // b for a, b in zip(w.video, w.sta_tile))
+        return fp.sta_plan(tg, w.sta_tile, w.sta_window).nnz
+    return nblk * (nblk + 1) // 2 if w.causal else nblk * nblk
+
+
+def quant_bytes(w: workloads.Workload) -> float:
+    """Algorithmic HBM bytes of one step's quantization (two-pass amax)."""
+    n = w.B * w.H * w.N * w.d
+    if w.qk_format == "nvfp4":
+        qk = 2 * n * (2 + 2 + 0.5 + 1.0 / 16)   # amax read + quant read + codes + scales
+    else:
+        qk = 2 * n * (2 + 1)                    # single pass per 128-token tile
+    v = n * (2 + 2 + 1)                         # channel amax pass + quant pass
+    return qk + v
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks):
+    """Run the oracle (as it stands) on a bounded sample; returns (flops, seconds)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import parity
+    from oracle import attention as oatt
+    t0 = time.perf_counter()
+    qh, kh, vh = parity.oracle_operands(q, k, v, w.qk_format, heads)
+    flops = 0.0
+    for i, _ in enumerate(heads):
+        for qb in qblocks:
+            rows = np.arange(qb * 128, min(w.N, qb * 128 + 128))
+            oatt.attention_rows(qh[i], kh[i], vh[i], rows, causal=w.causal)
+            keys = (rows + 1) if w.causal else np.full(len(rows), w.N)
+            flops += float(np.sum(4.0 * keys * w.d))
+    return flops, time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, w):
+    """CPU oracle arm: each step a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v = workloads.make_qkv(w, heads=1, batch=1)
+    nblk = (w.N + 127) // 128
+    qblocks = [nblk - 1, nblk // 2]
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, q, k, v, [0], qblocks)
+    tot_f, tot_s = 0.0, 0.0
+    for _ in range(args.steps):
+        f, s = cpu_oracle_sample(w, q, k, v, [0], qblocks)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    sample = f"1 head, query blocks {qblocks} of {w.name} per step (oracle quantization of that head included)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "qk": w.qk_format, "pv": "e4m3", "sparse": w.sparse,
+            "l2": "inputs larger than L2 (bf16 Q,K,V of the step exceed 126 MB)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llm_prefill_causal")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import precision_attention_nvfp4_b200 as fp
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # weak scaling: every rank runs one full batch of the workload
+    q_h, k_h, v_h = workloads.make_qkv(w)
+    q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
+    mask = None
+    if w.sparse:
+        tg = tuple(a // b for a, b in zip(w.video, w.sta_tile))
+        mask = fp.sta_plan(tg, w.sta_tile, w.sta_window).to("cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev_pair=None):
+        if w.qk_format == "nvfp4":
+            qq, kq = fp.quantize_nvfp4(q), fp.quantize_nvfp4(k)
+        else:
+            qq, kq = fp.quantize_fp8(q, "tile128"), fp.quantize_fp8(k, "tile128")
+        vq = fp.quantize_fp8(v, "channel")
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+        return out
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert fp.device_error() == 0
+
+    clocks = ClockSampler(local)
+    attn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    for i in range(args.steps):
+        step(attn_events[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total)
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_events]))
+    attn_ms = max_over_ranks(attn_ms)
+    err = fp.device_error()
+
+    flops = w.dense_flops()
+    pairs = executed_block_pairs(w)
+    exec_flops = 4.0 * 128 * 128 * w.d * pairs * w.B * w.H
+    ms_step = ms_total / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    bf16 = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
+    peak = 2.0 / (1.0 / p4 + 1.0 / p8) if w.qk_format == "nvfp4" else p8
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    quant_ms = ms_step - attn_ms
+    quant_gbs = quant_bytes(w) / (quant_ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host bf16 in, host bf16 out
+    e2e = None
+    if rank == 0 or world > 1:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
+        lse_h = torch.empty(q_h.shape[:3], dtype=torch.float32, pin_memory=True)
+        fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
+                     lse_host=lse_h)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
+                         lse_host=lse_h)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
+        h2d = 3 * q_h.numel() * 2
+        d2h = out_h.numel() * 2 + lse_h.numel() * 4
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nblk = (w.N + 127) // 128
+        heads = [0, w.B * w.H // 2]
+        qblocks = [nblk - 1, nblk // 2, 1]
+        f, s = cpu_oracle_sample(w, q_h, k_h, v_h, heads, qblocks)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
+               "sample": f"heads {heads}, query blocks {qblocks} of {w.name} (fp64 numpy, oracle "
+                         f"quantization of those heads included), {s:.1f} s"}
+
+    launches_per_step = (6 if w.qk_format == "nvfp4" else 2) + 3 + 1
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e2m1/e4m3 MMA, f32 accumulate", "data": "synthetic",
+            "config": config_dict(w),
+            "attn_ms": attn_ms, "attn_tflops_dense_eq": attn_tflops,
+            "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,
+            "quant_ms": quant_ms, "quant_gbs": quant_gbs, "quant_frac_hbm": quant_gbs / peaks["hbm_gbs"],
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": attn_tflops / peak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 sustained {bf16} x nominal fp8 2x / fp4 4x; "
+                                        f"{'harmonic mix of fp4 QK and fp8 PV' if w.qk_format == 'nvfp4' else 'fp8'}"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk, "device_error": err,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,233 @@
+/*
+ * fpattn: quantized attention forward for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of the library. Every entry point takes plain pointers and sizes; no
+ * C++ or framework types cross this boundary.
+ *
+ * What the library computes
+ *   softmax(Q K^T / sqrt(d)) V  (FP4-attention tutorial page, section 2.1),
+ *   with Q, K, V first quantized either
+ *     - to NVFP4: E2M1 values in 16-element blocks along d, an E4M3 block
+ *       scale per block and an FP32 tensor scale (Blackwell FP4 practice page,
+ *       section 1, "micro-scaling": the scale is stored in FP8), or
+ *     - to FP8 E4M3 in the FPSAttention staged scheme (FPSAttention page,
+ *       section 2.1 conversion formula, section 3.1 "staged quantization":
+ *       Q/K per block, V per channel, P per tensor at a fixed scale 1/448),
+ *   and attention then run as one fused kernel with FP32 accumulation and an
+ *   online softmax over 128-key tiles (FlashAttention-4 article: tiling,
+ *   online softmax, kernel fusion), optionally restricted to a 3D
+ *   sliding-tile pattern over video tokens (FPSAttention page, section 2.2)
+ *   and/or a causal mask.
+ *
+ * Conventions shared by all entry points
+ *   - The caller owns all memory. Tensor data pointers are DEVICE pointers on
+ *     the current CUDA device unless stated otherwise. The library allocates
+ *     no memory and never synchronizes the device; work is enqueued on the
+ *     given stream in stream order.
+ *   - Tensors are contiguous [B, H, N, d] row-major (d fastest). Data pointers
+ *     must be 16-byte aligned (FPATTN_ERR_ALIGNMENT otherwise).
+ *   - Argument and shape errors are returned before any work is enqueued.
+ *     A failed launch returns FPATTN_ERR_CUDA. A bounded device-side wait
+ *     that expired is recorded in a device error word that
+ *     fpattn_device_error() reads.
+ *   - Inputs are expected to be finite; non-finite inputs give unspecified
+ *     codes and set the optional device flag *nonfinite_flag to 1.
+ *   - Self-attention only: Q, K and V share B, H, N and d.
+ */
+#ifndef FPATTN_H_
+#define FPATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fpattn_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  FPATTN_OK = 0,
+  FPATTN_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, inconsistent tensors */
+  FPATTN_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}, dtype pair not supported, tile mask shape */
+  FPATTN_ERR_ALIGNMENT = 3,    /* a data pointer is not 16-byte aligned */
+  FPATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  FPATTN_ERR_TIMEOUT = 5       /* a bounded device wait expired (see fpattn_device_error) */
+} fpattn_status;
+
+typedef enum {
+  FPATTN_BF16 = 0,  /* 2 bytes per element */
+  FPATTN_E4M3 = 1,  /* 1 byte per element (OCP FP8 E4M3, max 448) */
+  FPATTN_NVFP4 = 2  /* packed E2M1 codes, 2 per byte: element 2i in the low nibble of byte i */
+} fpattn_dtype;
+
+/* A contiguous [B, H, N, d] tensor. For NVFP4 the data holds B*H*N*d/2 bytes. */
+typedef struct {
+  void* data;
+  int32_t dtype; /* fpattn_dtype */
+  int32_t B, H, N, d;
+} fpattn_tensor;
+
+/* Quantization granularity for fpattn_quantize_fp8. */
+typedef enum {
+  FPATTN_FP8_TILE128 = 0, /* one scale per (b, h, 128-token tile): Q and K */
+  FPATTN_FP8_CHANNEL = 1  /* one scale per (b, h, channel) over all N tokens: V */
+} fpattn_fp8_granularity;
+
+/*
+ * Size in bytes of the NVFP4 block-scale buffer for a [B, H, N, d] tensor:
+ * B*H*ceil(N/128)*(d/64)*512.
+ *
+ * Layout ("tensor-core scale layout"): for each (b, h), each 128-row block nb
+ * and each group a of four 16-element scale columns, 512 bytes in which the
+ * E4M3 scale of row r = nb*128 + 32*j + i (i < 32, j < 4) and column
+ * 4*a + c (c < 4) is byte 16*i + 4*j + c. Rows at or past N are zero. This is
+ * the arrangement the block-scaled tensor-core MMA reads its scale vectors
+ * in, so the attention kernel copies it to tensor memory unchanged.
+ */
+size_t fpattn_nvfp4_sf_bytes(int32_t B, int32_t H, int32_t N, int32_t d);
+
+/*
+ * NVFP4 quantization of a bf16 tensor (Blackwell FP4 practice page,
+ * section 1, micro-scaling with an FP8 scale; two-level arithmetic as below).
+ *
+ *   A_t = static_amax ? *static_amax : max|x| over the whole tensor
+ *   s_t = A_t / 2688            (2688 = 6 * 448; 1 when A_t == 0)
+ *   per 16-element block along d:
+ *     sb   = E4M3(A_b / (6 * s_t)),   den = dec(sb) * s_t,
+ *     code = E2M1(x * (1/den))  (round to nearest even, saturating at 6;
+ *                                all codes 0 when den == 0)
+ * Every step is one correctly rounded fp32 operation, so results are bit-exact
+ * against the CPU oracle. Dequantized value: E2M1val * dec(sb) * s_t.
+ *
+ * x             bf16 input tensor (dtype FPATTN_BF16), d in {64, 128}
+ * static_amax   device pointer to one float, or NULL for dynamic (per call)
+ * codes         device, B*H*N*d/2 bytes, packed E2M1
+ * block_sf      device, fpattn_nvfp4_sf_bytes() bytes, tensor-core scale layout
+ * tensor_scale  device pointer to one float: receives s_t
+ * nonfinite_flag  optional device int, set to 1 if x holds a non-finite value
+ *                 (only written in dynamic mode; the caller zeroes it)
+ */
+fpattn_status fpattn_quantize_nvfp4(const fpattn_tensor* x, const float* static_amax,
+                                    uint8_t* codes, uint8_t* block_sf, float* tensor_scale,
+                                    int32_t* nonfinite_flag, fpattn_stream_t stream);
+
+/*
+ * FP8 E4M3 quantization of a bf16 tensor (FPSAttention page, section 2.1:
+ * X_hat = dequantize(FP8_convert(X * s_g)) / s_g; section 3.1: Q/K per block,
+ * V per channel).
+ *
+ *   s    = 448 / A   (A = amax of the tile or channel; 1 when A == 0)
+ *   code = E4M3(x * s), round to nearest even, saturating at 448.
+ *
+ * x            bf16 input tensor, d in {64, 128}
+ * granularity  FPATTN_FP8_TILE128: A over one (b, h, 128-token tile) x d
+ *              (a last partial tile uses its valid tokens); scales has
+ *              B*H*ceil(N/128) floats.
+ *              FPATTN_FP8_CHANNEL: A over all N tokens of one (b, h, channel);
+ *              scales has B*H*d floats.
+ * codes        device, B*H*N*d bytes, same [B, H, N, d] layout as x
+ * scales       device floats: receives s (a multiplier: x ~ dec(code) / s)
+ * nonfinite_flag  optional device int (see above)
+ */
+fpattn_status fpattn_quantize_fp8(const fpattn_tensor* x, int32_t granularity, uint8_t* codes,
+                                  float* scales, int32_t* nonfinite_flag, fpattn_stream_t stream);
+
+/* Scales consumed by fpattn_fwd. */
+typedef struct {
+  /* NVFP4 Q/K: device pointer to the one-float tensor scale s_t.
+     E4M3 Q/K: device pointer to B*H*ceil(N/128) per-tile multipliers. */
+  const float* q_scale;
+  const float* k_scale;
+  /* E4M3 V: device pointer to B*H*d per-channel multipliers. */
+  const float* v_scale;
+  /* NVFP4 Q/K: device block scales in the tensor-core scale layout; else NULL. */
+  const uint8_t* q_block_sf;
+  const uint8_t* k_block_sf;
+  /* Scale of the E4M3 softmax probabilities; must be 1/448 (FPSAttention
+     page, section 3.1: P per tensor at a fixed 1/448). */
+  float p_scale;
+  /* Multiplier of Q K^T before the softmax; 0 selects 1/sqrt(d). */
+  float softmax_scale;
+} fpattn_scales;
+
+/*
+ * Block-sparse tile mask over 128-token blocks, shared by all (b, h):
+ * query block qb attends exactly key blocks col_idx[row_ptr[qb] ..
+ * row_ptr[qb+1]), which must be ascending and < ceil(N/128). All arrays are
+ * DEVICE int32. row_order (optional, may be NULL) lists the query blocks in
+ * the order the kernel should schedule them (a permutation of 0..nblk_q-1,
+ * e.g. longest row first).
+ */
+typedef struct {
+  int32_t nblk_q;          /* must equal ceil(N/128) */
+  int32_t nnz;             /* row_ptr[nblk_q] */
+  const int32_t* row_ptr;  /* nblk_q + 1 entries */
+  const int32_t* col_idx;  /* nnz entries */
+  const int32_t* row_order;
+} fpattn_tile_mask_desc;
+
+/*
+ * 3D sliding-tile planner (FPSAttention page, section 2.2: query tile u
+ * attends key tiles v with ||c_u - c_v||_inf within the window). HOST-only,
+ * integer work.
+ *
+ * Tokens of an nt*tt x nh*th x nw*tw video are taken in tile-major order
+ * (tiles in raster order, tokens raster order within a tile). The tile volume
+ * tt*th*tw must be a multiple of 128 so that every 128-token block lies in one
+ * tile (FPATTN_ERR_UNSUPPORTED otherwise). The window (wt, wh, ww) is in
+ * tiles; the half-width per axis is floor(w/2), clipped at the grid edges.
+ *
+ * Writes the CSR of fpattn_tile_mask_desc into HOST arrays:
+ *   row_ptr[nblk_q + 1], col_idx[nnz], row_order[nblk_q] (rows sorted by
+ *   descending length, ties by index). *nblk_q_out and *nnz_out receive the
+ *   sizes. If col_cap < nnz (or any array is NULL), nothing but the sizes is
+ *   written and FPATTN_OK is returned, so a first call with col_cap = 0 sizes
+ *   the buffers.
+ */
+fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, int32_t th,
+                              int32_t tw, int32_t wt, int32_t wh, int32_t ww,
+                              int32_t* row_ptr, int32_t* col_idx, int32_t* row_order,
+                              size_t col_cap, int32_t* nblk_q_out, int32_t* nnz_out);
+
+/*
+ * Fused quantized attention forward.
+ *
+ * q, k        both FPATTN_NVFP4 (QK^T on block-scaled FP4 tensor cores) or
+ *             both FPATTN_E4M3 (FP8 tensor cores)
+ * v           FPATTN_E4M3 with per-channel scales (PV on FP8 tensor cores,
+ *             P in E4M3 at scale 1/448)
+ * scales      as described in fpattn_scales
+ * tile_mask   NULL for dense, else a block mask (may be combined with causal)
+ * causal      nonzero: key j attends query i only when j <= i
+ * out         device bf16 [B, H, N, d]
+ * lse         device float [B, H, N], natural-log log-sum-exp of the scaled
+ *             scores of each row, or NULL
+ * Per row, keys are walked in ascending 128-key tiles with a running max m,
+ * a running sum l of the unquantized P, and O += E4M3(448 P) V; the output is
+ * O / (448 l) with the V and P scales folded in. A row with no allowed key
+ * gets out = 0 and lse = -inf.
+ */
+fpattn_status fpattn_fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                         const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask,
+                         int32_t causal, void* out, float* lse, fpattn_stream_t stream);
+
+/*
+ * Reads (and, if clear != 0, resets) the library's device error word on the
+ * current device. Synchronizes `stream`. Returns FPATTN_OK when no bounded
+ * wait has expired, FPATTN_ERR_TIMEOUT otherwise; *code (if non-NULL)
+ * receives the raw word (which wait gave up).
+ */
+fpattn_status fpattn_device_error(fpattn_stream_t stream, int32_t clear, int32_t* code);
+
+/* Human-readable name of a status code (static storage). */
+const char* fpattn_status_string(fpattn_status status);
+
+/* Library version string, e.g. "fpattn 0.1 sm_100a". */
+const char* fpattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FPATTN_H_ */

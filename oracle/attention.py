@@ -73,13 +73,16 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray
     O = np.zeros((R, v.shape[1]))
     ntiles = -(-N // TILE)
     qblk = rows // TILE
+    listed_sets = None
+    if key_blocks is not None:
+        listed_sets = {int(b): set(key_blocks[b]) for b in np.unique(qblk)}
     for t in range(ntiles):
         keys = np.arange(t * TILE, min((t + 1) * TILE, N))
         allowed = np.ones((R, len(keys)), dtype=bool)
         if causal:
             allowed &= keys[None, :] <= rows[:, None]
         if key_blocks is not None:
-            listed = np.array([t in key_blocks[b] for b in qblk])
+            listed = np.array([t in listed_sets[int(b)] for b in qblk])
             allowed &= listed[:, None]
         live = allowed.any(axis=1)
         if not live.any():

@@ -1,0 +1,229 @@
+"""Quantized attention forward (NVFP4 / FP8) for B200, Python binding.
+
+Every function marshals torch tensors into the C ABI of ``libfpattn.so``
+(include/fpattn.h) and enqueues the library's CUDA kernels on the current
+torch stream; torch only provides device memory and streams. Nothing here
+computes any part of the method on the host.
+
+Public calls
+  quantize_nvfp4(x)            -> Nvfp4Tensor(codes, block_sf, tensor_scale)
+  quantize_fp8(x, granularity) -> Fp8Tensor(codes, scales)
+  sta_plan(grid, tile, window) -> StaPlan (host CSR over 128-token blocks)
+  attention_fwd(q, k, v, ...)  -> (out, lse) on quantized operands
+  attention(q, k, v, ...)      -> (out, lse) from bf16 inputs: quantize + fwd;
+                                  host (pinned) inputs are copied in and the
+                                  result copied back.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import FpattnError
+
+__all__ = ["Nvfp4Tensor", "Fp8Tensor", "StaPlan", "quantize_nvfp4", "quantize_fp8", "sta_plan",
+           "attention_fwd", "attention", "device_error", "library", "FpattnError"]
+
+
+def library() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _desc(t: torch.Tensor, dtype: int, B: int, H: int, N: int, d: int) -> _lib.Tensor:
+    return _lib.Tensor(t.data_ptr(), dtype, B, H, N, d)
+
+
+def _check_bf16(x: torch.Tensor) -> Tuple[int, int, int, int]:
+    if x.dim() != 4 or x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("expected a contiguous CUDA bf16 tensor [B, H, N, d]")
+    return tuple(x.shape)
+
+
+@dataclasses.dataclass
+class Nvfp4Tensor:
+    codes: torch.Tensor         # uint8 [B, H, N, d/2], packed E2M1
+    block_sf: torch.Tensor      # uint8 [B*H*ceil(N/128)*(d/64)*512], tensor-core scale layout
+    tensor_scale: torch.Tensor  # float32 [1]
+    shape: Tuple[int, int, int, int]
+
+
+@dataclasses.dataclass
+class Fp8Tensor:
+    codes: torch.Tensor         # uint8 [B, H, N, d] (E4M3 bits)
+    scales: torch.Tensor        # float32 [B, H, ceil(N/128)] or [B, H, d]
+    granularity: str            # "tile128" or "channel"
+    shape: Tuple[int, int, int, int]
+
+
+def quantize_nvfp4(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
+                   nonfinite_flag: Optional[torch.Tensor] = None) -> Nvfp4Tensor:
+    B, H, N, d = _check_bf16(x)
+    lib = library()
+    codes = torch.empty((B, H, N, d // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(lib.fpattn_nvfp4_sf_bytes(B, H, N, d), dtype=torch.uint8, device=x.device)
+    ts = torch.empty(1, dtype=torch.float32, device=x.device)
+    st = lib.fpattn_quantize_nvfp4(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), _ptr(static_amax),
+                                   codes.data_ptr(), sf.data_ptr(), ts.data_ptr(), _ptr(nonfinite_flag),
+                                   _stream())
+    _lib.check(st, "fpattn_quantize_nvfp4")
+    return Nvfp4Tensor(codes, sf, ts, (B, H, N, d))
+
+
+def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
+                 nonfinite_flag: Optional[torch.Tensor] = None) -> Fp8Tensor:
+    B, H, N, d = _check_bf16(x)
+    lib = library()
+    codes = torch.empty((B, H, N, d), dtype=torch.uint8, device=x.device)
+    if granularity == "tile128":
+        g, scales = _lib.FP8_TILE128, torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
+    elif granularity == "channel":
+        g, scales = _lib.FP8_CHANNEL, torch.empty((B, H, d), dtype=torch.float32, device=x.device)
+    else:
+        raise ValueError("granularity must be 'tile128' or 'channel'")
+    st = lib.fpattn_quantize_fp8(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), g, codes.data_ptr(),
+                                 scales.data_ptr(), _ptr(nonfinite_flag), _stream())
+    _lib.check(st, "fpattn_quantize_fp8")
+    return Fp8Tensor(codes, scales, granularity, (B, H, N, d))
+
+
+@dataclasses.dataclass
+class StaPlan:
+    row_ptr: np.ndarray    # int32 [nblk + 1]
+    col_idx: np.ndarray    # int32 [nnz]
+    row_order: np.ndarray  # int32 [nblk], longest rows first
+
+    @property
+    def nblk(self) -> int:
+        return len(self.row_ptr) - 1
+
+    @property
+    def nnz(self) -> int:
+        return len(self.col_idx)
+
+    def to(self, device) -> "DeviceTileMask":
+        return DeviceTileMask(self.nblk, self.nnz,
+                              torch.from_numpy(self.row_ptr).to(device),
+                              torch.from_numpy(self.col_idx).to(device),
+                              torch.from_numpy(self.row_order).to(device))
+
+
+@dataclasses.dataclass
+class DeviceTileMask:
+    nblk: int
+    nnz: int
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    row_order: Optional[torch.Tensor]
+
+    def desc(self) -> _lib.TileMask:
+        return _lib.TileMask(self.nblk, self.nnz, self.row_ptr.data_ptr(), self.col_idx.data_ptr(),
+                             _ptr(self.row_order))
+
+
+def sta_plan(tile_grid: Sequence[int], tile: Sequence[int], window: Sequence[int]) -> StaPlan:
+    """Block CSR of the 3D sliding-tile pattern (host-only planner)."""
+    lib = library()
+    nblk, nnz = ctypes.c_int32(0), ctypes.c_int32(0)
+    args = [int(v) for v in (*tile_grid, *tile, *window)]
+    _lib.check(lib.fpattn_sta_plan(*args, None, None, None, 0, ctypes.byref(nblk), ctypes.byref(nnz)),
+               "fpattn_sta_plan")
+    row_ptr = np.zeros(nblk.value + 1, dtype=np.int32)
+    col_idx = np.zeros(max(nnz.value, 1), dtype=np.int32)
+    row_order = np.zeros(nblk.value, dtype=np.int32)
+    _lib.check(lib.fpattn_sta_plan(*args, row_ptr.ctypes.data, col_idx.ctypes.data, row_order.ctypes.data,
+                                   nnz.value, ctypes.byref(nblk), ctypes.byref(nnz)), "fpattn_sta_plan")
+    return StaPlan(row_ptr, col_idx[:nnz.value], row_order)
+
+
+def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
+                  softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, return_lse: bool = True):
+    """Fused attention on quantized operands.
+
+    q, k: both Nvfp4Tensor or both Fp8Tensor (tile128); v: Fp8Tensor (channel).
+    Returns (out bf16 [B,H,N,d], lse float32 [B,H,N] or None).
+    """
+    B, H, N, d = v.shape
+    lib = library()
+    if isinstance(q, Nvfp4Tensor) and isinstance(k, Nvfp4Tensor):
+        qd = _desc(q.codes, _lib.NVFP4, B, H, N, d)
+        kd = _desc(k.codes, _lib.NVFP4, B, H, N, d)
+        sc = _lib.Scales(q.tensor_scale.data_ptr(), k.tensor_scale.data_ptr(), v.scales.data_ptr(),
+                         q.block_sf.data_ptr(), k.block_sf.data_ptr(), 1.0 / 448.0, softmax_scale)
+    elif isinstance(q, Fp8Tensor) and isinstance(k, Fp8Tensor):
+        qd = _desc(q.codes, _lib.E4M3, B, H, N, d)
+        kd = _desc(k.codes, _lib.E4M3, B, H, N, d)
+        sc = _lib.Scales(q.scales.data_ptr(), k.scales.data_ptr(), v.scales.data_ptr(), None, None,
+                         1.0 / 448.0, softmax_scale)
+    else:
+        raise TypeError("q and k must both be Nvfp4Tensor or both Fp8Tensor")
+    vd = _desc(v.codes, _lib.E4M3, B, H, N, d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.codes.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.codes.device)
+    mask = ctypes.byref(tile_mask.desc()) if tile_mask is not None else None
+    st = lib.fpattn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(sc), mask,
+                        1 if causal else 0, out.data_ptr(), _ptr(lse), _stream())
+    _lib.check(st, "fpattn_fwd")
+    return out, lse
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: str = "nvfp4",
+              causal: bool = False, tile_mask: Optional[DeviceTileMask] = None, softmax_scale: float = 0.0,
+              return_lse: bool = True, device: Optional[torch.device] = None,
+              out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None):
+    """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
+
+    CUDA inputs stay where they are. Host inputs (ideally pinned) are copied
+    to ``device`` (default cuda:0) on the current stream, and the output (and
+    lse) are copied back to host memory: into ``out_host`` / ``lse_host`` when
+    given (pinned buffers the caller reuses), else into new pinned tensors.
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device(device or "cuda:0")
+        q = q.to(dev, non_blocking=True)
+        k = k.to(dev, non_blocking=True)
+        v = v.to(dev, non_blocking=True)
+    if qk_format == "nvfp4":
+        qq, kq = quantize_nvfp4(q), quantize_nvfp4(k)
+    elif qk_format == "fp8":
+        qq, kq = quantize_fp8(q, "tile128"), quantize_fp8(k, "tile128")
+    else:
+        raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
+    vq = quantize_fp8(v, "channel")
+    out, lse = attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
+                             return_lse=return_lse)
+    if host:
+        out_h = out_host if out_host is not None else torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_h.copy_(out, non_blocking=True)
+        lse_h = None
+        if lse is not None:
+            lse_h = lse_host if lse_host is not None else torch.empty(lse.shape, dtype=lse.dtype,
+                                                                      pin_memory=True)
+            lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return out_h, lse_h
+    return out, lse
+
+
+def device_error(clear: bool = True) -> int:
+    """Raw device error word (0 = no bounded wait expired). Synchronizes."""
+    code = ctypes.c_int32(0)
+    library().fpattn_device_error(_stream(), 1 if clear else 0, ctypes.byref(code))
+    return code.value

@@ -1,0 +1,220 @@
+// C ABI of the library: argument validation, dispatch to the kernels, the
+// host-side sliding-tile planner, status strings. See include/fpattn.h.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <numeric>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/fpattn.h"
+#include "fpattn_internal.h"
+
+namespace {
+
+using fpattn::AttnArgs;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fpattn_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return FPATTN_OK;
+  if (e == cudaErrorNotSupported) return FPATTN_ERR_UNSUPPORTED;
+  return FPATTN_ERR_CUDA;
+}
+
+// Common shape checks for a [B,H,N,d] tensor with the given dtype.
+fpattn_status check_tensor(const fpattn_tensor* t, int dtype) {
+  if (!t || !t->data) return FPATTN_ERR_INVALID_ARG;
+  if (t->dtype != dtype) return FPATTN_ERR_INVALID_ARG;
+  if (t->B <= 0 || t->H <= 0 || t->N <= 0 || t->d <= 0) return FPATTN_ERR_INVALID_ARG;
+  if (t->d != 64 && t->d != 128) return FPATTN_ERR_UNSUPPORTED;
+  // keep every index of the kernels inside 32-bit block / item counters
+  const long long bh = static_cast<long long>(t->B) * t->H;
+  const long long nblk = (t->N + 127) / 128;
+  if (bh * nblk > (1ll << 30) || t->N > (1 << 28)) return FPATTN_ERR_UNSUPPORTED;
+  if (!aligned16(t->data)) return FPATTN_ERR_ALIGNMENT;
+  return FPATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fpattn_nvfp4_sf_bytes(int32_t B, int32_t H, int32_t N, int32_t d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || d % 64 != 0) return 0;
+  return static_cast<size_t>(B) * H * ((N + 127) / 128) * (d / 64) * 512;
+}
+
+fpattn_status fpattn_quantize_nvfp4(const fpattn_tensor* x, const float* static_amax, uint8_t* codes,
+                                    uint8_t* block_sf, float* tensor_scale, int32_t* nonfinite_flag,
+                                    fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  if (!codes || !block_sf || !tensor_scale) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(block_sf) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+    return FPATTN_ERR_ALIGNMENT;
+  return from_cuda(fpattn::launch_quantize_nvfp4(x->data, x->B * x->H, x->N, x->d, static_amax, codes, block_sf,
+                                                 tensor_scale, nonfinite_flag,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fpattn_status fpattn_quantize_fp8(const fpattn_tensor* x, int32_t granularity, uint8_t* codes, float* scales,
+                                  int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  if (!codes || !scales) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FPATTN_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = x->B * x->H;
+  if (granularity == FPATTN_FP8_TILE128)
+    return from_cuda(fpattn::launch_quantize_fp8_tile(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, st));
+  if (granularity == FPATTN_FP8_CHANNEL)
+    return from_cuda(
+        fpattn::launch_quantize_fp8_channel(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, st));
+  return FPATTN_ERR_INVALID_ARG;
+}
+
+fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, int32_t th, int32_t tw, int32_t wt,
+                              int32_t wh, int32_t ww, int32_t* row_ptr, int32_t* col_idx, int32_t* row_order,
+                              size_t col_cap, int32_t* nblk_q_out, int32_t* nnz_out) {
+  if (nt <= 0 || nh <= 0 || nw <= 0 || tt <= 0 || th <= 0 || tw <= 0 || wt <= 0 || wh <= 0 || ww <= 0)
+    return FPATTN_ERR_INVALID_ARG;
+  if (!nblk_q_out || !nnz_out) return FPATTN_ERR_INVALID_ARG;
+  const long long vol = static_cast<long long>(tt) * th * tw;
+  const long long ntiles = static_cast<long long>(nt) * nh * nw;
+  if (vol % 128 != 0) return FPATTN_ERR_UNSUPPORTED;
+  const long long per = vol / 128;  // 128-token blocks per tile
+  if (ntiles * per > (1ll << 28)) return FPATTN_ERR_UNSUPPORTED;
+  const int ht = wt / 2, hh = wh / 2, hw = ww / 2;
+  // tiles in W(u) for tile u = (a, b, c): clipped ranges per axis
+  auto range = [](int u, int half, int n, int* lo, int* hi) {
+    *lo = std::max(0, u - half);
+    *hi = std::min(n - 1, u + half);
+  };
+  long long nnz = 0;
+  for (int a = 0; a < nt; ++a)
+    for (int b = 0; b < nh; ++b)
+      for (int c = 0; c < nw; ++c) {
+        int a0, a1, b0, b1, c0, c1;
+        range(a, ht, nt, &a0, &a1);
+        range(b, hh, nh, &b0, &b1);
+        range(c, hw, nw, &c0, &c1);
+        nnz += static_cast<long long>(a1 - a0 + 1) * (b1 - b0 + 1) * (c1 - c0 + 1) * per * per;
+      }
+  if (nnz > (1ll << 31) - 1) return FPATTN_ERR_UNSUPPORTED;
+  const int nblk = static_cast<int>(ntiles * per);
+  *nblk_q_out = nblk;
+  *nnz_out = static_cast<int32_t>(nnz);
+  if (!row_ptr || !col_idx || !row_order || col_cap < static_cast<size_t>(nnz)) return FPATTN_OK;
+  int32_t pos = 0;
+  int qb = 0;
+  row_ptr[0] = 0;
+  std::vector<int32_t> blocks;
+  for (int a = 0; a < nt; ++a)
+    for (int b = 0; b < nh; ++b)
+      for (int c = 0; c < nw; ++c) {
+        int a0, a1, b0, b1, c0, c1;
+        range(a, ht, nt, &a0, &a1);
+        range(b, hh, nh, &b0, &b1);
+        range(c, hw, nw, &c0, &c1);
+        // key blocks of W(u): tile indices in raster order are ascending, so
+        // the list comes out sorted
+        blocks.clear();
+        for (int x = a0; x <= a1; ++x)
+          for (int y = b0; y <= b1; ++y)
+            for (int z = c0; z <= c1; ++z) {
+              const long long v = (static_cast<long long>(x) * nh + y) * nw + z;
+              for (long long i = 0; i < per; ++i) blocks.push_back(static_cast<int32_t>(v * per + i));
+            }
+        // every 128-token query block of tile u gets the same list
+        for (long long i = 0; i < per; ++i) {
+          std::memcpy(col_idx + pos, blocks.data(), sizeof(int32_t) * blocks.size());
+          pos += static_cast<int32_t>(blocks.size());
+          row_ptr[qb + 1] = pos;
+          ++qb;
+        }
+      }
+  std::vector<int32_t> order(nblk);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    return (row_ptr[x + 1] - row_ptr[x]) > (row_ptr[y + 1] - row_ptr[y]);
+  });
+  std::memcpy(row_order, order.data(), sizeof(int32_t) * nblk);
+  return FPATTN_OK;
+}
+
+fpattn_status fpattn_fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                         const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask, int32_t causal,
+                         void* out, float* lse, fpattn_stream_t stream) {
+  if (!q || !k || !v || !scales || !out) return FPATTN_ERR_INVALID_ARG;
+  const int qk_dtype = q->dtype;
+  if (qk_dtype != FPATTN_NVFP4 && qk_dtype != FPATTN_E4M3) return FPATTN_ERR_UNSUPPORTED;
+  fpattn_status s;
+  if ((s = check_tensor(q, qk_dtype)) != FPATTN_OK) return s;
+  if ((s = check_tensor(k, qk_dtype)) != FPATTN_OK) return s;
+  if ((s = check_tensor(v, FPATTN_E4M3)) != FPATTN_OK) return s;
+  if (k->B != q->B || k->H != q->H || k->N != q->N || k->d != q->d || v->B != q->B || v->H != q->H ||
+      v->N != q->N || v->d != q->d)
+    return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FPATTN_ERR_ALIGNMENT;
+  if (!scales->q_scale || !scales->k_scale || !scales->v_scale) return FPATTN_ERR_INVALID_ARG;
+  const bool fp4 = qk_dtype == FPATTN_NVFP4;
+  if (fp4 && (!scales->q_block_sf || !scales->k_block_sf)) return FPATTN_ERR_INVALID_ARG;
+  if (fp4 && (!aligned16(scales->q_block_sf) || !aligned16(scales->k_block_sf))) return FPATTN_ERR_ALIGNMENT;
+  // P is stored in E4M3 at the fixed scale 1/448.
+  if (!(scales->p_scale > 0.f) || std::abs(scales->p_scale * 448.f - 1.f) > 1e-6f) return FPATTN_ERR_INVALID_ARG;
+  if (!(scales->softmax_scale >= 0.f) || scales->softmax_scale > 1e30f) return FPATTN_ERR_INVALID_ARG;
+  const int nblk = (q->N + 127) / 128;
+  if (tile_mask) {
+    if (tile_mask->nblk_q != nblk || !tile_mask->row_ptr || !tile_mask->col_idx || tile_mask->nnz < 0)
+      return FPATTN_ERR_INVALID_ARG;
+  }
+  AttnArgs a{};
+  a.q = q->data;
+  a.k = k->data;
+  a.v = v->data;
+  a.q_sf = fp4 ? scales->q_block_sf : nullptr;
+  a.k_sf = fp4 ? scales->k_block_sf : nullptr;
+  a.q_scale = scales->q_scale;
+  a.k_scale = scales->k_scale;
+  a.v_scale = scales->v_scale;
+  a.out = out;
+  a.lse = lse;
+  a.row_ptr = tile_mask ? tile_mask->row_ptr : nullptr;
+  a.col_idx = tile_mask ? tile_mask->col_idx : nullptr;
+  a.row_order = tile_mask ? tile_mask->row_order : nullptr;
+  a.B = q->B;
+  a.H = q->H;
+  a.N = q->N;
+  a.d = q->d;
+  a.qk_fp4 = fp4;
+  a.causal = causal != 0;
+  a.softmax_scale = scales->softmax_scale > 0.f ? scales->softmax_scale : 1.0f / std::sqrt(static_cast<float>(q->d));
+  return from_cuda(fpattn::launch_attn_fwd(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fpattn_status fpattn_device_error(fpattn_stream_t stream, int32_t clear, int32_t* code) {
+  int v = 0;
+  cudaError_t e = fpattn::read_device_error(reinterpret_cast<cudaStream_t>(stream), clear, &v);
+  if (code) *code = v;
+  if (e != cudaSuccess) return FPATTN_ERR_CUDA;
+  return v == 0 ? FPATTN_OK : FPATTN_ERR_TIMEOUT;
+}
+
+const char* fpattn_status_string(fpattn_status status) {
+  switch (status) {
+    case FPATTN_OK: return "ok";
+    case FPATTN_ERR_INVALID_ARG: return "invalid argument";
+    case FPATTN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case FPATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case FPATTN_ERR_CUDA: return "CUDA error";
+    case FPATTN_ERR_TIMEOUT: return "bounded device wait expired";
+  }
+  return "unknown status";
+}
+
+const char* fpattn_version(void) { return "fpattn 0.1 sm_100a"; }
+
+}  // extern "C"

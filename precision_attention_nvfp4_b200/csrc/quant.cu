@@ -1,0 +1,366 @@
+// Quantize kernels: bf16 [B,H,N,d] -> NVFP4 (packed E2M1 + E4M3 block scales
+// + FP32 tensor scale) or FP8 E4M3 (per-128-token-tile or per-channel
+// scales).
+//
+// NVFP4 follows the micro-scaling scheme of the Blackwell FP4 practice page
+// (section 1: values divided by a block scale and rounded to FP4, the scale
+// itself stored in FP8). FP8 follows the FPSAttention conversion formula
+// (section 2.1) and staged granularities (section 3.1).
+//
+// All kernels are bandwidth-bound streams: 16-byte loads per thread,
+// consecutive threads on consecutive 16-byte chunks, warp-shuffle reductions.
+// Every scale step is one correctly rounded fp32 operation (__fdiv_rn,
+// __fmul_rn: never contracted into an FMA) so the codes are bit-exact against
+// the CPU oracle, and the element conversions use the hardware's
+// round-to-nearest-even, saturating cvt instructions.
+#include <cfloat>
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "fpattn_internal.h"
+#include "sm100.cuh"
+
+namespace fpattn {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+  f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+  f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+  f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+// max |x| over 8 bf16 values; *bad |= non-finite seen.
+__device__ __forceinline__ float amax8(const uint4& v, bool* bad) {
+  float f[8];
+  unpack8(v, f);
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float a = fabsf(f[i]);
+    *bad |= !(a <= FLT_MAX);
+    m = fmaxf(m, a);
+  }
+  return m;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide max over kThreads threads; result valid in all threads.
+__device__ __forceinline__ float block_max(float v, float* red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int i = 1; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
+  __syncthreads();
+  return r;
+}
+
+// s = 448 / A (fp32, correctly rounded); 1 when A == 0.
+__device__ __forceinline__ float fp8_scale_from_amax(float a) { return a == 0.f ? 1.f : __fdiv_rn(448.f, a); }
+
+// 8 bf16 * s -> 8 E4M3 codes packed in a uint2 (element 0 in the low byte).
+__device__ __forceinline__ uint2 quant8_e4m3(const uint4& v, float s) {
+  float f[8];
+  unpack8(v, f);
+  uint2 r;
+  r.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[0], s), __fmul_rn(f[1], s))) |
+        (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[2], s), __fmul_rn(f[3], s))) << 16);
+  r.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[4], s), __fmul_rn(f[5], s))) |
+        (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[6], s), __fmul_rn(f[7], s))) << 16);
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// FP8, one scale per (b, h, 128-token tile). grid = (ceil(N/128), B*H).
+// The tile (<= 128 x 128 bf16 = 32 KiB) stays in registers between the amax
+// reduction and the conversion, so x is read from HBM exactly once.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restrict__ x, int N,
+                                                            uint2* __restrict__ codes, float* __restrict__ scales,
+                                                            int* nonfinite) {
+  constexpr int kChunksPerRow = D / 8;
+  constexpr int kChunks = 128 * kChunksPerRow;  // 16-byte chunks per full tile
+  constexpr int kPer = kChunks / kThreads;
+  __shared__ float red[kThreads / 32];
+  const int tile = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int rows = min(128, N - tile * 128);
+  const size_t base = (bh * N + static_cast<size_t>(tile) * 128) * kChunksPerRow;
+  uint4 v[kPer];
+  float m = 0.f;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = threadIdx.x + i * kThreads;
+    if (c / kChunksPerRow < rows) {
+      v[i] = x[base + c];
+      m = fmaxf(m, amax8(v[i], &bad));
+    }
+  }
+  if (bad && nonfinite) atomicExch(nonfinite, 1);
+  const float a = block_max(m, red);
+  const float s = fp8_scale_from_amax(a);
+  if (threadIdx.x == 0) scales[bh * gridDim.x + tile] = s;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = threadIdx.x + i * kThreads;
+    if (c / kChunksPerRow < rows) codes[base + c] = quant8_e4m3(v[i], s);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// FP8, one scale per (b, h, channel), amax over all N tokens.
+// Pass 1 reduces per-channel amax of a token chunk and folds it into
+// amax[bh, c] with an integer atomicMax (valid for non-negative floats).
+// Pass 2 converts with s_c = 448 / amax_c. Pass 3 turns amax into s in place.
+// grid = (ceil(N / kRowsPerCta), B*H).
+// ---------------------------------------------------------------------------
+constexpr int kRowsPerCta = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4* __restrict__ x, int N,
+                                                                    float* __restrict__ amax, int* nonfinite) {
+  constexpr int kCpr = D / 8;                 // chunks per row
+  constexpr int kRowsPerIter = kThreads / kCpr;
+  __shared__ float part[kRowsPerIter][D];
+  const size_t bh = blockIdx.y;
+  const int r0 = blockIdx.x * kRowsPerCta;
+  const int cg = threadIdx.x % kCpr;          // channel group of 8
+  const int rr = threadIdx.x / kCpr;
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = 0.f;
+  bool bad = false;
+  const int rend = min(N, r0 + kRowsPerCta);
+  for (int r = r0 + rr; r < rend; r += kRowsPerIter) {
+    const uint4 v = x[(bh * N + r) * kCpr + cg];
+    float f[8];
+    unpack8(v, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float a = fabsf(f[i]);
+      bad |= !(a <= FLT_MAX);
+      m[i] = fmaxf(m[i], a);
+    }
+  }
+  if (bad && nonfinite) atomicExch(nonfinite, 1);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[rr][cg * 8 + i] = m[i];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += kThreads) {
+    float a = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < kRowsPerIter; ++j) a = fmaxf(a, part[j][c]);
+    atomicMax(reinterpret_cast<int*>(amax) + bh * D + c, __float_as_int(a));
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4* __restrict__ x, int N,
+                                                                     const float* __restrict__ amax,
+                                                                     uint2* __restrict__ codes) {
+  constexpr int kCpr = D / 8;
+  constexpr int kRowsPerIter = kThreads / kCpr;
+  const size_t bh = blockIdx.y;
+  const int r0 = blockIdx.x * kRowsPerCta;
+  const int cg = threadIdx.x % kCpr;
+  const int rr = threadIdx.x / kCpr;
+  float s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s[i] = fp8_scale_from_amax(amax[bh * D + cg * 8 + i]);
+  const int rend = min(N, r0 + kRowsPerCta);
+  for (int r = r0 + rr; r < rend; r += kRowsPerIter) {
+    const size_t idx = (bh * N + r) * kCpr + cg;
+    const uint4 v = x[idx];
+    float f[8];
+    unpack8(v, f);
+    uint2 o;
+    o.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[0], s[0]), __fmul_rn(f[1], s[1]))) |
+          (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[2], s[2]), __fmul_rn(f[3], s[3]))) << 16);
+    o.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[4], s[4]), __fmul_rn(f[5], s[5]))) |
+          (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[6], s[6]), __fmul_rn(f[7], s[7]))) << 16);
+    codes[idx] = o;
+  }
+}
+
+__global__ void fp8_channel_finalize_kernel(float* __restrict__ s, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) s[i] = fp8_scale_from_amax(s[i]);
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4.
+// Pass 1 (dynamic only): tensor amax -> *amax_out via integer atomicMax.
+// Pass 2: one thread per (row, group of 64 elements = four 16-element blocks):
+//   s_t = A_t / 2688 (1 if A_t == 0)
+//   sb  = E4M3(A_b / (6 * s_t)), den = dec(sb) * s_t, inv = 1 / den,
+//   code = E2M1(x * inv)   (all zero when den == 0 or inv is not finite)
+//   32 code bytes + 4 scale bytes (one aligned 32-bit store into the
+//   tensor-core scale layout). Threads past N write the zero scale padding.
+// Pass 3: *tensor_scale = s_t.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __restrict__ x, size_t nchunks,
+                                                               float* __restrict__ amax_out, int* nonfinite) {
+  __shared__ float red[kThreads / 32];
+  float m = 0.f;
+  bool bad = false;
+  for (size_t c = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x; c < nchunks;
+       c += static_cast<size_t>(gridDim.x) * kThreads)
+    m = fmaxf(m, amax8(x[c], &bad));
+  if (bad && nonfinite) atomicExch(nonfinite, 1);
+  m = block_max(m, red);
+  if (threadIdx.x == 0) atomicMax(reinterpret_cast<int*>(amax_out), __float_as_int(m));
+}
+
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 2688.f);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __restrict__ x, int N, int nblk,
+                                                               const float* __restrict__ amax_ptr,
+                                                               uint4* __restrict__ codes,
+                                                               uint32_t* __restrict__ sf, size_t total_groups) {
+  constexpr int kGroups = D / 64;  // 64-element groups per row
+  const size_t g = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x;
+  if (g >= total_groups) return;
+  // g enumerates (bh, padded row, group) with rows padded to 128 per (b, h).
+  const int grp = static_cast<int>(g % kGroups);
+  const size_t prow = g / kGroups;                // padded row over all (b, h)
+  const size_t rows_pad = static_cast<size_t>(nblk) * 128;
+  const size_t bh = prow / rows_pad;
+  const int r = static_cast<int>(prow % rows_pad);
+  // scale-layout offset (in 32-bit words): [bh][nb][grp] x 512 bytes, then
+  // byte 16*i + 4*j for row 32*j + i of the 128-row block.
+  const int nb = r >> 7, rr = r & 127;
+  const size_t sf_word = ((bh * nblk + nb) * kGroups + grp) * 128 + (rr & 31) * 4 + (rr >> 5);
+  if (r >= N) {
+    sf[sf_word] = 0u;
+    return;
+  }
+  const float s_t = nvfp4_tensor_scale(*amax_ptr);
+  const float six_st = __fmul_rn(6.f, s_t);
+  const size_t row = bh * N + r;
+  const uint4* src = x + (row * D + grp * 64) / 8;
+  uint4* dst = codes + (row * D + grp * 64) / 32;
+  uint32_t sfw = 0;
+  uint32_t out[8];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {  // four 16-element blocks
+    float f[16];
+    unpack8(src[2 * b], f);
+    unpack8(src[2 * b + 1], f + 8);
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(f[i]));
+    const uint32_t sb = cvt_e4m3x2(__fdiv_rn(a, six_st), 0.f) & 0xFFu;
+    const float den = __fmul_rn(e4m3_to_float(sb), s_t);
+    const float inv = __fdiv_rn(1.f, den);
+    const bool usable = (den != 0.f) && (fabsf(inv) <= FLT_MAX);
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = usable ? __fmul_rn(f[i], inv) : 0.f;
+    out[2 * b] = usable ? cvt_e2m1x8(y) : 0u;
+    out[2 * b + 1] = usable ? cvt_e2m1x8(y + 8) : 0u;
+    sfw |= sb << (8 * b);
+  }
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  sf[sf_word] = sfw;
+}
+
+__global__ void nvfp4_finalize_kernel(const float* __restrict__ amax_ptr, float* __restrict__ tensor_scale) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) *tensor_scale = nvfp4_tensor_scale(*amax_ptr);
+}
+
+inline int num_sms() {
+  static int sms = [] {
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+  }();
+  return sms;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Host launchers (arguments already validated by the C ABI layer).
+// ---------------------------------------------------------------------------
+cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
+                                     int* nonfinite, cudaStream_t st) {
+  dim3 grid((N + 127) / 128, BH);
+  if (d == 128)
+    fp8_tile_kernel<128><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(x), N,
+                                                    reinterpret_cast<uint2*>(codes), scales, nonfinite);
+  else
+    fp8_tile_kernel<64><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(x), N,
+                                                   reinterpret_cast<uint2*>(codes), scales, nonfinite);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
+                                        int* nonfinite, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(scales, 0, sizeof(float) * BH * d, st);
+  if (e != cudaSuccess) return e;
+  dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, BH);
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint2* cv = reinterpret_cast<uint2*>(codes);
+  if (d == 128) {
+    fp8_channel_amax_kernel<128><<<grid, kThreads, 0, st>>>(xv, N, scales, nonfinite);
+    fp8_channel_quant_kernel<128><<<grid, kThreads, 0, st>>>(xv, N, scales, cv);
+  } else {
+    fp8_channel_amax_kernel<64><<<grid, kThreads, 0, st>>>(xv, N, scales, nonfinite);
+    fp8_channel_quant_kernel<64><<<grid, kThreads, 0, st>>>(xv, N, scales, cv);
+  }
+  const int n = BH * d;
+  fp8_channel_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(scales, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const float* static_amax,
+                                  uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
+                                  cudaStream_t st) {
+  const float* amax_ptr = static_amax;
+  if (!static_amax) {
+    // tensor_scale doubles as the amax accumulator until pass 3 overwrites it.
+    cudaError_t e = cudaMemsetAsync(tensor_scale, 0, sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
+    const int blocks = num_sms() * 8;
+    tensor_amax_kernel<<<blocks, kThreads, 0, st>>>(static_cast<const uint4*>(x), nchunks, tensor_scale,
+                                                    nonfinite);
+    amax_ptr = tensor_scale;
+  }
+  const int nblk = (N + 127) / 128;
+  const size_t groups = static_cast<size_t>(BH) * nblk * 128 * (d / 64);
+  const unsigned blocks = static_cast<unsigned>((groups + kThreads - 1) / kThreads);
+  if (d == 128)
+    nvfp4_quant_kernel<128><<<blocks, kThreads, 0, st>>>(static_cast<const uint4*>(x), N, nblk, amax_ptr,
+                                                         reinterpret_cast<uint4*>(codes),
+                                                         reinterpret_cast<uint32_t*>(block_sf), groups);
+  else
+    nvfp4_quant_kernel<64><<<blocks, kThreads, 0, st>>>(static_cast<const uint4*>(x), N, nblk, amax_ptr,
+                                                        reinterpret_cast<uint4*>(codes),
+                                                        reinterpret_cast<uint32_t*>(block_sf), groups);
+  nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax_ptr, tensor_scale);
+  return cudaGetLastError();
+}
+
+}  // namespace fpattn
