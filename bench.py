@@ -176,6 +176,26 @@ def run_reference(args, w):
     return 0
 
 
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 if absent)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(per_rank_flops: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOPS: every rank runs one batch (weak scaling), time = max over ranks."""
+    return world * per_rank_flops / (ms_per_step * 1e-3) / 1e12
+
+
 def config_dict(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "qk": w.qk_format, "pv": "e4m3", "sparse": w.sparse,
@@ -185,8 +205,8 @@ def config_dict(w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llm_prefill_causal")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -197,9 +217,7 @@ def main():
         return run_reference(args, w)
 
     import precision_attention_nvfp4_b200 as fp
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -211,12 +229,8 @@ def main():
         if dist is not None:
             dist.barrier(device_ids=[local])
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x: float) -> float:
+        return max_over_ranks(dist, x, "cuda")
 
     # weak scaling: every rank runs one full batch of the workload
     q_h, k_h, v_h = workloads.make_qkv(w)
@@ -260,16 +274,16 @@ def main():
     barrier()
     clk = clocks.stop()
     ms_total = start.elapsed_time(end)
-    ms_total = max_over_ranks(ms_total)
+    ms_total = rank_max(ms_total)
     attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_events]))
-    attn_ms = max_over_ranks(attn_ms)
+    attn_ms = rank_max(attn_ms)
     err = fp.device_error()
 
     flops = w.dense_flops()
     pairs = executed_block_pairs(w)
     exec_flops = 4.0 * 128 * 128 * w.d * pairs * w.B * w.H
     ms_step = ms_total / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = aggregate_value(flops, world, ms_step)
     peaks, peak_src = load_peaks()
     bf16 = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
@@ -295,7 +309,7 @@ def main():
                          lse_host=lse_h)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
+        e_ms = rank_max(e0.elapsed_time(e1) / args.e2e_steps)
         h2d = 3 * q_h.numel() * 2
         d2h = out_h.numel() * 2 + lse_h.numel() * 4
         e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,

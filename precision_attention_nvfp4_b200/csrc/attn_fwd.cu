@@ -68,6 +68,11 @@ struct Cfg {
   static constexpr uint32_t kVSwz = D == 128 ? 2u : 4u;
   static constexpr uint32_t kVSbo = 8 * D;
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
+#ifndef FPATTN_POLY_PAIRS
+  static constexpr int kPolyPairs = 12;                   // of 32 exp2 pairs per thread and tile
+#else
+  static constexpr int kPolyPairs = FPATTN_POLY_PAIRS;
+#endif
   static constexpr uint32_t kColO = 256;
   static constexpr uint32_t kColSFQ = 256 + D;
   static constexpr uint32_t kSFCols = 4 * (D / 64);
@@ -142,6 +147,54 @@ __device__ __forceinline__ KList key_list(const Params& p, int qb) {
 
 __device__ __forceinline__ int key_block(const Params& p, const KList& L, int j) {
   return p.sparse ? p.col_idx[L.begin + j] : j;
+}
+
+// Row max of 64 scores: a tree of three-input max instructions (depth 5).
+__device__ __forceinline__ float row_max64(const float (&s)[64]) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmax3(s[8 * k], s[8 * k + 1], s[8 * k + 2]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[8 * k + 3], s[8 * k + 4]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[8 * k + 5], s[8 * k + 6]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[8 * k + 7]);
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// P = 2^(c*s + nbias) for 64 scores (nbias folds -m and log2 448), packed to
+// E4M3 four per word (key 4j+b in byte b of pk[j]); returns the sum of the
+// unquantized P. kPoly of the 32 pairs take the FMA-pipe polynomial exp2, the
+// rest the MUFU ex2, spread evenly so both pipes stay busy.
+template <int kPoly>
+__device__ __forceinline__ float exp_pack64(const float (&s)[64], float c, float nbias, uint32_t (&pk)[16]) {
+  const uint64_t c2 = f2_pack(c, c), nb2 = f2_pack(nbias, nbias);
+  uint64_t acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = 0ull;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint64_t x = f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nb2);
+    uint64_t p;
+    if (((i * kPoly) % 32) < kPoly) {
+      p = exp2_poly2(x);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      p = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    }
+    acc[i & 3] = f2_add(acc[i & 3], p);
+    float p0, p1;
+    f2_unpack(p, p0, p1);
+    const uint32_t h = cvt_e4m3x2(p0, p1);
+    if (i & 1) pk[i >> 1] |= h << 16;
+    else pk[i >> 1] = h;
+  }
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float lo, hi;
+  f2_unpack(t, lo, hi);
+  return lo + hi;
 }
 
 // AND of `v` over the 256 softmax threads; doubles as their shared barrier.
@@ -381,8 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
               if ((p.causal && key > qrow) || key >= p.N) s[i] = -INFINITY;
             }
           }
-#pragma unroll
-          for (int i = 0; i < 64; ++i) pmax = fmaxf(pmax, s[i]);
+          pmax = row_max64(s);
           xmax[(buf * 2 + h) * 128 + row] = pmax;
         }
         ok = softmax_sync_and(mine && ok);
@@ -394,16 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const float alpha = (m == m_use) ? 1.f : ex2_approx(m - m_use);
         const float nbias = kLog2_448 - m_use;
         uint32_t pk[16];
-        float psum = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(s[4 * i + 0], c, nbias));
-          const float p1 = ex2_approx(fmaf(s[4 * i + 1], c, nbias));
-          const float p2 = ex2_approx(fmaf(s[4 * i + 2], c, nbias));
-          const float p3 = ex2_approx(fmaf(s[4 * i + 3], c, nbias));
-          psum += (p0 + p1) + (p2 + p3);
-          pk[i] = static_cast<uint32_t>(cvt_e4m3x2(p0, p1)) | (static_cast<uint32_t>(cvt_e4m3x2(p2, p3)) << 16);
-        }
+        const float psum = exp_pack64<C::kPolyPairs>(s, c, nbias, pk);
         l = l * alpha + psum;
         m = m_new;
         // O correction: rows whose max moved scale O by alpha once PV of the

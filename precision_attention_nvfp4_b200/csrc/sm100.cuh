@@ -300,6 +300,68 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
   return __half2float(h);
 }
 
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs (f32x2 arithmetic, sm_100+): two lanes per instruction.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three floats in one instruction (sm_100+)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no MUFU), for x <= 128.
+// Range reduction x = j + f with j = round-to-nearest(x) (via the 1.5*2^23
+// rounding constant) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients were fitted for this library (iteratively reweighted least
+// squares at 400 Chebyshev nodes, i.e. a discrete minimax fit of the relative
+// error; max relative error 7.5e-5 in fp32); 2^j by adding j to the exponent
+// field. x is clamped at -125 first so the exponent cannot underflow: 2^-125 is
+// far below anything that reaches an E4M3 probability or the row sum.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t kRound = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(x, kRound);      // j sits in the low mantissa bits
+  const uint64_t f = f2_sub(x, f2_sub(t, kRound));
+  uint64_t p = f2_fma(f, f2_pack(0.05517156794667244f, 0.05517156794667244f),
+                      f2_pack(0.2426111102104187f, 0.2426111102104187f));
+  p = f2_fma(p, f, f2_pack(0.6932610273361206f, 0.6932610273361206f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  uint32_t plo, phi, tlo, thi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(p));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(tlo), "=r"(thi) : "l"(t));
+  plo += tlo << 23;
+  phi += thi << 23;
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(plo), "r"(phi));
+  return r;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -10,6 +10,7 @@ sum near 1e-5 and the fp32 scores carry about 1e-6 relative error, so
 """
 from __future__ import annotations
 
+import functools
 import math
 
 import numpy as np
@@ -20,6 +21,13 @@ from oracle import codec, quant
 
 ATOL_FRAC = 2e-2
 REL_L2 = 5e-3
+
+
+@functools.lru_cache(maxsize=2)
+def workload_qkv(name: str):
+    """Full-size seeded inputs of a named workload, generated once per session."""
+    import workloads
+    return workloads.make_qkv(workloads.get(name))
 
 
 def f32(x: torch.Tensor) -> np.ndarray:

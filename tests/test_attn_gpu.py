@@ -31,7 +31,7 @@ def _run_gpu(q, k, v, fmt, causal=False, tile_mask=None):
 
 
 def _check_case(q, k, v, fmt, causal=False, key_blocks=None, tile_mask=None, qblocks=None, heads=None,
-                min_cos=None):
+                min_cos=None, outliers=False):
     B, H, N, d = q.shape
     out, lse = _run_gpu(q, k, v, fmt, causal, tile_mask)
     out = out.reshape(B * H, N, d)
@@ -46,19 +46,29 @@ def _check_case(q, k, v, fmt, causal=False, key_blocks=None, tile_mask=None, qbl
                                        key_blocks=key_blocks)
         parity.assert_close(res, f"{fmt} bh={bh}")
         if min_cos is not None:
+            # Cosine against unquantized fp64 attention. With x20 outlier
+            # channels the scores are so peaked that quantizing Q/K moves the
+            # argmax of many rows, for the oracle as much as for the kernel, so
+            # there the kernel must track the oracle's own cosine instead.
             qe, ke, ve = (t.reshape(B * H, N, d)[bh].double().numpy() for t in (q, k, v))
             cos = parity.cosine_vs_exact(out[bh][rows], qe, ke, ve, rows, causal=causal, key_blocks=key_blocks)
-            assert cos >= min_cos, f"cosine vs exact {cos}"
+            if outliers:
+                ref, _ = parity.oatt.attention_rows(qh[i], kh[i], vh[i], rows, causal=causal, key_blocks=key_blocks)
+                cos_oracle = parity.cosine_vs_exact(ref, qe, ke, ve, rows, causal=causal, key_blocks=key_blocks)
+                assert cos >= cos_oracle - 0.01, f"cosine vs exact {cos} (oracle {cos_oracle})"
+            else:
+                assert cos >= min_cos, f"cosine vs exact {cos}"
 
 
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [128, 300, 1000])
-def test_reduced(fmt, d, causal, N):
-    w = workloads.Workload("t", B=1, H=2, N=N, d=d, causal=causal, qk_format=fmt, seed=N + d, outliers=True)
+@pytest.mark.parametrize("outliers", [False, True])
+def test_reduced(fmt, d, causal, N, outliers):
+    w = workloads.Workload("t", B=1, H=2, N=N, d=d, causal=causal, qk_format=fmt, seed=N + d, outliers=outliers)
     q, k, v = workloads.make_qkv(w)
-    _check_case(q, k, v, fmt, causal=causal, min_cos=0.99 if fmt == "fp8" else 0.98)
+    _check_case(q, k, v, fmt, causal=causal, min_cos=0.99 if fmt == "fp8" else 0.98, outliers=outliers)
 
 
 def test_tiny_nvfp4_workload():
@@ -127,7 +137,7 @@ def test_empty_mask_rows():
 # ---------------------------------------------------------------- full size
 def _full(name, qblocks_fn, heads_fn, fmt=None, tile_mask=None, key_blocks=None):
     w = workloads.get(name)
-    q, k, v = workloads.make_qkv(w)
+    q, k, v = parity.workload_qkv(name)
     B, H, N, d = q.shape
     nblk = (N + 127) // 128
     _check_case(q, k, v, fmt or w.qk_format, causal=w.causal, key_blocks=key_blocks, tile_mask=tile_mask,

@@ -11,6 +11,7 @@ import torch
 import precision_attention_nvfp4_b200 as fp
 import workloads
 from oracle import codec, quant
+import parity
 
 pytestmark = pytest.mark.gpu
 
@@ -138,7 +139,7 @@ def test_workload_nvfp4_full_tensor(name):
     """Full-size workload tensor on the GPU; every code and scale compared on a
     sample of heads (the tensor scale is over the whole tensor)."""
     w = workloads.get(name)
-    q, k, v = workloads.make_qkv(w)
+    q, k, v = parity.workload_qkv(name)
     B, H, N, d = q.shape
     for x in (q, k):
         r = fp.quantize_nvfp4(x.cuda())
@@ -160,7 +161,7 @@ def test_workload_fp8_heads(name):
     """Video workload shapes (N = 75600 with an 80-token tail, N = 69120) on a
     subset of heads: per-tile Q/K and per-channel V, bit-exact."""
     w = workloads.get(name)
-    q, k, v = workloads.make_qkv(w)
+    q, k, v = parity.workload_qkv(name)
     sub = slice(0, 3)
     _check_fp8(q[:, sub].contiguous(), "tile128")
     _check_fp8(v[:, sub].contiguous(), "channel")
