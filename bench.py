@@ -48,6 +48,28 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def profiled_traffic():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, or None when the kernel sources changed since that capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                a, b = line.split(":", 1)
+                kv[a.strip()] = b.strip()
+    h = hashlib.sha256()
+    for src in ("attn_fwd.cu", "sm100.cuh"):
+        with open(os.path.join(ROOT, "precision_attention_nvfp4_b200", "csrc", src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != kv.get("source_sha256_16"):
+        return None
+    return float(kv["traffic_bytes"])
+
+
 def executed_block_pairs(w: workloads.Workload) -> int:
     """128x128 (query block, key block) pairs the kernel computes per head."""
     nblk = (w.N + 127) // 128
@@ -336,7 +358,8 @@ def main():
             "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,
             "quant_ms": quant_ms, "quant_gbs": quant_gbs, "quant_frac_hbm": quant_gbs / peaks["hbm_gbs"],
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": attn_tflops / peak, "traffic": None,
+                         "frac": attn_tflops / peak,
+                         "traffic": profiled_traffic() if w.name == "llm_prefill_causal" else None,
                          "peak_source": f"{peak_src} bf16 sustained {bf16} x nominal fp8 2x / fp4 4x; "
                                         f"{'harmonic mix of fp4 QK and fp8 PV' if w.qk_format == 'nvfp4' else 'fp8'}"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,

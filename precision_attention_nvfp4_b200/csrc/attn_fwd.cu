@@ -10,23 +10,33 @@
 // The online softmax follows the FlashAttention tiling the pages describe
 // (FlashAttention-4 article: S and P kept on chip, O accumulated in tensor
 // memory, asynchronous pipeline between loads, MMA and softmax). The running
-// row max is always the exact max; the O/l rescale is skipped for rows whose
-// max did not change (a warp skips the tensor-memory round trip when none of
-// its rows changed), which is exact.
+// row max is always the exact max of the keys seen so far; O and the row sum
+// are rescaled only for rows whose max moved (a warp skips the tensor-memory
+// round trip when none of its rows moved), which is exact.
 //
-// CTA organisation (persistent, one CTA per SM, 384 threads):
-//   warp 0       TMA producer: Q once per work item, K/V tiles into a
-//                4-stage shared-memory ring (plus NVFP4 block scales)
-//   warp 1       tensor-memory allocator and single-thread MMA issuer
-//   warps 2-3    idle
-//   warps 4-11   two softmax warpgroups; warpgroup h owns keys 64h..64h+63 of
-//                every 128-key S tile and output columns h*d/2..(h+1)*d/2-1;
-//                thread (warp w, lane t) owns query row 32*(w%4)+t. They
-//                exchange row maxima through shared memory once per tile.
+// CTA organisation (persistent, one CTA per SM, 512 threads):
+//   warp 0        TMA producer: Q once per work item, K/V tiles into a
+//                 4-stage shared-memory ring (plus NVFP4 block scales)
+//   warp 1        tensor-memory allocator; issues O += P V (one thread)
+//   warp 2        issues S = Q K^T (one thread)
+//   warp 3        idle
+//   warps 4-7     softmax warpgroup 0: key blocks with even global index
+//   warps 8-11    softmax warpgroup 1: key blocks with odd global index
+//   warps 12-15   O rescale (correction) and epilogue
+// Thread (warp quarter q, lane t) of a softmax warpgroup owns query row
+// 32q + t and all 128 keys of its block, read from TMEM in 32-column chunks
+// twice (row max, then exponentials). The two softmax warpgroups alternate
+// blocks, so one group's exponentials (MUFU and FMA pipes) overlap the
+// other's tensor-memory loads and waits; the only value they exchange is the
+// running row max, passed per warp pair through shared memory and an
+// mbarrier. Each keeps its own row sum relative to the last max it used; the
+// epilogue combines them.
 // Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32
-// 128x128), P (E4M3) written over the first 16 columns of each 64-column half
-// of its S buffer, O at column 256 (d fp32 columns), NVFP4 scale vectors of Q
-// and of two K tiles after O.
+// 128x128, buffer = block parity), O at column 256 (d fp32 columns), P double
+// buffer (E4M3, 32 columns each) at 384, NVFP4 scale vectors of Q and of two
+// K tiles at 448. S and P having their own buffers lets the S of a block be
+// issued as soon as its buffer's previous tile has been read, independently
+// of the PV of that tile; the two MMA kinds are issued by separate threads.
 // Work items are (batch*head, 128-query block); causal runs schedule the
 // longest query blocks first, tile-mask runs follow the mask's row order.
 #include <cfloat>
@@ -46,7 +56,7 @@ __device__ int g_error_word = 0;
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kStages = 4;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
@@ -54,7 +64,8 @@ constexpr float kLn2 = 0.6931471805599453f;
 // error codes recorded on a wait timeout (which wait gave up)
 enum : int {
   kErrQEmpty = 0x101, kErrKvEmpty = 0x102, kErrQFull = 0x201, kErrKFull = 0x202, kErrVFull = 0x203,
-  kErrPFull = 0x204, kErrSFull = 0x301, kErrODone = 0x302, kErrDrain = 0x401
+  kErrPFull = 0x204, kErrOReady = 0x205, kErrSFull = 0x301, kErrMax = 0x303, kErrFin = 0x304,
+  kErrAlpha = 0x305, kErrSFree = 0x306, kErrPFree = 0x307, kErrODone = 0x302, kErrDrain = 0x401
 };
 
 template <int D, bool FP4>
@@ -68,13 +79,11 @@ struct Cfg {
   static constexpr uint32_t kVSwz = D == 128 ? 2u : 4u;
   static constexpr uint32_t kVSbo = 8 * D;
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
-#ifndef FPATTN_POLY_PAIRS
-  static constexpr int kPolyPairs = 12;                   // of 32 exp2 pairs per thread and tile
-#else
-  static constexpr int kPolyPairs = FPATTN_POLY_PAIRS;
-#endif
-  static constexpr uint32_t kColO = 256;
-  static constexpr uint32_t kColSFQ = 256 + D;
+  static constexpr int kPolyPairs = 4;                    // of 16 exp2 pairs per 32-score chunk
+  static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
+  static constexpr int kPBufs = 3;                        // P buffers: 32 columns each (128 E4M3 keys)
+  static constexpr uint32_t kColP = 384;
+  static constexpr uint32_t kColSFQ = kColP + 32 * kPBufs;
   static constexpr uint32_t kSFCols = 4 * (D / 64);
   static constexpr uint32_t kColSFK = kColSFQ + kSFCols;  // + buf * kSFCols
   // shared memory layout (offsets from a 1024-byte aligned base)
@@ -84,11 +93,17 @@ struct Cfg {
   static constexpr int kOffSFQ = kOffV + kStages * kVTile;
   static constexpr int kOffSFK = kOffSFQ + kSF;
   static constexpr int kOffBar = kOffSFK + kStages * kSF;
-  static constexpr int kNumBars = 2 + 3 * kStages + 2 + 2 + 2;
+  // mbarrier indices (one chain, so the pointers and the count cannot drift)
+  static constexpr int kBarQFull = 0, kBarQEmpty = 1, kBarKFull = 2;
+  static constexpr int kBarVFull = kBarKFull + kStages, kBarKVEmpty = kBarVFull + kStages;
+  static constexpr int kBarSFull = kBarKVEmpty + kStages, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2;
+  static constexpr int kBarPFree = kBarPFull + kPBufs, kBarOReady = kBarPFree + kPBufs, kBarODone = kBarOReady + kStages;
+  static constexpr int kBarDrain = kBarODone + kStages, kBarM = kBarDrain + 2, kBarA = kBarM + 8;
+  static constexpr int kBarFin = kBarA + 4 * kStages, kBarFinFree = kBarFin + 2;
+  static constexpr int kNumBars = kBarFinFree + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kOffXMax = (kOffMisc + 64 + 15) & ~15;   // float[2][2][128]
-  static constexpr int kOffXL = kOffXMax + 2 * 2 * 128 * 4;     // float[2][2][128]
-  static constexpr int kBytes = kOffXL + 2 * 2 * 128 * 4;
+  static constexpr int kOffX = (kOffMisc + 64 + 15) & ~15;      // running max, rescale, per-item (l, m)
+  static constexpr int kBytes = kOffX + (2 * 128 + kStages * 128 + 2 * 2 * 2 * 128) * 4;
   // Request at least this much so that a single CTA fits per SM (it takes
   // all 512 tensor-memory columns).
   static constexpr int kSmemRequest = (kBytes + 1024 > 120 * 1024 ? kBytes + 1024 : 120 * 1024);
@@ -116,6 +131,14 @@ struct __align__(64) Params {
 struct KList {
   int begin, count;
 };
+
+// Work item of this CTA in scheduling round r: a snake over the CTAs (forward
+// on even rounds, backward on odd ones) so that with items sorted longest
+// first every CTA gets a near-equal share.
+__device__ __forceinline__ int sched_item(int r) {
+  return r * gridDim.x + ((r & 1) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                                  : static_cast<int>(blockIdx.x));
+}
 
 __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, int& qb) {
   if (p.sparse) {
@@ -149,66 +172,57 @@ __device__ __forceinline__ int key_block(const Params& p, const KList& L, int j)
   return p.sparse ? p.col_idx[L.begin + j] : j;
 }
 
-// Row max of 64 scores: a tree of three-input max instructions (depth 5).
-__device__ __forceinline__ float row_max64(const float (&s)[64]) {
-  float a[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmax3(s[8 * k], s[8 * k + 1], s[8 * k + 2]);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[8 * k + 3], s[8 * k + 4]);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[8 * k + 5], s[8 * k + 6]);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[8 * k + 7]);
-  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-}
-
-// P = 2^(c*s + nbias) for 64 scores (nbias folds -m and log2 448), packed to
-// E4M3 four per word (key 4j+b in byte b of pk[j]); returns the sum of the
-// unquantized P. kPoly of the 32 pairs take the FMA-pipe polynomial exp2, the
-// rest the MUFU ex2, spread evenly so both pipes stay busy.
-template <int kPoly>
-__device__ __forceinline__ float exp_pack64(const float (&s)[64], float c, float nbias, uint32_t (&pk)[16]) {
-  const uint64_t c2 = f2_pack(c, c), nb2 = f2_pack(nbias, nbias);
-  uint64_t acc[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = 0ull;
+// Masks the scores of one 32-key chunk (keys key0..key0+31) that fall past
+// the sequence end or, on the causal diagonal, after the query row.
+__device__ __forceinline__ void mask_chunk(uint32_t (&r)[32], int key0, int qrow, bool causal_diag, int N) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    const uint64_t x = f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nb2);
-    uint64_t p;
-    if (((i * kPoly) % 32) < kPoly) {
-      p = exp2_poly2(x);
+    const int key = key0 + i;
+    if ((causal_diag && key > qrow) || key >= N) r[i] = 0xff800000u;  // -inf
+  }
+}
+
+// Max of 32 scores: a tree of three-input max instructions.
+__device__ __forceinline__ float max32(const uint32_t (&r)[32], float m) {
+  float a[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    a[k] = fmax3(fmax3(__uint_as_float(r[8 * k]), __uint_as_float(r[8 * k + 1]), __uint_as_float(r[8 * k + 2])),
+                 fmax3(__uint_as_float(r[8 * k + 3]), __uint_as_float(r[8 * k + 4]), __uint_as_float(r[8 * k + 5])),
+                 fmaxf(__uint_as_float(r[8 * k + 6]), __uint_as_float(r[8 * k + 7])));
+  return fmax3(fmax3(a[0], a[1], m), a[2], a[3]);
+}
+
+// P = 2^(c*s + nbias) for 32 scores (nbias folds -m and log2 448), packed to
+// E4M3 four per word (key 4j+b in byte b of pk[j]); returns the sum of the
+// unquantized P. kPoly of the 16 pairs take the FMA-pipe polynomial exp2, the
+// rest the MUFU ex2, spread evenly so both pipes stay busy.
+template <int kPoly>
+__device__ __forceinline__ float exp_pack32(const uint32_t (&r)[32], float c, float nbias, uint32_t (&pk)[8]) {
+  const uint64_t c2 = f2_pack(c, c), nb2 = f2_pack(nbias, nbias);
+  uint64_t acc0 = 0ull, acc1 = 0ull;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nb2);
+    uint64_t pr;
+    if (((i * kPoly) % 16) < kPoly) {
+      pr = exp2_poly2(x);
     } else {
       float x0, x1;
       f2_unpack(x, x0, x1);
-      p = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      pr = f2_pack(ex2_approx(x0), ex2_approx(x1));
     }
-    acc[i & 3] = f2_add(acc[i & 3], p);
+    if (i & 1) acc1 = f2_add(acc1, pr);
+    else acc0 = f2_add(acc0, pr);
     float p0, p1;
-    f2_unpack(p, p0, p1);
+    f2_unpack(pr, p0, p1);
     const uint32_t h = cvt_e4m3x2(p0, p1);
     if (i & 1) pk[i >> 1] |= h << 16;
     else pk[i >> 1] = h;
   }
-  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
   float lo, hi;
-  f2_unpack(t, lo, hi);
+  f2_unpack(f2_add(acc0, acc1), lo, hi);
   return lo + hi;
-}
-
-// AND of `v` over the 256 softmax threads; doubles as their shared barrier.
-__device__ __forceinline__ bool softmax_sync_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, 256, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return r != 0;
 }
 
 // Lane 0 waits, the result is broadcast to the warp.
@@ -219,27 +233,46 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return ok != 0;
 }
 
+// Lane 0 arrives once all lanes of the warp are past this point.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 template <int D, bool FP4>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   using C = Cfg<D, FP4>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
-  uint64_t* v_full = bars + 2 + kStages;
-  uint64_t* kv_empty = bars + 2 + 2 * kStages;
-  uint64_t* s_full = bars + 2 + 3 * kStages;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 1;
+  uint64_t* q_full = bars + C::kBarQFull;
+  uint64_t* q_empty = bars + C::kBarQEmpty;
+  uint64_t* k_full = bars + C::kBarKFull;      // [stage]
+  uint64_t* v_full = bars + C::kBarVFull;      // [stage]
+  uint64_t* kv_empty = bars + C::kBarKVEmpty;  // [stage], 2 arrivals: S issuer (K), PV issuer (V)
+  uint64_t* s_full = bars + C::kBarSFull;      // [buffer]
+  uint64_t* s_free = bars + C::kBarSFree;      // [buffer], 4 arrivals: owner warpgroup read S
+  uint64_t* p_full = bars + C::kBarPFull;      // [g % kPBufs], 4 arrivals: owner warpgroup wrote P
+  uint64_t* p_free = bars + C::kBarPFree;      // [g % kPBufs]: PV consumed P
+  // Rings whose two sides may drift apart are kStages deep. A block's S needs
+  // its K/V stage, which is released only when PV of the block kStages back has
+  // completed, so in these rings no producer laps its consumer and no waiter is
+  // ever more than one phase behind the phase it waits for (the condition for
+  // a parity wait to be exact).
+  uint64_t* o_ready = bars + C::kBarOReady;    // [g % kStages], 4 arrivals: correction warps
+  uint64_t* o_done = bars + C::kBarODone;      // [g % kStages]: PV of block g completed
+  uint64_t* drain = bars + C::kBarDrain;       // [2]: PV issuer, S issuer
+  uint64_t* m_bar = bars + C::kBarM;           // [quarter][parity]: running max published
+  uint64_t* a_bar = bars + C::kBarA;           // [quarter][g % kStages]: rescale factor published
+  uint64_t* fin_bar = bars + C::kBarFin;       // [item parity], 8 arrivals: per-item (l, m) published
+  uint64_t* fin_free = bars + C::kBarFinFree;  // [item parity], 4 arrivals: correction warps read them
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* issued_cnt = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
   volatile int* consumed_cnt = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
-  float* xmax = reinterpret_cast<float*>(smem + C::kOffXMax);
-  float* xl = reinterpret_cast<float*>(smem + C::kOffXL);
+  float* mx = reinterpret_cast<float*>(smem + C::kOffX);       // [2][128] running max per block parity
+  float* ax = mx + 256;                                         // [kStages][128] O rescale factor
+  float* fin = ax + kStages * 128;                              // [2 items][2 wg][2 (l, m)][128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -250,14 +283,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     for (int s = 0; s < kStages; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(v_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(kv_empty + s, 2);  // S issuer (K read) and PV issuer (V read)
+    }
+    for (int s = 0; s < kStages; ++s) mbar_init(o_ready + s, 4);
+    for (int b = 0; b < C::kPBufs; ++b) {
+      mbar_init(p_full + b, 4);
+      mbar_init(p_free + b, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(p_full + b, 8);  // one arrival per softmax warp
+      mbar_init(s_free + b, 4);
+      mbar_init(fin_bar + b, 8);
+      mbar_init(fin_free + b, 4);
     }
-    mbar_init(o_done, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(o_done + s, 1);
     mbar_init(drain, 1);
+    mbar_init(drain + 1, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(m_bar + i, 1);
+    for (int i = 0; i < 4 * kStages; ++i) mbar_init(a_bar + i, 1);
     *abort_flag = 0;
     *issued_cnt = 0;
     *consumed_cnt = 0;
@@ -276,13 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp < 4) {
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       int g = 0, it = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x, ++it) {
+      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
@@ -296,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int j = 0; j < L.count; ++j, ++g) {
           const int st = g % kStages;
           const int use = g / kStages;
-          if (use > 0 && !(ok = mbar_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty))) break;
+          if (use > 0 && !(ok = mbar_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty)))
+            break;
           const int kb = key_block(p, L, j);
           mbar_arrive_expect_tx(k_full + st, C::kQKTile + C::kSF);
           tma_load_3d(smem + C::kOffK + st * C::kQKTile, &p.tm_k, k_full + st, 0, kb * 128, bh);
@@ -310,34 +354,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescPV = idesc_e4m3(128, D, true);
+      int g = 0;
+      bool ok = true;
+      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
+        int bh, qb;
+        decode_item(p, item, bh, qb);
+        const KList L = key_list(p, qb);
+        for (int j = 0; j < L.count; ++j, ++g) {
+          // O += P V once P is in TMEM, O has been rescaled and V has landed.
+          const int st = g % kStages;
+          const int pb = g % C::kPBufs;
+          if (!(ok = mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
+          if (!(ok = mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
+          if (!(ok = mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
+          tc_fence_after();
+          const uint64_t v_desc =
+              make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
+                          v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(kv_empty + st);
+          mma_commit(p_free + pb);
+          mma_commit(o_done + st);
+          *consumed_cnt = g + 1;
+        }
+      }
+      // Drain: every issued MMA completes before tensor memory is released.
+      mma_commit(drain);
+      uint32_t drained = 0;
+      const unsigned long long t0 = globaltimer_ns();
+      while (!(drained = mbar_try_wait(smem_u32(drain), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+      if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- S issuer
     if (lane == 0) {
       constexpr uint32_t kIdescS = FP4 ? idesc_nvf4(128, 128) : idesc_e4m3(128, 128, false);
-      constexpr uint32_t kIdescPV = idesc_e4m3(128, D, true);
       const uint64_t q_desc = make_smem_desc(smem_u32(smem + C::kOffQ), 16, C::kQKSbo, C::kQKSwz);
       int g = 0, it = 0;
       bool ok = true;
-
-      auto issue_pv = [&](int gg, int jj) -> bool {
-        const int st = gg % kStages;
-        const int buf = gg & 1;
-        if (!mbar_wait(p_full + buf, (gg >> 1) & 1, abort_flag, &g_error_word, kErrPFull)) return false;
-        if (!mbar_wait(v_full + st, (gg / kStages) & 1, abort_flag, &g_error_word, kErrVFull)) return false;
-        tc_fence_after();
-        const uint64_t v_desc = make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a_tmem = tmem + buf * 128 + 64 * (kk >> 1) + 8 * (kk & 1);
-          mma_f8f6f4_ts(tmem + C::kColO, a_tmem, v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV,
-                        (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(kv_empty + st);
-        mma_commit(o_done);
-        *consumed_cnt = gg + 1;
-        return true;
-      };
-
-      for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x, ++it) {
+      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
@@ -349,14 +410,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tmem_cp_32x128_warpx4(tmem + C::kColSFQ + 4 * a,
                                   make_smem_desc(smem_u32(smem + C::kOffSFQ + 512 * a), 128, 128, 0));
         }
-        if (L.count == 0) {
-          mma_commit(q_empty);
-          continue;
-        }
         for (int j = 0; j < L.count; ++j, ++g) {
+          // S = Q K^T into buffer g % 2 once K has landed and the owner
+          // warpgroup has read the buffer's previous tile.
           const int st = g % kStages;
           const int buf = g & 1;
           if (!(ok = mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
+          if (g >= 2 && !(ok = mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
+            break;
           tc_fence_after();
           const uint64_t k_desc =
               make_smem_desc(smem_u32(smem + C::kOffK + st * C::kQKTile), 16, C::kQKSbo, C::kQKSwz);
@@ -377,143 +438,211 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
               mma_f8f6f4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
           }
           mma_commit(s_full + buf);
-          if (j == L.count - 1) mma_commit(q_empty);
-          if (j > 0 && !(ok = issue_pv(g - 1, j - 1))) break;
+          mma_commit(kv_empty + st);
         }
         if (!ok) break;
-        if (!(ok = issue_pv(g - 1, L.count - 1))) break;
+        mma_commit(q_empty);  // all S of the item issued: Q (and its scales) may be replaced
       }
-      // Drain: every issued MMA completes before tensor memory is released.
-      mma_commit(drain);
+      mma_commit(drain + 1);
       uint32_t drained = 0;
       const unsigned long long t0 = globaltimer_ns();
-      while (!(drained = mbar_try_wait(smem_u32(drain), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!(drained = mbar_try_wait(smem_u32(drain + 1), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
-  } else if (warp >= 4) {
-    // -------------------------------------------------------------- softmax
-    const int h = (warp - 4) >> 2;           // key / output half
-    const int q4 = warp & 3;                 // TMEM lane quarter
-    const int row = q4 * 32 + lane;          // query row within the tile
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+  }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------- softmax
+    // Warpgroup w owns the blocks with g % 2 == w (and S buffer w); thread
+    // (warp quarter q, lane t) owns query row 32q + t, all 128 keys.
+    const int w = (warp - 4) >> 2;
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t s_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + w * 128;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     int g = 0, it = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x, ++it) {
+    for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
       int bh, qb;
       decode_item(p, item, bh, qb);
       const KList L = key_list(p, qb);
-      float* xl_it = xl + (it & 1) * 256;  // double-buffered across items
       const int qrow = qb * 128 + row;
       float c_fp4 = 0.f, inv_sq = 0.f;
       if (FP4) c_fp4 = p.q_scale[0] * p.k_scale[0] * p.sm_scale_log2;
       else inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(bh) * p.nblk + qb];
-      float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < L.count; ++j, ++g) {
-        const int buf = g & 1;
+      float l = 0.f, m_ref = -INFINITY;
+      for (int j = 0; j < L.count && ok; ++j, ++g) {
+        if ((g & 1) != w) continue;
         const int kb = key_block(p, L, j);
-        bool mine = warp_wait(s_full + buf, (g >> 1) & 1, abort_flag, &g_error_word, kErrSFull);
-        float s[64];
-        float pmax = -INFINITY;
-        if (mine) {
-          tc_fence_after();
+        if (!(ok = warp_wait(s_full + w, (g >> 1) & 1, abort_flag, &g_error_word, kErrSFull))) break;
+        tc_fence_after();
+        const bool diag = p.causal && kb == qb;
+        const bool masked = diag || (kb + 1) * 128 > p.N;
+        // pass 1: row max of the raw scores, 64 columns at a time
+        float rawmax = -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < 128; cc += 64) {
           uint32_t r0[32], r1[32];
-          tmem_ld32(lane_base + buf * 128 + 64 * h, r0);
-          tmem_ld32(lane_base + buf * 128 + 64 * h + 32, r1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            s[i] = __uint_as_float(r0[i]);
-            s[32 + i] = __uint_as_float(r1[i]);
+          tmem_ld32(s_base + cc, r0);
+          tmem_ld32(s_base + cc + 32, r1);
+          tmem_wait_ld(r0);
+          tmem_wait_ld(r1);
+          if (masked) {
+            mask_chunk(r0, kb * 128 + cc, qrow, diag, p.N);
+            mask_chunk(r1, kb * 128 + cc + 32, qrow, diag, p.N);
           }
-          const int key0 = kb * 128 + 64 * h;
-          if ((p.causal && kb == qb) || key0 + 64 > p.N) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-              const int key = key0 + i;
-              if ((p.causal && key > qrow) || key >= p.N) s[i] = -INFINITY;
-            }
-          }
-          pmax = row_max64(s);
-          xmax[(buf * 2 + h) * 128 + row] = pmax;
+          rawmax = max32(r1, max32(r0, rawmax));
         }
-        ok = softmax_sync_and(mine && ok);
-        if (!ok) break;
-        const float rawmax = fmaxf(pmax, xmax[(buf * 2 + (h ^ 1)) * 128 + row]);
+        // running max: previous block's value from the other warpgroup. The
+        // wait is kept across item boundaries (the value is then unused) so
+        // the two warpgroups stay in lockstep and the two-slot ring never laps.
+        float m_prev = -INFINITY;
+        if (g > 0) {
+          if (!(ok = warp_wait(m_bar + q4 * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, &g_error_word,
+                               kErrMax)))
+            break;
+          if (j > 0) m_prev = mx[((g - 1) & 1) * 128 + row];
+        }
         const float c = FP4 ? c_fp4 : inv_sq / p.k_scale[static_cast<size_t>(bh) * p.nblk + kb];
-        const float m_new = rawmax == -INFINITY ? m : fmaxf(m, rawmax * c);
+        const float m_new = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
+        mx[(g & 1) * 128 + row] = m_new;
+        warp_arrive(m_bar + q4 * 2 + (g & 1));
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float alpha = (m == m_use) ? 1.f : ex2_approx(m - m_use);
-        const float nbias = kLog2_448 - m_use;
-        uint32_t pk[16];
-        const float psum = exp_pack64<C::kPolyPairs>(s, c, nbias, pk);
-        l = l * alpha + psum;
-        m = m_new;
-        // O correction: rows whose max moved scale O by alpha once PV of the
-        // previous tile has landed.
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!warp_wait(o_done, (g - 1) & 1, abort_flag, &g_error_word, kErrODone)) {
-            ok = false;
-            continue;  // skip the P store; the next tile's barrier ends all warps
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int cc = 0; cc < D / 2; cc += 32) {
-            uint32_t o[32];
-            const uint32_t addr = lane_base + C::kColO + h * (D / 2) + cc;
-            tmem_ld32(addr, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(addr, o);
-          }
+        // O rescale factor; a row that has seen no key yet has O = 0, scaled by 0.
+        ax[(g % kStages) * 128 + row] =
+            m_prev == -INFINITY ? 0.f : (m_prev == m_use ? 1.f : ex2_approx(m_prev - m_use));
+        warp_arrive(a_bar + q4 * kStages + g % kStages);
+        if (m_ref != m_use) {
+          if (l != 0.f) l *= ex2_approx(m_ref - m_use);
+          m_ref = m_use;
         }
-        tmem_st16(lane_base + buf * 128 + 64 * h, pk);
+        // pass 2: P = 2^(c s - m + log2 448) -> E4M3 into P buffer g % kPBufs.
+        // The S buffer is released right after its last chunk is read; the P
+        // buffer is waited for only before the first P store.
+        const float nbias = kLog2_448 - m_use;
+        const int pb = g % C::kPBufs;
+        const uint32_t p_base = tmem + lane_off + C::kColP + pb * 32;
+        float psum = 0.f;
+        // The next chunk's tensor-memory load is in flight while the current
+        // one is exponentiated.
+        uint32_t ra[32], rb[32];
+        tmem_ld32(s_base, ra);
+        tmem_wait_ld(ra);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t(&cur)[32] = (cc & 1) ? rb : ra;
+          uint32_t(&nxt)[32] = (cc & 1) ? ra : rb;
+          if (cc < 3) tmem_ld32(s_base + 32 * (cc + 1), nxt);
+          if (cc == 3) {  // all four chunks are in registers: release S
+            tc_fence_before();
+            warp_arrive(s_free + w);
+          }
+          if (masked) mask_chunk(cur, kb * 128 + 32 * cc, qrow, diag, p.N);
+          uint32_t pk[8];
+          psum += exp_pack32<C::kPolyPairs>(cur, c, nbias, pk);
+          if (cc == 0 && g >= C::kPBufs &&
+              !(ok = warp_wait(p_free + pb, ((g / C::kPBufs) - 1) & 1, abort_flag, &g_error_word, kErrPFree)))
+            break;
+          tmem_st8(p_base + 8 * cc, pk);
+          if (cc < 3) tmem_wait_ld(nxt);
+        }
+        if (!ok) break;
+        l += psum;
         tmem_wait_st();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + buf);
+        warp_arrive(p_full + pb);
       }
       if (!ok) break;
-      // ---------------------------------------------------------- epilogue
-      bool done = true;
+      // per-item (l, m) of this warpgroup for the epilogue
+      if (it >= 2 && !(ok = warp_wait(fin_free + (it & 1), ((it >> 1) - 1) & 1, abort_flag, &g_error_word,
+                                      kErrFin)))
+        break;
+      fin[(((it & 1) * 2 + w) * 2 + 0) * 128 + row] = l;
+      fin[(((it & 1) * 2 + w) * 2 + 1) * 128 + row] = m_ref;
+      warp_arrive(fin_bar + (it & 1));
+    }
+  } else {
+    // ------------------------------------------------- correction, epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t o_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::kColO;
+    int g = 0, it = 0;
+    bool ok = true;
+    for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+      int bh, qb;
+      decode_item(p, item, bh, qb);
+      const KList L = key_list(p, qb);
+      for (int j = 0; j < L.count; ++j, ++g) {
+        const int slot = g % kStages;
+        if (!(ok = warp_wait(a_bar + q4 * kStages + slot, (g / kStages) & 1, abort_flag, &g_error_word, kErrAlpha)))
+          break;
+        const float alpha = ax[slot * 128 + row];
+        // Rows whose running max moved scale O by alpha, once PV of the
+        // previous block has landed (block 0 overwrites O instead).
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!(ok = warp_wait(o_done + (g - 1) % kStages, ((g - 1) / kStages) & 1, abort_flag, &g_error_word,
+                               kErrODone)))
+            break;
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32(o_base + cc, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(o_base + cc, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        warp_arrive(o_ready + slot);
+      }
+      if (!ok) break;
+      // epilogue: combine the two warpgroups' row sums, normalize, store
+      if (!(ok = warp_wait(fin_bar + (it & 1), (it >> 1) & 1, abort_flag, &g_error_word, kErrFin))) break;
+      const float* f = fin + (it & 1) * 512;
+      const float l0 = f[0 * 128 + row], m0 = f[1 * 128 + row];
+      const float l1 = f[2 * 128 + row], m1 = f[3 * 128 + row];
+      warp_arrive(fin_free + (it & 1));
+      const float m = fmaxf(m0, m1);
+      const float ltot = (l0 > 0.f ? l0 * ex2_approx(m0 - m) : 0.f) + (l1 > 0.f ? l1 * ex2_approx(m1 - m) : 0.f);
+      const float inv_l = ltot > 0.f ? 1.f / ltot : 0.f;
       if (L.count > 0) {
-        done = warp_wait(o_done, (g - 1) & 1, abort_flag, &g_error_word, kErrODone);
+        if (!(ok = warp_wait(o_done + (g - 1) % kStages, ((g - 1) / kStages) & 1, abort_flag, &g_error_word,
+                             kErrODone)))
+          break;
         tc_fence_after();
       }
-      xl_it[h * 128 + row] = l;
-      ok = softmax_sync_and(done && ok);
-      if (!ok) break;
-      const float ltot = l + xl_it[(h ^ 1) * 128 + row];
-      const float inv_l = ltot > 0.f ? 1.f / ltot : 0.f;
+      const int qrow = qb * 128 + row;
       const bool store = qrow < p.N;
-      __nv_bfloat16* orow = p.out + (static_cast<size_t>(bh) * p.N + (store ? qrow : 0)) * D + h * (D / 2);
-      const float* vs = p.v_scale + static_cast<size_t>(bh) * D + h * (D / 2);
+      __nv_bfloat16* orow = p.out + (static_cast<size_t>(bh) * p.N + (store ? qrow : 0)) * D;
+      const float* vs = p.v_scale + static_cast<size_t>(bh) * D;
 #pragma unroll
-      for (int cc = 0; cc < D / 2; cc += 32) {
+      for (int cc = 0; cc < D; cc += 32) {
         uint32_t o[32];
         if (L.count > 0) {
-          tmem_ld32(lane_base + C::kColO + h * (D / 2) + cc, o);
-          tmem_wait_ld();
+          tmem_ld32(o_base + cc, o);
+          tmem_wait_ld(o);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        uint32_t w[16];
+        uint32_t wd[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float a = __uint_as_float(o[2 * i]) * inv_l / __ldg(vs + cc + 2 * i);
-          const float b = __uint_as_float(o[2 * i + 1]) * inv_l / __ldg(vs + cc + 2 * i + 1);
+          const float a = __uint_as_float(o[2 * i]) * __fdividef(inv_l, __ldg(vs + cc + 2 * i));
+          const float b = __uint_as_float(o[2 * i + 1]) * __fdividef(inv_l, __ldg(vs + cc + 2 * i + 1));
           __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
-          w[i] = *reinterpret_cast<uint32_t*>(&t);
+          wd[i] = *reinterpret_cast<uint32_t*>(&t);
         }
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
         }
       }
-      if (h == 0 && store && p.lse)
+      if (store && p.lse)
         p.lse[static_cast<size_t>(bh) * p.N + qrow] =
             ltot > 0.f ? (m + __log2f(ltot) - kLog2_448) * kLn2 : -INFINITY;
       tc_fence_before();
