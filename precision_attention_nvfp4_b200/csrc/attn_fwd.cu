@@ -20,21 +20,20 @@
 //   warp 1        tensor-memory allocator; issues O += P V (one thread)
 //   warp 2        issues S = Q K^T (one thread)
 //   warp 3        idle
-//   warps 4-7     softmax warpgroup 0: key blocks with even global index
-//   warps 8-11    softmax warpgroup 1: key blocks with odd global index
+//   warps 4-7     softmax warpgroup 0: keys 0-63 of every key block
+//   warps 8-11    softmax warpgroup 1: keys 64-127 of every key block
 //   warps 12-15   O rescale (correction) and epilogue
 // Thread (warp quarter q, lane t) of a softmax warpgroup owns query row
-// 32q + t and all 128 keys of its block, read from TMEM in 32-column chunks
-// twice (row max, then exponentials). The two softmax warpgroups alternate
-// blocks, so one group's exponentials (MUFU and FMA pipes) overlap the
-// other's tensor-memory loads and waits; the only value they exchange is the
-// running row max, passed per warp pair through shared memory and an
-// mbarrier. Each keeps its own row sum relative to the last max it used; the
-// epilogue combines them.
+// 32q + t and its warpgroup's 64 keys of the block, read from TMEM once into
+// registers. The two warps sharing a row quarter (and an SM sub-partition)
+// work on the same block at the same time, so their exponentials keep the
+// MUFU and FMA pipes busy together; they exchange only their half-block row
+// maxima, per lane, through tagged shared-memory words. Each keeps the row
+// sum of its half; the epilogue adds the two.
 // Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32
-// 128x128, buffer = block parity), O at column 256 (d fp32 columns), P double
-// buffer (E4M3, 32 columns each) at 384, NVFP4 scale vectors of Q and of two
-// K tiles at 448. S and P having their own buffers lets the S of a block be
+// 128x128, buffer = block parity), O at column 256 (d fp32 columns), a ring
+// of three P buffers (E4M3, 32 columns each) at 384, NVFP4 scale vectors of Q
+// and of two K tiles at 480. S and P having their own buffers lets the S of a block be
 // issued as soon as its buffer's previous tile has been read, independently
 // of the PV of that tile; the two MMA kinds are issued by separate threads.
 // Work items are (batch*head, 128-query block); causal runs schedule the
@@ -57,7 +56,7 @@ __device__ int g_error_word = 0;
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -65,7 +64,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 enum : int {
   kErrQEmpty = 0x101, kErrKvEmpty = 0x102, kErrQFull = 0x201, kErrKFull = 0x202, kErrVFull = 0x203,
   kErrPFull = 0x204, kErrOReady = 0x205, kErrSFull = 0x301, kErrMax = 0x303, kErrFin = 0x304,
-  kErrAlpha = 0x305, kErrSFree = 0x306, kErrPFree = 0x307, kErrODone = 0x302, kErrDrain = 0x401
+  kErrAlpha = 0x305, kErrSFree = 0x306, kErrODone = 0x302, kErrDrain = 0x401
 };
 
 template <int D, bool FP4>
@@ -81,7 +80,12 @@ struct Cfg {
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
   static constexpr int kPolyPairs = 4;                    // of 16 exp2 pairs per 32-score chunk
   static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
-  static constexpr int kPBufs = 3;                        // P buffers: 32 columns each (128 E4M3 keys)
+  // P buffers, 32 columns each (128 E4M3 keys). As many as K/V stages: the
+  // S of block g needs K stage g % kStages, which is refilled only after the
+  // PV of block g - kStages has completed, and that PV was the last reader of
+  // P buffer g % kPBufs. So a softmax thread that has seen S(g) may overwrite
+  // the buffer without a barrier of its own.
+  static constexpr int kPBufs = kStages;
   static constexpr uint32_t kColP = 384;
   static constexpr uint32_t kColSFQ = kColP + 32 * kPBufs;
   static constexpr uint32_t kSFCols = 4 * (D / 64);
@@ -97,13 +101,13 @@ struct Cfg {
   static constexpr int kBarQFull = 0, kBarQEmpty = 1, kBarKFull = 2;
   static constexpr int kBarVFull = kBarKFull + kStages, kBarKVEmpty = kBarVFull + kStages;
   static constexpr int kBarSFull = kBarKVEmpty + kStages, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2;
-  static constexpr int kBarPFree = kBarPFull + kPBufs, kBarOReady = kBarPFree + kPBufs, kBarODone = kBarOReady + kStages;
-  static constexpr int kBarDrain = kBarODone + kStages, kBarM = kBarDrain + 2, kBarA = kBarM + 8;
+  static constexpr int kBarOReady = kBarPFull + kPBufs, kBarODone = kBarOReady + kStages;
+  static constexpr int kBarDrain = kBarODone + kStages, kBarA = kBarDrain + 2;
   static constexpr int kBarFin = kBarA + 4 * kStages, kBarFinFree = kBarFin + 2;
   static constexpr int kNumBars = kBarFinFree + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffX = (kOffMisc + 64 + 15) & ~15;      // running max, rescale, per-item (l, m)
-  static constexpr int kBytes = kOffX + (2 * 128 + kStages * 128 + 2 * 2 * 2 * 128) * 4;
+  static constexpr int kBytes = kOffX + 4 * 128 * 8 + (kStages * 128 + 2 * 2 * 2 * 128) * 4;
   // Request at least this much so that a single CTA fits per SM (it takes
   // all 512 tensor-memory columns).
   static constexpr int kSmemRequest = (kBytes + 1024 > 120 * 1024 ? kBytes + 1024 : 120 * 1024);
@@ -225,12 +229,35 @@ __device__ __forceinline__ float exp_pack32(const uint32_t (&r)[32], float c, fl
   return lo + hi;
 }
 
-// Lane 0 waits, the result is broadcast to the warp.
+// Every lane polls the barrier (one broadcast shared-memory access per poll),
+// so the warp never diverges around the wait.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
-  uint32_t ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, code) ? 1u : 0u;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return ok != 0;
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err, code));
+}
+
+// Polls a shared-memory word until its high half equals tag, then returns
+// its low half (a float) in val. A 64-bit aligned store is single-copy
+// atomic, so the value and its tag arrive together. Bounded like mbar_wait.
+__device__ __forceinline__ bool tagged_wait(const volatile unsigned long long* slot, uint32_t tag, float& val,
+                                            volatile int* abort, int* err, int code) {
+  unsigned long long v, t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    v = *slot;
+    if (static_cast<uint32_t>(v >> 32) == tag) break;
+    if ((it & 63u) == 63u) {
+      if (*abort) return false;
+      const unsigned long long now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitTimeoutNs) {
+        atomicCAS(err, 0, code);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+  val = __uint_as_float(static_cast<uint32_t>(v));
+  return true;
 }
 
 // Lane 0 arrives once all lanes of the warp are past this point.
@@ -251,9 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   uint64_t* v_full = bars + C::kBarVFull;      // [stage]
   uint64_t* kv_empty = bars + C::kBarKVEmpty;  // [stage], 2 arrivals: S issuer (K), PV issuer (V)
   uint64_t* s_full = bars + C::kBarSFull;      // [buffer]
-  uint64_t* s_free = bars + C::kBarSFree;      // [buffer], 4 arrivals: owner warpgroup read S
-  uint64_t* p_full = bars + C::kBarPFull;      // [g % kPBufs], 4 arrivals: owner warpgroup wrote P
-  uint64_t* p_free = bars + C::kBarPFree;      // [g % kPBufs]: PV consumed P
+  uint64_t* s_free = bars + C::kBarSFree;      // [buffer], 8 arrivals: softmax warps read S
+  uint64_t* p_full = bars + C::kBarPFull;      // [g % kPBufs], 8 arrivals: softmax warps wrote P
   // Rings whose two sides may drift apart are kStages deep. A block's S needs
   // its K/V stage, which is released only when PV of the block kStages back has
   // completed, so in these rings no producer laps its consumer and no waiter is
@@ -262,16 +288,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   uint64_t* o_ready = bars + C::kBarOReady;    // [g % kStages], 4 arrivals: correction warps
   uint64_t* o_done = bars + C::kBarODone;      // [g % kStages]: PV of block g completed
   uint64_t* drain = bars + C::kBarDrain;       // [2]: PV issuer, S issuer
-  uint64_t* m_bar = bars + C::kBarM;           // [quarter][parity]: running max published
-  uint64_t* a_bar = bars + C::kBarA;           // [quarter][g % kStages]: rescale factor published
+  uint64_t* a_bar = bars + C::kBarA;           // [quarter][g % kStages]: rescale factor published (warpgroup 0)
   uint64_t* fin_bar = bars + C::kBarFin;       // [item parity], 8 arrivals: per-item (l, m) published
   uint64_t* fin_free = bars + C::kBarFinFree;  // [item parity], 4 arrivals: correction warps read them
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* issued_cnt = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
   volatile int* consumed_cnt = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
-  float* mx = reinterpret_cast<float*>(smem + C::kOffX);       // [2][128] running max per block parity
-  float* ax = mx + 256;                                         // [kStages][128] O rescale factor
+  // [block parity][warpgroup][128]: half-block row max, tag g + 1 in the high word
+  volatile unsigned long long* xs = reinterpret_cast<volatile unsigned long long*>(smem + C::kOffX);
+  float* ax = reinterpret_cast<float*>(smem + C::kOffX + 4 * 128 * 8);  // [kStages][128] O rescale factor
   float* fin = ax + kStages * 128;                              // [2 items][2 wg][2 (l, m)][128]
 
   const int warp = threadIdx.x >> 5;
@@ -287,25 +313,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     for (int s = 0; s < kStages; ++s) mbar_init(o_ready + s, 4);
     for (int b = 0; b < C::kPBufs; ++b) {
-      mbar_init(p_full + b, 4);
-      mbar_init(p_free + b, 1);
+      mbar_init(p_full + b, 8);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_free + b, 4);
+      mbar_init(s_free + b, 8);
       mbar_init(fin_bar + b, 8);
       mbar_init(fin_free + b, 4);
     }
     for (int s = 0; s < kStages; ++s) mbar_init(o_done + s, 1);
     mbar_init(drain, 1);
     mbar_init(drain + 1, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(m_bar + i, 1);
     for (int i = 0; i < 4 * kStages; ++i) mbar_init(a_bar + i, 1);
     *abort_flag = 0;
     *issued_cnt = 0;
     *consumed_cnt = 0;
     fence_barrier_init();
   }
+  for (int i = threadIdx.x; i < 4 * 128; i += kThreads) xs[i] = 0ull;
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
@@ -378,7 +403,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
                           v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(kv_empty + st);
-          mma_commit(p_free + pb);
           mma_commit(o_done + st);
           *consumed_cnt = g + 1;
         }
@@ -453,12 +477,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
   } else if (warp < 12) {
     // ------------------------------------------------------------- softmax
-    // Warpgroup w owns the blocks with g % 2 == w (and S buffer w); thread
-    // (warp quarter q, lane t) owns query row 32q + t, all 128 keys.
+    // Both warpgroups work on every key block: warpgroup w takes keys
+    // 64w..64w+63 of it. Thread (warp quarter q, lane t) owns query row
+    // 32q + t; its 64 scores are read from tensor memory once and stay in
+    // registers. The two halves' row maxima are exchanged per lane through a
+    // tagged shared-memory word, so each thread holds the exact running max
+    // of its row without any chain between blocks.
     const int w = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
-    const uint32_t s_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + w * 128;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     int g = 0, it = 0;
     bool ok = true;
@@ -472,88 +499,69 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       else inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(bh) * p.nblk + qb];
       float l = 0.f, m_ref = -INFINITY;
       for (int j = 0; j < L.count && ok; ++j, ++g) {
-        if ((g & 1) != w) continue;
         const int kb = key_block(p, L, j);
-        if (!(ok = warp_wait(s_full + w, (g >> 1) & 1, abort_flag, &g_error_word, kErrSFull))) break;
+        const int buf = g & 1;
+        // A failed wait raises the abort flag; the block then runs to its end
+        // on whatever the buffers hold (every later wait returns at once) and
+        // the loop stops after it.
+        ok = warp_wait(s_full + buf, (g >> 1) & 1, abort_flag, &g_error_word, kErrSFull);
         tc_fence_after();
+        uint32_t r0[32], r1[32];
+        const uint32_t s_addr = tmem + lane_off + buf * 128 + 64 * w;
+        tmem_ld32(s_addr, r0);
+        tmem_ld32(s_addr + 32, r1);
+        tmem_wait_ld(r0);
+        tmem_wait_ld(r1);
+        // both halves are in registers: the buffer may take the next S
+        tc_fence_before();
+        warp_arrive(s_free + buf);
+        const int key0 = kb * 128 + 64 * w;
         const bool diag = p.causal && kb == qb;
-        const bool masked = diag || (kb + 1) * 128 > p.N;
-        // pass 1: row max of the raw scores, 64 columns at a time
-        float rawmax = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < 128; cc += 64) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(s_base + cc, r0);
-          tmem_ld32(s_base + cc + 32, r1);
-          tmem_wait_ld(r0);
-          tmem_wait_ld(r1);
-          if (masked) {
-            mask_chunk(r0, kb * 128 + cc, qrow, diag, p.N);
-            mask_chunk(r1, kb * 128 + cc + 32, qrow, diag, p.N);
-          }
-          rawmax = max32(r1, max32(r0, rawmax));
+        if (diag || (kb + 1) * 128 > p.N) {
+          mask_chunk(r0, key0, qrow, diag, p.N);
+          mask_chunk(r1, key0 + 32, qrow, diag, p.N);
         }
-        // running max: previous block's value from the other warpgroup. The
-        // wait is kept across item boundaries (the value is then unused) so
-        // the two warpgroups stay in lockstep and the two-slot ring never laps.
-        float m_prev = -INFINITY;
-        if (g > 0) {
-          if (!(ok = warp_wait(m_bar + q4 * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, &g_error_word,
-                               kErrMax)))
-            break;
-          if (j > 0) m_prev = mx[((g - 1) & 1) * 128 + row];
-        }
+        const float half_max = max32(r1, max32(r0, -INFINITY));
+        // exchange the half maxima (tag g + 1; slots alternate by block parity)
+        xs[(buf * 2 + w) * 128 + row] =
+            (static_cast<unsigned long long>(g + 1) << 32) | __float_as_uint(half_max);
+        float other_max;
+        const bool got = tagged_wait(xs + (buf * 2 + (w ^ 1)) * 128 + row, static_cast<uint32_t>(g + 1), other_max,
+                                     abort_flag, &g_error_word, kErrMax);
+        ok = __all_sync(0xffffffffu, got) && ok;
+        const float rawmax = w == 0 ? fmaxf(half_max, other_max) : fmaxf(other_max, half_max);
         const float c = FP4 ? c_fp4 : inv_sq / p.k_scale[static_cast<size_t>(bh) * p.nblk + kb];
+        // m_ref: exact running max (-inf while every key so far is masked);
+        // m_use: the offset the exponentials use (0 in that case).
+        const float m_prev = m_ref;
         const float m_new = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
-        mx[(g & 1) * 128 + row] = m_new;
-        warp_arrive(m_bar + q4 * 2 + (g & 1));
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        // O rescale factor; a row that has seen no key yet has O = 0, scaled by 0.
-        ax[(g % kStages) * 128 + row] =
-            m_prev == -INFINITY ? 0.f : (m_prev == m_use ? 1.f : ex2_approx(m_prev - m_use));
-        warp_arrive(a_bar + q4 * kStages + g % kStages);
-        if (m_ref != m_use) {
-          if (l != 0.f) l *= ex2_approx(m_ref - m_use);
-          m_ref = m_use;
+        // Rescale factor of O and of the row sum; a row that has seen no key
+        // yet (m_prev = -inf) has O = 0 and l = 0, scaled by 2^-inf = 0.
+        const float alpha = m_prev == m_new ? 1.f : ex2_approx(m_prev - m_use);
+        if (w == 0) {
+          ax[(g % kStages) * 128 + row] = alpha;
+          warp_arrive(a_bar + q4 * kStages + g % kStages);
         }
-        // pass 2: P = 2^(c s - m + log2 448) -> E4M3 into P buffer g % kPBufs.
-        // The S buffer is released right after its last chunk is read; the P
-        // buffer is waited for only before the first P store.
+        l *= alpha;
+        m_ref = m_new;
+        // P = 2^(c s - m + log2 448) -> E4M3, this half's 16 columns of P
+        // buffer g % kPBufs.
         const float nbias = kLog2_448 - m_use;
         const int pb = g % C::kPBufs;
-        const uint32_t p_base = tmem + lane_off + C::kColP + pb * 32;
-        float psum = 0.f;
-        // The next chunk's tensor-memory load is in flight while the current
-        // one is exponentiated.
-        uint32_t ra[32], rb[32];
-        tmem_ld32(s_base, ra);
-        tmem_wait_ld(ra);
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t(&cur)[32] = (cc & 1) ? rb : ra;
-          uint32_t(&nxt)[32] = (cc & 1) ? ra : rb;
-          if (cc < 3) tmem_ld32(s_base + 32 * (cc + 1), nxt);
-          if (cc == 3) {  // all four chunks are in registers: release S
-            tc_fence_before();
-            warp_arrive(s_free + w);
-          }
-          if (masked) mask_chunk(cur, kb * 128 + 32 * cc, qrow, diag, p.N);
-          uint32_t pk[8];
-          psum += exp_pack32<C::kPolyPairs>(cur, c, nbias, pk);
-          if (cc == 0 && g >= C::kPBufs &&
-              !(ok = warp_wait(p_free + pb, ((g / C::kPBufs) - 1) & 1, abort_flag, &g_error_word, kErrPFree)))
-            break;
-          tmem_st8(p_base + 8 * cc, pk);
-          if (cc < 3) tmem_wait_ld(nxt);
-        }
-        if (!ok) break;
+        const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32 + 16 * w;
+        uint32_t pk0[8], pk1[8];
+        float psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
+        tmem_st8(p_addr, pk0);
+        psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
+        tmem_st8(p_addr + 8, pk1);
         l += psum;
         tmem_wait_st();
         tc_fence_before();
         warp_arrive(p_full + pb);
       }
       if (!ok) break;
-      // per-item (l, m) of this warpgroup for the epilogue
+      // per-item (l, m) of this warpgroup's half of the keys for the epilogue
       if (it >= 2 && !(ok = warp_wait(fin_free + (it & 1), ((it >> 1) - 1) & 1, abort_flag, &g_error_word,
                                       kErrFin)))
         break;
@@ -584,13 +592,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                                kErrODone)))
             break;
           tc_fence_after();
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
           for (int cc = 0; cc < D; cc += 32) {
             uint32_t o[32];
             tmem_ld32(o_base + cc, o);
             tmem_wait_ld(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            for (int i = 0; i < 16; ++i) {
+              const uint64_t v = f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2);
+              float lo, hi;
+              f2_unpack(v, lo, hi);
+              o[2 * i] = __float_as_uint(lo);
+              o[2 * i + 1] = __float_as_uint(hi);
+            }
             tmem_st32(o_base + cc, o);
           }
           tmem_wait_st();
