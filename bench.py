@@ -9,6 +9,7 @@ events on the launching stream; multi-GPU runs take the max over ranks. Rank 0
 prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py --sweep     # sequence-length sweep, one JSON line per configuration
 
 ``--impl reference`` times the CPU oracle (the only other implementation of
 this path) on a bounded sample of the same workload, on the host cores.
@@ -144,21 +145,27 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks):
-    """Run the oracle (as it stands) on a bounded sample; returns (flops, seconds)."""
+def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks, budget_s: float = 0.0):
+    """Run the oracle (as it stands) on a bounded sample; returns (flops,
+    seconds, (head, query block) pairs done). With budget_s > 0 the sample
+    stops after the first pair that ends past the budget."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import parity
     from oracle import attention as oatt
     t0 = time.perf_counter()
-    qh, kh, vh = parity.oracle_operands(q, k, v, w.qk_format, heads)
     flops = 0.0
-    for i, _ in enumerate(heads):
+    done = []
+    for h in heads:
+        qh, kh, vh = parity.oracle_operands(q, k, v, w.qk_format, [h])
         for qb in qblocks:
             rows = np.arange(qb * 128, min(w.N, qb * 128 + 128))
-            oatt.attention_rows(qh[i], kh[i], vh[i], rows, causal=w.causal)
+            oatt.attention_rows(qh[0], kh[0], vh[0], rows, causal=w.causal)
             keys = (rows + 1) if w.causal else np.full(len(rows), w.N)
             flops += float(np.sum(4.0 * keys * w.d))
-    return flops, time.perf_counter() - t0
+            done.append((h, qb))
+            if budget_s > 0 and time.perf_counter() - t0 > budget_s:
+                return flops, time.perf_counter() - t0, done
+    return flops, time.perf_counter() - t0, done
 
 
 def host_cores():
@@ -180,7 +187,7 @@ def run_reference(args, w):
         cpu_oracle_sample(w, q, k, v, [0], qblocks)
     tot_f, tot_s = 0.0, 0.0
     for _ in range(args.steps):
-        f, s = cpu_oracle_sample(w, q, k, v, [0], qblocks)
+        f, s, _ = cpu_oracle_sample(w, q, k, v, [0], qblocks)
         tot_f += f
         tot_s += s
     value = tot_f / tot_s / 1e12
@@ -224,6 +231,91 @@ def config_dict(w):
             "l2": "inputs larger than L2 (bf16 Q,K,V of the step exceed 126 MB)"}
 
 
+def time_cuda(fn, min_runs: int = 5, budget_ms: float = 1500.0) -> float:
+    """Median device time (ms) of fn() over enough runs to fill about budget_ms
+    (at least min_runs), after 3 warm-up calls."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fn()
+    e1.record()
+    torch.cuda.synchronize()
+    one = e0.elapsed_time(e1)
+    runs = max(min_runs, min(50, int(budget_ms / max(one, 1e-3))))
+    times = []
+    for _ in range(runs):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return float(np.median(times))
+
+
+def run_sweep(args):
+    """Sequence sweep: N in 1K..128K, H = 32, B*H*N = 2^22, d in {64, 128},
+    causal and not, NVFP4 QK + FP8 PV against all-FP8. Inputs are drawn on the
+    device from a seeded CUDA generator (~N(0,1), four x20 outlier channels per
+    head shared by Q and K); every N views the same buffers. One JSON line per
+    configuration: attention time, dense-equivalent and executed TFLOPS, the
+    fraction of the tensor peak, and the quantization bandwidth."""
+    import precision_attention_nvfp4_b200 as fp
+    torch.cuda.set_device(0)
+    peaks, peak_src = load_peaks()
+    bf16 = peaks.get("bf16_tflops", 1590.0)
+    p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    tokens = 1 << 22
+    for d in (64, 128):
+        qf = torch.randn(tokens, d, device="cuda", generator=gen)
+        kf = torch.randn(tokens, d, device="cuda", generator=gen)
+        vf = torch.randn(tokens, d, device="cuda", generator=gen)
+        for N in (1024, 4096, 16384, 32768, 65536, 131072):
+            B = tokens // (32 * N)
+            q = qf.view(B, 32, N, d).clone()
+            k = kf.view(B, 32, N, d).clone()
+            ch = torch.randperm(d, device="cuda", generator=gen)[:4]
+            q[..., ch] *= 20.0
+            k[..., ch] *= 20.0
+            q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+            v = vf.view(B, 32, N, d).to(torch.bfloat16)
+            vq = fp.quantize_fp8(v, "channel")
+            for fmt in ("nvfp4", "fp8"):
+                if fmt == "nvfp4":
+                    qq, kq = fp.quantize_nvfp4(q), fp.quantize_nvfp4(k)
+                    quant = lambda: (fp.quantize_nvfp4(q), fp.quantize_nvfp4(k))
+                    qbytes = 2 * q.numel() * (2 + 2 + 0.5 + 1 / 16)
+                else:
+                    qq, kq = fp.quantize_fp8(q, "tile128"), fp.quantize_fp8(k, "tile128")
+                    quant = lambda: (fp.quantize_fp8(q, "tile128"), fp.quantize_fp8(k, "tile128"))
+                    qbytes = 2 * q.numel() * (2 + 1)
+                q_ms = time_cuda(quant)
+                for causal in (False, True):
+                    out, lse = fp.attention_fwd(qq, kq, vq, causal=causal)
+                    ms = time_cuda(lambda: fp.attention_fwd(qq, kq, vq, causal=causal, out=out, lse=lse))
+                    err = fp.device_error()
+                    w = workloads.Workload("sweep", B=B, H=32, N=N, d=d, causal=causal, qk_format=fmt, seed=5)
+                    flops = w.dense_flops()
+                    exec_flops = 4.0 * 128 * 128 * d * executed_block_pairs(w) * B * 32
+                    peak = 2.0 / (1.0 / p4 + 1.0 / p8) if fmt == "nvfp4" else p8
+                    tf = flops / (ms * 1e-3) / 1e12
+                    print(json.dumps({
+                        "sweep": True, "N": N, "B": B, "H": 32, "d": d, "causal": causal, "qk": fmt,
+                        "attn_ms": ms, "tflops_dense_eq": tf,
+                        "tflops_executed": exec_flops / (ms * 1e-3) / 1e12,
+                        "frac_of_peak": tf / peak, "peak_tflops": peak,
+                        "peak_source": f"{peak_src} bf16 burst {bf16} x nominal fp8 2x / fp4 4x",
+                        "quant_qk_ms": q_ms, "quant_qk_gbs": qbytes / (q_ms * 1e-3) / 1e9,
+                        "device_error": err}), flush=True)
+            del q, k, v, vq
+        del qf, kf, vf
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -233,7 +325,10 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
     w = workloads.get(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)
@@ -301,9 +396,12 @@ def main():
     attn_ms = rank_max(attn_ms)
     err = fp.device_error()
 
-    flops = w.dense_flops()
     pairs = executed_block_pairs(w)
     exec_flops = 4.0 * 128 * 128 * w.d * pairs * w.B * w.H
+    # Algorithmic flops: 4*B*H*N^2*d, halved under the causal mask; under the
+    # sliding-tile mask only the allowed (tile, tile) token pairs, which the
+    # mask makes whole 128x128 blocks, so exactly the executed blocks.
+    flops = exec_flops if w.sparse else w.dense_flops()
     ms_step = ms_total / args.steps
     value = aggregate_value(flops, world, ms_step)
     peaks, peak_src = load_peaks()
@@ -339,13 +437,16 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # about 15 s of oracle work: query blocks spread over the rows and heads
         nblk = (w.N + 127) // 128
-        heads = [0, w.B * w.H // 2]
-        qblocks = [nblk - 1, nblk // 2, 1]
-        f, s = cpu_oracle_sample(w, q_h, k_h, v_h, heads, qblocks)
+        bh = w.B * w.H
+        heads = list(range(0, bh, max(1, bh // 32)))
+        qblocks = sorted({nblk - 1, (3 * nblk) // 4, nblk // 2, nblk // 4, 1, 0}, reverse=True)
+        f, s, done = cpu_oracle_sample(w, q_h, k_h, v_h, heads, qblocks, budget_s=15.0)
         cpu = {"value": f / s / 1e12, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
-               "sample": f"heads {heads}, query blocks {qblocks} of {w.name} (fp64 numpy, oracle "
-                         f"quantization of those heads included), {s:.1f} s"}
+               "sample": f"{len(done)} (batch*head, 128-query block) pairs of {w.name}: heads "
+                         f"{sorted(set(h for h, _ in done))} x query blocks {qblocks} in that order (fp64 "
+                         f"numpy oracle, its quantization of those heads included), {s:.1f} s"}
 
     launches_per_step = (6 if w.qk_format == "nvfp4" else 2) + 3 + 1
     if rank == 0:
@@ -354,7 +455,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e2m1/e4m3 MMA, f32 accumulate", "data": "synthetic",
             "config": config_dict(w),
-            "attn_ms": attn_ms, "attn_tflops_dense_eq": attn_tflops,
+            "attn_ms": attn_ms, "attn_tflops_algorithmic": attn_tflops,
+            "attn_tflops_dense_eq": w.dense_flops() / (attn_ms * 1e-3) / 1e12,
             "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,
             "quant_ms": quant_ms, "quant_gbs": quant_gbs, "quant_frac_hbm": quant_gbs / peaks["hbm_gbs"],
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
