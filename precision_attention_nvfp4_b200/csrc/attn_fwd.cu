@@ -107,7 +107,10 @@ struct Cfg {
   static constexpr int kNumBars = kBarFinFree + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffX = (kOffMisc + 64 + 15) & ~15;      // running max, rescale, per-item (l, m)
-  static constexpr int kBytes = kOffX + 4 * 128 * 8 + (kStages * 128 + 2 * 2 * 2 * 128) * 4;
+  static constexpr int kOutWarpBytes = 32 * 2 * D;
+  static constexpr int kOffOut =
+      (kOffX + 4 * 128 * 8 + (kStages * 128 + 2 * 2 * 2 * 128 + 4 * D) * 4 + 1023) & ~1023;
+  static constexpr int kBytes = kOffOut + 4 * kOutWarpBytes;
   // Request at least this much so that a single CTA fits per SM (it takes
   // all 512 tensor-memory columns).
   static constexpr int kSmemRequest = (kBytes + 1024 > 120 * 1024 ? kBytes + 1024 : 120 * 1024);
@@ -117,6 +120,7 @@ struct __align__(64) Params {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
+  CUtensorMap tm_out;  // bf16 [BH][N][d], box 64 x 32 rows, 128-byte swizzle
   const uint8_t* q_sf;
   const uint8_t* k_sf;
   const float* q_scale;
@@ -299,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   volatile unsigned long long* xs = reinterpret_cast<volatile unsigned long long*>(smem + C::kOffX);
   float* ax = reinterpret_cast<float*>(smem + C::kOffX + 4 * 128 * 8);  // [kStages][128] O rescale factor
   float* fin = ax + kStages * 128;                              // [2 items][2 wg][2 (l, m)][128]
+  float* inv_vs = fin + 2 * 2 * 2 * 128;                        // [correction warp][d]: 1 / V scale
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -580,6 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       int bh, qb;
       decode_item(p, item, bh, qb);
       const KList L = key_list(p, qb);
+      // this head's V scales, loaded now so their latency hides behind the
+      // item's blocks (lane t holds channels t, t + 32, ...)
+      float vsv[D / 32];
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) vsv[i] = __ldg(p.v_scale + static_cast<size_t>(bh) * D + lane + 32 * i);
       for (int j = 0; j < L.count; ++j, ++g) {
         const int slot = g % kStages;
         if (!(ok = warp_wait(a_bar + q4 * kStages + slot, (g / kStages) & 1, abort_flag, &g_error_word, kErrAlpha)))
@@ -631,37 +641,59 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       const int qrow = qb * 128 + row;
       const bool store = qrow < p.N;
-      __nv_bfloat16* orow = p.out + (static_cast<size_t>(bh) * p.N + (store ? qrow : 0)) * D;
-      const float* vs = p.v_scale + static_cast<size_t>(bh) * D;
+      // per-channel 1 / V scale in the warp's own shared-memory slice (read
+      // back as broadcasts)
+      float* rv = inv_vs + q4 * D;
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 32) {
-        uint32_t o[32];
+      for (int i = 0; i < D / 32; ++i) rv[lane + 32 * i] = __frcp_rn(vsv[i]);
+      // the staging tile's previous contents must have been read out
+      if (lane == 0) bulk_wait_read();
+      __syncwarp();
+      // Each thread writes its bf16 row into the warp's staging tiles (32 rows
+      // x 64 columns each, 16-byte granule g of row r at g ^ (r % 8): the
+      // tensor map's 128-byte swizzle, free of bank conflicts); one thread
+      // then stores them with the tensor engine, which also clips rows >= N.
+      // The next item's first PV overwrites O, so this epilogue is on the
+      // critical path only until O has been read.
+      uint8_t* tile = smem + C::kOffOut + q4 * C::kOutWarpBytes;
+#pragma unroll 2
+      for (int cc = 0; cc < D; cc += 16) {
+        uint32_t o[16];
         if (L.count > 0) {
-          tmem_ld32(o_base + cc, o);
+          tmem_ld16(o_base + cc, o);
           tmem_wait_ld(o);
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int i = 0; i < 16; ++i) o[i] = 0u;
         }
-        uint32_t wd[16];
+        uint32_t wd[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = __uint_as_float(o[2 * i]) * __fdividef(inv_l, __ldg(vs + cc + 2 * i));
-          const float b = __uint_as_float(o[2 * i + 1]) * __fdividef(inv_l, __ldg(vs + cc + 2 * i + 1));
-          __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+        for (int i = 0; i < 8; ++i) {
+          __nv_bfloat162 t = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv_l * rv[cc + 2 * i],
+                                                  __uint_as_float(o[2 * i + 1]) * inv_l * rv[cc + 2 * i + 1]);
           wd[i] = *reinterpret_cast<uint32_t*>(&t);
         }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
+        for (int k = 0; k < 2; ++k) {
+          const int col = cc + 8 * k;
+          const int gr = (col & 63) >> 3;
+          uint4* dst = reinterpret_cast<uint4*>(tile + (col >> 6) * 4096 + lane * 128 + ((gr ^ (lane & 7)) << 4));
+          *dst = make_uint4(wd[4 * k], wd[4 * k + 1], wd[4 * k + 2], wd[4 * k + 3]);
         }
+      }
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) tma_store_3d(&p.tm_out, tile + h * 4096, h * 64, qb * 128 + q4 * 32, bh);
+        bulk_commit();
       }
       if (store && p.lse)
         p.lse[static_cast<size_t>(bh) * p.N + qrow] =
             ltot > 0.f ? (m + __log2f(ltot) - kLog2_448) * kLn2 : -INFINITY;
       tc_fence_before();
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncthreads();
@@ -718,6 +750,18 @@ bool make_map(CUtensorMap* m, const void* base, int row_bytes, int N, int BH, CU
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_out_map(CUtensorMap* m, void* base, int d, int N, int BH) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(N)};
+  cuuint32_t box[3] = {64u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 CUtensorMapSwizzle swizzle_for(int row_bytes) {
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                           : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -741,7 +785,7 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   const int qk_row = C::kQKRow;
   if (!make_map(&p.tm_q, a.q, qk_row, a.N, BH, swizzle_for(qk_row)) ||
       !make_map(&p.tm_k, a.k, qk_row, a.N, BH, swizzle_for(qk_row)) ||
-      !make_map(&p.tm_v, a.v, D, a.N, BH, swizzle_for(D)))
+      !make_map(&p.tm_v, a.v, D, a.N, BH, swizzle_for(D)) || !make_out_map(&p.tm_out, a.out, D, a.N, BH))
     return cudaErrorNotSupported;
   p.q_sf = a.q_sf;
   p.k_sf = a.k_sf;
