@@ -160,3 +160,19 @@ def test_full_video_sta_fp8():
     # corner tile (fewest neighbours), an interior tile, the last tile
     _full("video_sta_fp8", lambda n: [0, 3 * (1 * 60 + 2 * 10 + 5), n - 1], lambda bh: [bh // 2],
           tile_mask=plan.to("cuda"), key_blocks=kb)
+
+
+# ----------------------------------------------------- sequence-sweep shapes
+# The sweep's configurations differ from one another only in N, d, the mask,
+# the QK format and the batch count (B * H * N = 2^22); each head is an
+# independent problem, so two heads at the sweep's full N, drawn with the
+# sweep's recipe, cover a configuration. Sampled query blocks: first, middle,
+# last.
+@pytest.mark.parametrize("N,d,causal,fmt", [(16384, 64, True, "fp8"), (16384, 64, False, "nvfp4"),
+                                            (131072, 128, False, "nvfp4"), (131072, 128, True, "fp8")])
+def test_sweep_shape_sampled(N, d, causal, fmt):
+    w = next(x for x in workloads.sweep_workloads() if x.N == N and x.d == d and x.causal == causal
+             and x.qk_format == fmt)
+    q, k, v = workloads.make_qkv(w, heads=2, batch=1)
+    nblk = (N + 127) // 128
+    _check_case(q, k, v, fmt, causal=causal, qblocks=[0, nblk // 2, nblk - 1], heads=[0, 1])
