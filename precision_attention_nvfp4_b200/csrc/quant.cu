@@ -219,9 +219,14 @@ __global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __re
   __shared__ float red[kThreads / 32];
   float m = 0.f;
   bool bad = false;
-  for (size_t c = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x; c < nchunks;
-       c += static_cast<size_t>(gridDim.x) * kThreads)
-    m = fmaxf(m, amax8(x[c], &bad));
+  const size_t stride = static_cast<size_t>(gridDim.x) * kThreads;
+  size_t c = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x;
+  // four loads in flight per thread
+  for (; c + 3 * stride < nchunks; c += 4 * stride) {
+    const uint4 v0 = x[c], v1 = x[c + stride], v2 = x[c + 2 * stride], v3 = x[c + 3 * stride];
+    m = fmaxf(fmaxf(m, amax8(v0, &bad)), fmaxf(amax8(v1, &bad), fmaxf(amax8(v2, &bad), amax8(v3, &bad))));
+  }
+  for (; c < nchunks; c += stride) m = fmaxf(m, amax8(x[c], &bad));
   if (bad && nonfinite) atomicExch(nonfinite, 1);
   m = block_max(m, red);
   if (threadIdx.x == 0) atomicMax(reinterpret_cast<int*>(amax_out), __float_as_int(m));
