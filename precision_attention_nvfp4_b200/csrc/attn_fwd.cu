@@ -78,7 +78,9 @@ struct Cfg {
   static constexpr uint32_t kVSwz = D == 128 ? 2u : 4u;
   static constexpr uint32_t kVSbo = 8 * D;
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
-  static constexpr int kPolyPairs = 4;                    // of 16 exp2 pairs per 32-score chunk
+  // of the 16 exp2 pairs of a 32-score chunk, how many take the FMA-pipe
+  // polynomial (measured best: 3 next to the cheaper FP4 QK^T, 4 with FP8)
+  static constexpr int kPolyPairs = FP4 ? 3 : 4;
   static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
   // P buffers, 32 columns each (128 E4M3 keys). As many as K/V stages: the
   // S of block g needs K stage g % kStages, which is refilled only after the
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   uint64_t* o_ready = bars + C::kBarOReady;    // [g % kStages], 4 arrivals: correction warps
   uint64_t* o_done = bars + C::kBarODone;      // [g % kStages]: PV of block g completed
   uint64_t* drain = bars + C::kBarDrain;       // [2]: PV issuer, S issuer
-  uint64_t* a_bar = bars + C::kBarA;           // [quarter][g % kStages]: rescale factor published (warpgroup 0)
+  uint64_t* a_bar = bars + C::kBarA;           // [quarter][g % kStages]: rescale factor published (warpgroup g % 2)
   uint64_t* fin_bar = bars + C::kBarFin;       // [item parity], 8 arrivals: per-item (l, m) published
   uint64_t* fin_free = bars + C::kBarFinFree;  // [item parity], 4 arrivals: correction warps read them
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
@@ -544,7 +546,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // Rescale factor of O and of the row sum; a row that has seen no key
         // yet (m_prev = -inf) has O = 0 and l = 0, scaled by 2^-inf = 0.
         const float alpha = m_prev == m_new ? 1.f : ex2_approx(m_prev - m_use);
-        if (w == 0) {
+        // the two warpgroups take turns publishing it, which keeps their
+        // per-block work equal
+        if (w == (g & 1)) {
           ax[(g % kStages) * 128 + row] = alpha;
           warp_arrive(a_bar + q4 * kStages + g % kStages);
         }
