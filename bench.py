@@ -148,10 +148,15 @@ class ClockSampler:
 def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks, budget_s: float = 0.0):
     """Run the oracle (as it stands) on a bounded sample; returns (flops,
     seconds, (head, query block) pairs done). With budget_s > 0 the sample
-    stops after the first pair that ends past the budget."""
+    stops after the first pair that ends past the budget. q, k, v are in the
+    order the kernel computes in (tile-major for sliding-tile workloads)."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import parity
     from oracle import attention as oatt
+    kb = None
+    if w.sparse:
+        from oracle import sta
+        kb = sta.block_lists(w.video, w.sta_tile, w.sta_window)
     t0 = time.perf_counter()
     flops = 0.0
     done = []
@@ -159,8 +164,11 @@ def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks, budget_s: 
         qh, kh, vh = parity.oracle_operands(q, k, v, w.qk_format, [h])
         for qb in qblocks:
             rows = np.arange(qb * 128, min(w.N, qb * 128 + 128))
-            oatt.attention_rows(qh[0], kh[0], vh[0], rows, causal=w.causal)
-            keys = (rows + 1) if w.causal else np.full(len(rows), w.N)
+            oatt.attention_rows(qh[0], kh[0], vh[0], rows, causal=w.causal, key_blocks=kb)
+            if kb is not None:
+                keys = np.full(len(rows), 128 * len(kb[qb]))
+            else:
+                keys = (rows + 1) if w.causal else np.full(len(rows), w.N)
             flops += float(np.sum(4.0 * keys * w.d))
             done.append((h, qb))
             if budget_s > 0 and time.perf_counter() - t0 > budget_s:
@@ -226,9 +234,13 @@ def aggregate_value(per_rank_flops: float, world: int, ms_per_step: float) -> fl
 
 
 def config_dict(w):
-    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "qk": w.qk_format, "pv": "e4m3", "sparse": w.sparse,
-            "l2": "inputs larger than L2 (bf16 Q,K,V of the step exceed 126 MB)"}
+    c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+         "qk": w.qk_format, "pv": "e4m3", "sparse": w.sparse,
+         "l2": "inputs larger than L2 (bf16 Q,K,V of the step exceed 126 MB)"}
+    if w.sparse:
+        c["tokens"] = ("raster (time-major) bf16 in and out; the tile-major permutation runs inside the "
+                       "quantize kernels and the attention epilogue")
+    return c
 
 
 def time_cuda(fn, min_runs: int = 5, budget_ms: float = 1500.0) -> float:
@@ -349,24 +361,27 @@ def main():
     def rank_max(x: float) -> float:
         return max_over_ranks(dist, x, "cuda")
 
-    # weak scaling: every rank runs one full batch of the workload
-    q_h, k_h, v_h = workloads.make_qkv(w)
-    q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
-    mask = None
+    # weak scaling: every rank runs one full batch of the workload. Video
+    # tokens of the sliding-tile workload stay in raster order: the fused
+    # path permutes them inside the kernels.
+    mask, video = None, None
     if w.sparse:
         tg = tuple(a // b for a, b in zip(w.video, w.sta_tile))
         mask = fp.sta_plan(tg, w.sta_tile, w.sta_window).to("cuda")
+        video = fp.VideoLayout(w.video, w.sta_tile)
+    q_h, k_h, v_h = workloads.make_qkv(w, tile_major=video is None)
+    q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
     stream = torch.cuda.current_stream()
 
     def step(ev_pair=None):
         if w.qk_format == "nvfp4":
-            qq, kq = fp.quantize_nvfp4(q), fp.quantize_nvfp4(k)
+            qq, kq = fp.quantize_nvfp4(q, video=video), fp.quantize_nvfp4(k, video=video)
         else:
-            qq, kq = fp.quantize_fp8(q, "tile128"), fp.quantize_fp8(k, "tile128")
-        vq = fp.quantize_fp8(v, "channel")
+            qq, kq = fp.quantize_fp8(q, "tile128", video=video), fp.quantize_fp8(k, "tile128", video=video)
+        vq = fp.quantize_fp8(v, "channel", video=video)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask)
+        out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask, video=video)
         if ev_pair is not None:
             ev_pair[1].record(stream)
         return out
@@ -419,14 +434,14 @@ def main():
         out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
         lse_h = torch.empty(q_h.shape[:3], dtype=torch.float32, pin_memory=True)
         fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
-                     lse_host=lse_h)
+                     lse_host=lse_h, video=video)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         e0.record(stream)
         for _ in range(args.e2e_steps):
             fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
-                         lse_host=lse_h)
+                         lse_host=lse_h, video=video)
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = rank_max(e0.elapsed_time(e1) / args.e2e_steps)
@@ -442,7 +457,8 @@ def main():
         bh = w.B * w.H
         heads = list(range(0, bh, max(1, bh // 32)))
         qblocks = sorted({nblk - 1, (3 * nblk) // 4, nblk // 2, nblk // 4, 1, 0}, reverse=True)
-        f, s, done = cpu_oracle_sample(w, q_h, k_h, v_h, heads, qblocks, budget_s=15.0)
+        qo, ko, vo = (q_h, k_h, v_h) if video is None else workloads.make_qkv(w)
+        f, s, done = cpu_oracle_sample(w, qo, ko, vo, heads, qblocks, budget_s=15.0)
         cpu = {"value": f / s / 1e12, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
                "sample": f"{len(done)} (batch*head, 128-query block) pairs of {w.name}: heads "
                          f"{sorted(set(h for h, _ in done))} x query blocks {qblocks} in that order (fp64 "

@@ -213,6 +213,73 @@ fpattn_status fpattn_fwd(const fpattn_tensor* q, const fpattn_tensor* k, const f
                          int32_t causal, void* out, float* lse, fpattn_stream_t stream);
 
 /*
+ * Video token order (FPSAttention page, section 2.2: attention over 3D tiles
+ * of the video token grid; section 3.3, item 1: contiguous memory access
+ * through a tile transpose).
+ *
+ * A video of T x Hs x W tokens in raster (time-major) order holds token
+ * (t, h, w) in row (t*Hs + h)*W + w of its N = T*Hs*W rows. The attention
+ * kernel works in tile-major order: tiles of tt x th x tw tokens in raster
+ * order over the tile grid, and inside each tile its tokens in raster order
+ * (the order fpattn_sta_plan numbers blocks in). The _video entry points
+ * fuse that permutation into passes that touch the data anyway: the
+ * quantizers read raster-order bf16 and write tile-major codes and scales,
+ * and fpattn_fwd_video reads tile-major codes and writes out and lse in
+ * raster order. No pass or buffer of its own is needed.
+ *
+ * Supported when T, Hs and W are multiples of tt, th and tw, the tile volume
+ * tt*th*tw is a multiple of 128, and every 32 consecutive tile-major tokens
+ * of a tile form one box of the grid, that is: tw is a multiple of 32; or 32
+ * is a multiple of tw and th a multiple of 32/tw; or 32 is a multiple of
+ * th*tw and tt a multiple of 32/(th*tw). Tiles (6,8,8), (4,8,8) and
+ * (6,16,16) qualify. Other tiles give FPATTN_ERR_UNSUPPORTED; a layout with
+ * T*Hs*W != N gives FPATTN_ERR_INVALID_ARG.
+ */
+typedef struct {
+  int32_t T, Hs, W;    /* grid, in tokens */
+  int32_t tt, th, tw;  /* tile, in tokens */
+} fpattn_video_layout;
+
+/*
+ * HOST-only check of a video layout for N tokens, with no CUDA call:
+ * FPATTN_OK when the _video entry points accept it, FPATTN_ERR_UNSUPPORTED
+ * or FPATTN_ERR_INVALID_ARG (NULL, non-positive sizes, T*Hs*W != N) as they
+ * would return.
+ */
+fpattn_status fpattn_video_layout_check(const fpattn_video_layout* layout, int32_t N);
+
+/*
+ * fpattn_quantize_nvfp4 / fpattn_quantize_fp8 for raster-order input: x is
+ * bf16 [B, H, N, d] in raster order of `layout` (HOST pointer to the layout
+ * struct, read during the call); codes, block scales and per-tile scales are
+ * written in tile-major order, exactly as the non-video call would write them
+ * for x permuted to tile-major order. Per-tensor and per-channel scales are
+ * order-free and equal to the non-video call's. Arguments and errors
+ * otherwise as the non-video calls; layout NULL is FPATTN_ERR_INVALID_ARG.
+ */
+fpattn_status fpattn_quantize_nvfp4_video(const fpattn_tensor* x, const fpattn_video_layout* layout,
+                                          const float* static_amax, uint8_t* codes, uint8_t* block_sf,
+                                          float* tensor_scale, int32_t* nonfinite_flag,
+                                          fpattn_stream_t stream);
+fpattn_status fpattn_quantize_fp8_video(const fpattn_tensor* x, const fpattn_video_layout* layout,
+                                        int32_t granularity, uint8_t* codes, float* scales,
+                                        int32_t* nonfinite_flag, fpattn_stream_t stream);
+
+/*
+ * fpattn_fwd with q, k, v (and their block or tile scales) in tile-major
+ * order of `layout` (HOST pointer), and out [B, H, N, d] and lse [B, H, N]
+ * written in raster order: row r of the tile-major computation lands in the
+ * raster row of the same token. tile_mask, if given, is over tile-major
+ * blocks (as fpattn_sta_plan writes it). Results equal fpattn_fwd's,
+ * permuted. Arguments and errors otherwise as fpattn_fwd; layout NULL is
+ * FPATTN_ERR_INVALID_ARG.
+ */
+fpattn_status fpattn_fwd_video(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                               const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask,
+                               int32_t causal, const fpattn_video_layout* layout, void* out, float* lse,
+                               fpattn_stream_t stream);
+
+/*
  * Reads (and, if clear != 0, resets) the library's device error word on the
  * current device. Synchronizes `stream`. Returns FPATTN_OK when no bounded
  * wait has expired, FPATTN_ERR_TIMEOUT otherwise; *code (if non-NULL)

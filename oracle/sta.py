@@ -74,6 +74,17 @@ def token_coords_tile_major(grid, tile) -> np.ndarray:
     return np.array(coords, dtype=np.int64)
 
 
+def raster_index_of_tile_major(grid, tile) -> np.ndarray:
+    """perm[i] = raster (time-major) row of the token at tile-major position i.
+
+    Raster order numbers token (t, h, w) of a T x Hs x W grid as
+    (t * Hs + h) * W + w. FPSAttention page, section 3.3, item 1 (contiguous
+    memory through a tile transpose): x_tile_major = x_raster[perm].
+    """
+    coords = token_coords_tile_major(grid, tile)
+    return (coords[:, 0] * grid[1] + coords[:, 1]) * grid[2] + coords[:, 2]
+
+
 def token_mask(grid, tile, window, query_pos: np.ndarray) -> np.ndarray:
     """Brute-force token-level mask: rows = query positions, cols = all keys.
 

@@ -8,11 +8,16 @@ computes any part of the method on the host.
 Public calls
   quantize_nvfp4(x)            -> Nvfp4Tensor(codes, block_sf, tensor_scale)
   quantize_fp8(x, granularity) -> Fp8Tensor(codes, scales)
+                                  (with video=VideoLayout: x in raster order,
+                                  codes and scales in tile-major order)
   sta_plan(grid, tile, window) -> StaPlan (host CSR over 128-token blocks)
   attention_fwd(q, k, v, ...)  -> (out, lse) on quantized operands
   attention(q, k, v, ...)      -> (out, lse) from bf16 inputs: quantize + fwd;
                                   host (pinned) inputs are copied in and the
-                                  result copied back.
+                                  result copied back. With video=VideoLayout,
+                                  inputs and outputs are in raster order and
+                                  the tile-major permutation happens inside
+                                  the quantize and attention kernels.
 """
 from __future__ import annotations
 
@@ -27,7 +32,7 @@ import torch
 from . import _lib
 from ._lib import FpattnError
 
-__all__ = ["Nvfp4Tensor", "Fp8Tensor", "StaPlan", "quantize_nvfp4", "quantize_fp8", "sta_plan",
+__all__ = ["Nvfp4Tensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_fp8", "sta_plan",
            "attention_fwd", "attention", "device_error", "library", "FpattnError"]
 
 
@@ -53,6 +58,24 @@ def _check_bf16(x: torch.Tensor) -> Tuple[int, int, int, int]:
     return tuple(x.shape)
 
 
+@dataclasses.dataclass(frozen=True)
+class VideoLayout:
+    """A T x Hs x W video token grid cut into tt x th x tw tiles.
+
+    Raster order holds token (t, h, w) in row (t*Hs + h)*W + w; tile-major
+    order lists tiles in raster order and each tile's tokens in raster order.
+    """
+    grid: Tuple[int, int, int]
+    tile: Tuple[int, int, int]
+
+    def c(self) -> _lib.VideoLayout:
+        return _lib.VideoLayout(*(int(v) for v in self.grid), *(int(v) for v in self.tile))
+
+
+def _video_ref(video: Optional[VideoLayout]):
+    return None if video is None else ctypes.byref(video.c())
+
+
 @dataclasses.dataclass
 class Nvfp4Tensor:
     codes: torch.Tensor         # uint8 [B, H, N, d/2], packed E2M1
@@ -70,21 +93,27 @@ class Fp8Tensor:
 
 
 def quantize_nvfp4(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
-                   nonfinite_flag: Optional[torch.Tensor] = None) -> Nvfp4Tensor:
+                   nonfinite_flag: Optional[torch.Tensor] = None,
+                   video: Optional[VideoLayout] = None) -> Nvfp4Tensor:
     B, H, N, d = _check_bf16(x)
     lib = library()
     codes = torch.empty((B, H, N, d // 2), dtype=torch.uint8, device=x.device)
     sf = torch.empty(lib.fpattn_nvfp4_sf_bytes(B, H, N, d), dtype=torch.uint8, device=x.device)
     ts = torch.empty(1, dtype=torch.float32, device=x.device)
-    st = lib.fpattn_quantize_nvfp4(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), _ptr(static_amax),
-                                   codes.data_ptr(), sf.data_ptr(), ts.data_ptr(), _ptr(nonfinite_flag),
-                                   _stream())
-    _lib.check(st, "fpattn_quantize_nvfp4")
+    xd = ctypes.byref(_desc(x, _lib.BF16, B, H, N, d))
+    if video is None:
+        st = lib.fpattn_quantize_nvfp4(xd, _ptr(static_amax), codes.data_ptr(), sf.data_ptr(), ts.data_ptr(),
+                                       _ptr(nonfinite_flag), _stream())
+    else:
+        st = lib.fpattn_quantize_nvfp4_video(xd, _video_ref(video), _ptr(static_amax), codes.data_ptr(),
+                                             sf.data_ptr(), ts.data_ptr(), _ptr(nonfinite_flag), _stream())
+    _lib.check(st, "fpattn_quantize_nvfp4" + ("_video" if video is not None else ""))
     return Nvfp4Tensor(codes, sf, ts, (B, H, N, d))
 
 
 def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
-                 nonfinite_flag: Optional[torch.Tensor] = None) -> Fp8Tensor:
+                 nonfinite_flag: Optional[torch.Tensor] = None,
+                 video: Optional[VideoLayout] = None) -> Fp8Tensor:
     B, H, N, d = _check_bf16(x)
     lib = library()
     codes = torch.empty((B, H, N, d), dtype=torch.uint8, device=x.device)
@@ -94,9 +123,13 @@ def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
         g, scales = _lib.FP8_CHANNEL, torch.empty((B, H, d), dtype=torch.float32, device=x.device)
     else:
         raise ValueError("granularity must be 'tile128' or 'channel'")
-    st = lib.fpattn_quantize_fp8(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), g, codes.data_ptr(),
-                                 scales.data_ptr(), _ptr(nonfinite_flag), _stream())
-    _lib.check(st, "fpattn_quantize_fp8")
+    xd = ctypes.byref(_desc(x, _lib.BF16, B, H, N, d))
+    if video is None:
+        st = lib.fpattn_quantize_fp8(xd, g, codes.data_ptr(), scales.data_ptr(), _ptr(nonfinite_flag), _stream())
+    else:
+        st = lib.fpattn_quantize_fp8_video(xd, _video_ref(video), g, codes.data_ptr(), scales.data_ptr(),
+                                           _ptr(nonfinite_flag), _stream())
+    _lib.check(st, "fpattn_quantize_fp8" + ("_video" if video is not None else ""))
     return Fp8Tensor(codes, scales, granularity, (B, H, N, d))
 
 
@@ -151,11 +184,14 @@ def sta_plan(tile_grid: Sequence[int], tile: Sequence[int], window: Sequence[int
 
 def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
-                  lse: Optional[torch.Tensor] = None, return_lse: bool = True):
+                  lse: Optional[torch.Tensor] = None, return_lse: bool = True,
+                  video: Optional[VideoLayout] = None):
     """Fused attention on quantized operands.
 
     q, k: both Nvfp4Tensor or both Fp8Tensor (tile128); v: Fp8Tensor (channel).
-    Returns (out bf16 [B,H,N,d], lse float32 [B,H,N] or None).
+    Returns (out bf16 [B,H,N,d], lse float32 [B,H,N] or None). With ``video``
+    the operands are in tile-major order and out / lse come back in raster
+    order.
     """
     B, H, N, d = v.shape
     lib = library()
@@ -177,16 +213,21 @@ def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Option
     if lse is None and return_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=v.codes.device)
     mask = ctypes.byref(tile_mask.desc()) if tile_mask is not None else None
-    st = lib.fpattn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(sc), mask,
-                        1 if causal else 0, out.data_ptr(), _ptr(lse), _stream())
-    _lib.check(st, "fpattn_fwd")
+    if video is None:
+        st = lib.fpattn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(sc), mask,
+                            1 if causal else 0, out.data_ptr(), _ptr(lse), _stream())
+    else:
+        st = lib.fpattn_fwd_video(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(sc), mask,
+                                  1 if causal else 0, _video_ref(video), out.data_ptr(), _ptr(lse), _stream())
+    _lib.check(st, "fpattn_fwd" + ("_video" if video is not None else ""))
     return out, lse
 
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: str = "nvfp4",
               causal: bool = False, tile_mask: Optional[DeviceTileMask] = None, softmax_scale: float = 0.0,
               return_lse: bool = True, device: Optional[torch.device] = None,
-              out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None):
+              out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None,
+              video: Optional[VideoLayout] = None):
     """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
 
     CUDA inputs stay where they are. Host inputs (ideally pinned) are copied
@@ -201,14 +242,14 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
         k = k.to(dev, non_blocking=True)
         v = v.to(dev, non_blocking=True)
     if qk_format == "nvfp4":
-        qq, kq = quantize_nvfp4(q), quantize_nvfp4(k)
+        qq, kq = quantize_nvfp4(q, video=video), quantize_nvfp4(k, video=video)
     elif qk_format == "fp8":
-        qq, kq = quantize_fp8(q, "tile128"), quantize_fp8(k, "tile128")
+        qq, kq = quantize_fp8(q, "tile128", video=video), quantize_fp8(k, "tile128", video=video)
     else:
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
-    vq = quantize_fp8(v, "channel")
+    vq = quantize_fp8(v, "channel", video=video)
     out, lse = attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
-                             return_lse=return_lse)
+                             return_lse=return_lse, video=video)
     if host:
         out_h = out_host if out_host is not None else torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         out_h.copy_(out, non_blocking=True)

@@ -28,6 +28,11 @@ class TileMask(ctypes.Structure):
                 ("col_idx", ctypes.c_void_p), ("row_order", ctypes.c_void_p)]
 
 
+class VideoLayout(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("Hs", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("tt", ctypes.c_int32), ("th", ctypes.c_int32), ("tw", ctypes.c_int32)]
+
+
 _P = ctypes.POINTER
 _SIGNATURES = {
     "fpattn_nvfp4_sf_bytes": (ctypes.c_size_t, [ctypes.c_int32] * 4),
@@ -35,10 +40,19 @@ _SIGNATURES = {
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "fpattn_quantize_fp8": (ctypes.c_int, [_P(Tensor), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_void_p]),
+    "fpattn_video_layout_check": (ctypes.c_int, [_P(VideoLayout), ctypes.c_int32]),
+    "fpattn_quantize_nvfp4_video": (ctypes.c_int, [_P(Tensor), _P(VideoLayout), ctypes.c_void_p, ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                   ctypes.c_void_p]),
+    "fpattn_quantize_fp8_video": (ctypes.c_int, [_P(Tensor), _P(VideoLayout), ctypes.c_int32, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "fpattn_sta_plan": (ctypes.c_int, [ctypes.c_int32] * 9 + [ctypes.c_void_p] * 3 +
                         [ctypes.c_size_t, _P(ctypes.c_int32), _P(ctypes.c_int32)]),
     "fpattn_fwd": (ctypes.c_int, [_P(Tensor), _P(Tensor), _P(Tensor), _P(Scales), _P(TileMask),
                                   ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "fpattn_fwd_video": (ctypes.c_int, [_P(Tensor), _P(Tensor), _P(Tensor), _P(Scales), _P(TileMask),
+                                        ctypes.c_int32, _P(VideoLayout), ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p]),
     "fpattn_device_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, _P(ctypes.c_int32)]),
     "fpattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fpattn_version": (ctypes.c_char_p, []),

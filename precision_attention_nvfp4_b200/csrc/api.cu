@@ -38,6 +38,111 @@ fpattn_status check_tensor(const fpattn_tensor* t, int dtype) {
   return FPATTN_OK;
 }
 
+// Validates a video layout for N tokens and converts it; on success *tm
+// receives the tile-major -> raster map.
+fpattn_status check_layout(const fpattn_video_layout* l, int N, fpattn::VideoLayout* v, fpattn::TokenMap* tm) {
+  if (!l) return FPATTN_ERR_INVALID_ARG;
+  if (l->T <= 0 || l->Hs <= 0 || l->W <= 0 || l->tt <= 0 || l->th <= 0 || l->tw <= 0) return FPATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(l->T) * l->Hs * l->W != N) return FPATTN_ERR_INVALID_ARG;
+  if (l->T % l->tt != 0 || l->Hs % l->th != 0 || l->W % l->tw != 0) return FPATTN_ERR_UNSUPPORTED;
+  *v = fpattn::VideoLayout{l->T, l->Hs, l->W, l->tt, l->th, l->tw};
+  int bw, bh, bt;
+  if (!fpattn::video_chunk_box(*v, bw, bh, bt)) return FPATTN_ERR_UNSUPPORTED;
+  *tm = fpattn::make_token_map(l->T, l->Hs, l->W, l->tt, l->th, l->tw);
+  return FPATTN_OK;
+}
+
+fpattn_status quantize_nvfp4(const fpattn_tensor* x, const fpattn_video_layout* layout, const float* static_amax,
+                             uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int32_t* nonfinite_flag,
+                             fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  if (layout && (s = check_layout(layout, x->N, &vl, &tm)) != FPATTN_OK) return s;
+  if (!codes || !block_sf || !tensor_scale) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(block_sf) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+    return FPATTN_ERR_ALIGNMENT;
+  return from_cuda(fpattn::launch_quantize_nvfp4(x->data, x->B * x->H, x->N, x->d, static_amax, codes, block_sf,
+                                                 tensor_scale, nonfinite_flag, layout ? &tm : nullptr,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fpattn_status quantize_fp8(const fpattn_tensor* x, const fpattn_video_layout* layout, int32_t granularity,
+                           uint8_t* codes, float* scales, int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  if (layout && (s = check_layout(layout, x->N, &vl, &tm)) != FPATTN_OK) return s;
+  if (!codes || !scales) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FPATTN_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = x->B * x->H;
+  const fpattn::TokenMap* tmp = layout ? &tm : nullptr;
+  if (granularity == FPATTN_FP8_TILE128)
+    return from_cuda(
+        fpattn::launch_quantize_fp8_tile(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, tmp, st));
+  if (granularity == FPATTN_FP8_CHANNEL)
+    return from_cuda(
+        fpattn::launch_quantize_fp8_channel(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, tmp, st));
+  return FPATTN_ERR_INVALID_ARG;
+}
+
+fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                  const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask, int32_t causal,
+                  const fpattn_video_layout* layout, void* out, float* lse, fpattn_stream_t stream) {
+  if (!q || !k || !v || !scales || !out) return FPATTN_ERR_INVALID_ARG;
+  const int qk_dtype = q->dtype;
+  if (qk_dtype != FPATTN_NVFP4 && qk_dtype != FPATTN_E4M3) return FPATTN_ERR_UNSUPPORTED;
+  fpattn_status s;
+  if ((s = check_tensor(q, qk_dtype)) != FPATTN_OK) return s;
+  if ((s = check_tensor(k, qk_dtype)) != FPATTN_OK) return s;
+  if ((s = check_tensor(v, FPATTN_E4M3)) != FPATTN_OK) return s;
+  if (k->B != q->B || k->H != q->H || k->N != q->N || k->d != q->d || v->B != q->B || v->H != q->H ||
+      v->N != q->N || v->d != q->d)
+    return FPATTN_ERR_INVALID_ARG;
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  if (layout && (s = check_layout(layout, q->N, &vl, &tm)) != FPATTN_OK) return s;
+  if (!aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FPATTN_ERR_ALIGNMENT;
+  if (!scales->q_scale || !scales->k_scale || !scales->v_scale) return FPATTN_ERR_INVALID_ARG;
+  const bool fp4 = qk_dtype == FPATTN_NVFP4;
+  if (fp4 && (!scales->q_block_sf || !scales->k_block_sf)) return FPATTN_ERR_INVALID_ARG;
+  if (fp4 && (!aligned16(scales->q_block_sf) || !aligned16(scales->k_block_sf))) return FPATTN_ERR_ALIGNMENT;
+  // P is stored in E4M3 at the fixed scale 1/448.
+  if (!(scales->p_scale > 0.f) || std::abs(scales->p_scale * 448.f - 1.f) > 1e-6f) return FPATTN_ERR_INVALID_ARG;
+  if (!(scales->softmax_scale >= 0.f) || scales->softmax_scale > 1e30f) return FPATTN_ERR_INVALID_ARG;
+  const int nblk = (q->N + 127) / 128;
+  if (tile_mask) {
+    if (tile_mask->nblk_q != nblk || !tile_mask->row_ptr || !tile_mask->col_idx || tile_mask->nnz < 0)
+      return FPATTN_ERR_INVALID_ARG;
+  }
+  AttnArgs a{};
+  a.q = q->data;
+  a.k = k->data;
+  a.v = v->data;
+  a.q_sf = fp4 ? scales->q_block_sf : nullptr;
+  a.k_sf = fp4 ? scales->k_block_sf : nullptr;
+  a.q_scale = scales->q_scale;
+  a.k_scale = scales->k_scale;
+  a.v_scale = scales->v_scale;
+  a.out = out;
+  a.lse = lse;
+  a.row_ptr = tile_mask ? tile_mask->row_ptr : nullptr;
+  a.col_idx = tile_mask ? tile_mask->col_idx : nullptr;
+  a.row_order = tile_mask ? tile_mask->row_order : nullptr;
+  a.B = q->B;
+  a.H = q->H;
+  a.N = q->N;
+  a.d = q->d;
+  a.qk_fp4 = fp4;
+  a.causal = causal != 0;
+  a.softmax_scale = scales->softmax_scale > 0.f ? scales->softmax_scale : 1.0f / std::sqrt(static_cast<float>(q->d));
+  a.video = layout ? &vl : nullptr;
+  return from_cuda(fpattn::launch_attn_fwd(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace
 
 extern "C" {
@@ -50,30 +155,32 @@ size_t fpattn_nvfp4_sf_bytes(int32_t B, int32_t H, int32_t N, int32_t d) {
 fpattn_status fpattn_quantize_nvfp4(const fpattn_tensor* x, const float* static_amax, uint8_t* codes,
                                     uint8_t* block_sf, float* tensor_scale, int32_t* nonfinite_flag,
                                     fpattn_stream_t stream) {
-  fpattn_status s = check_tensor(x, FPATTN_BF16);
-  if (s != FPATTN_OK) return s;
-  if (!codes || !block_sf || !tensor_scale) return FPATTN_ERR_INVALID_ARG;
-  if (!aligned16(codes) || !aligned16(block_sf) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
-    return FPATTN_ERR_ALIGNMENT;
-  return from_cuda(fpattn::launch_quantize_nvfp4(x->data, x->B * x->H, x->N, x->d, static_amax, codes, block_sf,
-                                                 tensor_scale, nonfinite_flag,
-                                                 reinterpret_cast<cudaStream_t>(stream)));
+  return quantize_nvfp4(x, nullptr, static_amax, codes, block_sf, tensor_scale, nonfinite_flag, stream);
 }
 
 fpattn_status fpattn_quantize_fp8(const fpattn_tensor* x, int32_t granularity, uint8_t* codes, float* scales,
                                   int32_t* nonfinite_flag, fpattn_stream_t stream) {
-  fpattn_status s = check_tensor(x, FPATTN_BF16);
-  if (s != FPATTN_OK) return s;
-  if (!codes || !scales) return FPATTN_ERR_INVALID_ARG;
-  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FPATTN_ERR_ALIGNMENT;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = x->B * x->H;
-  if (granularity == FPATTN_FP8_TILE128)
-    return from_cuda(fpattn::launch_quantize_fp8_tile(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, st));
-  if (granularity == FPATTN_FP8_CHANNEL)
-    return from_cuda(
-        fpattn::launch_quantize_fp8_channel(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, st));
-  return FPATTN_ERR_INVALID_ARG;
+  return quantize_fp8(x, nullptr, granularity, codes, scales, nonfinite_flag, stream);
+}
+
+fpattn_status fpattn_video_layout_check(const fpattn_video_layout* layout, int32_t N) {
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  return check_layout(layout, N, &vl, &tm);
+}
+
+fpattn_status fpattn_quantize_nvfp4_video(const fpattn_tensor* x, const fpattn_video_layout* layout,
+                                          const float* static_amax, uint8_t* codes, uint8_t* block_sf,
+                                          float* tensor_scale, int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  if (!layout) return FPATTN_ERR_INVALID_ARG;
+  return quantize_nvfp4(x, layout, static_amax, codes, block_sf, tensor_scale, nonfinite_flag, stream);
+}
+
+fpattn_status fpattn_quantize_fp8_video(const fpattn_tensor* x, const fpattn_video_layout* layout,
+                                        int32_t granularity, uint8_t* codes, float* scales, int32_t* nonfinite_flag,
+                                        fpattn_stream_t stream) {
+  if (!layout) return FPATTN_ERR_INVALID_ARG;
+  return quantize_fp8(x, layout, granularity, codes, scales, nonfinite_flag, stream);
 }
 
 fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, int32_t th, int32_t tw, int32_t wt,
@@ -148,51 +255,14 @@ fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, in
 fpattn_status fpattn_fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
                          const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask, int32_t causal,
                          void* out, float* lse, fpattn_stream_t stream) {
-  if (!q || !k || !v || !scales || !out) return FPATTN_ERR_INVALID_ARG;
-  const int qk_dtype = q->dtype;
-  if (qk_dtype != FPATTN_NVFP4 && qk_dtype != FPATTN_E4M3) return FPATTN_ERR_UNSUPPORTED;
-  fpattn_status s;
-  if ((s = check_tensor(q, qk_dtype)) != FPATTN_OK) return s;
-  if ((s = check_tensor(k, qk_dtype)) != FPATTN_OK) return s;
-  if ((s = check_tensor(v, FPATTN_E4M3)) != FPATTN_OK) return s;
-  if (k->B != q->B || k->H != q->H || k->N != q->N || k->d != q->d || v->B != q->B || v->H != q->H ||
-      v->N != q->N || v->d != q->d)
-    return FPATTN_ERR_INVALID_ARG;
-  if (!aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FPATTN_ERR_ALIGNMENT;
-  if (!scales->q_scale || !scales->k_scale || !scales->v_scale) return FPATTN_ERR_INVALID_ARG;
-  const bool fp4 = qk_dtype == FPATTN_NVFP4;
-  if (fp4 && (!scales->q_block_sf || !scales->k_block_sf)) return FPATTN_ERR_INVALID_ARG;
-  if (fp4 && (!aligned16(scales->q_block_sf) || !aligned16(scales->k_block_sf))) return FPATTN_ERR_ALIGNMENT;
-  // P is stored in E4M3 at the fixed scale 1/448.
-  if (!(scales->p_scale > 0.f) || std::abs(scales->p_scale * 448.f - 1.f) > 1e-6f) return FPATTN_ERR_INVALID_ARG;
-  if (!(scales->softmax_scale >= 0.f) || scales->softmax_scale > 1e30f) return FPATTN_ERR_INVALID_ARG;
-  const int nblk = (q->N + 127) / 128;
-  if (tile_mask) {
-    if (tile_mask->nblk_q != nblk || !tile_mask->row_ptr || !tile_mask->col_idx || tile_mask->nnz < 0)
-      return FPATTN_ERR_INVALID_ARG;
-  }
-  AttnArgs a{};
-  a.q = q->data;
-  a.k = k->data;
-  a.v = v->data;
-  a.q_sf = fp4 ? scales->q_block_sf : nullptr;
-  a.k_sf = fp4 ? scales->k_block_sf : nullptr;
-  a.q_scale = scales->q_scale;
-  a.k_scale = scales->k_scale;
-  a.v_scale = scales->v_scale;
-  a.out = out;
-  a.lse = lse;
-  a.row_ptr = tile_mask ? tile_mask->row_ptr : nullptr;
-  a.col_idx = tile_mask ? tile_mask->col_idx : nullptr;
-  a.row_order = tile_mask ? tile_mask->row_order : nullptr;
-  a.B = q->B;
-  a.H = q->H;
-  a.N = q->N;
-  a.d = q->d;
-  a.qk_fp4 = fp4;
-  a.causal = causal != 0;
-  a.softmax_scale = scales->softmax_scale > 0.f ? scales->softmax_scale : 1.0f / std::sqrt(static_cast<float>(q->d));
-  return from_cuda(fpattn::launch_attn_fwd(a, reinterpret_cast<cudaStream_t>(stream)));
+  return fwd(q, k, v, scales, tile_mask, causal, nullptr, out, lse, stream);
+}
+
+fpattn_status fpattn_fwd_video(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                               const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask, int32_t causal,
+                               const fpattn_video_layout* layout, void* out, float* lse, fpattn_stream_t stream) {
+  if (!layout) return FPATTN_ERR_INVALID_ARG;
+  return fwd(q, k, v, scales, tile_mask, causal, layout, out, lse, stream);
 }
 
 fpattn_status fpattn_device_error(fpattn_stream_t stream, int32_t clear, int32_t* code) {

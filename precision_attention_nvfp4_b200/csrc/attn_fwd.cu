@@ -122,7 +122,10 @@ struct __align__(64) Params {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  CUtensorMap tm_out;  // bf16 [BH][N][d], box 64 x 32 rows, 128-byte swizzle
+  // bf16 out, 64 columns x 32 rows per store, 128-byte swizzle: [BH][N][d],
+  // or for a video layout [BH][T][Hs][W][d] with a box that covers one
+  // 32-row chunk of a tile-major block
+  CUtensorMap tm_out;
   const uint8_t* q_sf;
   const uint8_t* k_sf;
   const float* q_scale;
@@ -136,6 +139,7 @@ struct __align__(64) Params {
   int N, nblk, BH, num_items;
   int causal, sparse;
   float sm_scale_log2;
+  TokenMap tmap;  // on: rows are tile-major, out and lse go to raster positions
 };
 
 struct KList {
@@ -688,12 +692,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       fence_proxy_async_shared();
       __syncwarp();
       if (lane == 0) {
+        if (p.tmap.on) {
+          // the warp's 32 rows form one box of the raster grid; its first
+          // row is the box's corner
+          int t0, h0, w0;
+          tile_major_coords(p.tmap, static_cast<uint32_t>(qb * 128 + q4 * 32), t0, h0, w0);
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_store_3d(&p.tm_out, tile + h * 4096, h * 64, qb * 128 + q4 * 32, bh);
+          for (int h = 0; h < D / 64; ++h) tma_store_5d(&p.tm_out, tile + h * 4096, h * 64, w0, h0, t0, bh);
+        } else {
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) tma_store_3d(&p.tm_out, tile + h * 4096, h * 64, qb * 128 + q4 * 32, bh);
+        }
         bulk_commit();
       }
       if (store && p.lse)
-        p.lse[static_cast<size_t>(bh) * p.N + qrow] =
+        p.lse[static_cast<size_t>(bh) * p.N + to_raster(p.tmap, qrow)] =
             ltot > 0.f ? (m + __log2f(ltot) - kLog2_448) * kLn2 : -INFINITY;
       tc_fence_before();
     }
@@ -766,6 +779,23 @@ bool make_out_map(CUtensorMap* m, void* base, int d, int N, int BH) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [BH][T][Hs][W][d] with a box of 64 channels x one 32-row chunk.
+bool make_out_map_video(CUtensorMap* m, void* base, int d, const VideoLayout& v, int BH) {
+  EncodeTiledFn enc = get_encoder();
+  int bw, bh, bt;
+  if (!enc || !video_chunk_box(v, bw, bh, bt)) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(v.W), static_cast<cuuint64_t>(v.Hs),
+                        static_cast<cuuint64_t>(v.T), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[4] = {row, row * v.W, row * v.W * v.Hs, row * v.W * v.Hs * v.T};
+  cuuint32_t box[5] = {64u, static_cast<cuuint32_t>(bw), static_cast<cuuint32_t>(bh), static_cast<cuuint32_t>(bt),
+                       1u};
+  cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 CUtensorMapSwizzle swizzle_for(int row_bytes) {
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                           : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -789,8 +819,15 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   const int qk_row = C::kQKRow;
   if (!make_map(&p.tm_q, a.q, qk_row, a.N, BH, swizzle_for(qk_row)) ||
       !make_map(&p.tm_k, a.k, qk_row, a.N, BH, swizzle_for(qk_row)) ||
-      !make_map(&p.tm_v, a.v, D, a.N, BH, swizzle_for(D)) || !make_out_map(&p.tm_out, a.out, D, a.N, BH))
+      !make_map(&p.tm_v, a.v, D, a.N, BH, swizzle_for(D)))
     return cudaErrorNotSupported;
+  if (a.video) {
+    if (!make_out_map_video(&p.tm_out, a.out, D, *a.video, BH)) return cudaErrorNotSupported;
+    p.tmap = make_token_map(a.video->T, a.video->Hs, a.video->W, a.video->tt, a.video->th, a.video->tw);
+  } else {
+    if (!make_out_map(&p.tm_out, a.out, D, a.N, BH)) return cudaErrorNotSupported;
+    p.tmap = TokenMap{};
+  }
   p.q_sf = a.q_sf;
   p.k_sf = a.k_sf;
   p.q_scale = a.q_scale;

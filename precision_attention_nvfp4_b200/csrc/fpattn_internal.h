@@ -5,15 +5,44 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "token_map.cuh"
+
 namespace fpattn {
 
+// tmap: NULL when x is already in the order the codes take; otherwise x is
+// read in raster order and the codes are written in tile-major order.
 cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
-                                     int* nonfinite, cudaStream_t st);
+                                     int* nonfinite, const TokenMap* tmap, cudaStream_t st);
 cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
-                                        int* nonfinite, cudaStream_t st);
+                                        int* nonfinite, const TokenMap* tmap, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const float* static_amax,
                                   uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
-                                  cudaStream_t st);
+                                  const TokenMap* tmap, cudaStream_t st);
+
+// Video grid and tile of a tile-major token order.
+struct VideoLayout {
+  int T, Hs, W;
+  int tt, th, tw;
+};
+
+// Box (w, h, t extents) that one 32-row chunk of a 128-token block covers in
+// the raster grid. False when the layout does not cut every such chunk into a
+// box, or the tile volume is not a multiple of 128.
+inline bool video_chunk_box(const VideoLayout& v, int& bw, int& bh, int& bt) {
+  const int plane = v.th * v.tw;
+  if ((v.tt * plane) % 128 != 0) return false;
+  if (v.tw >= 32) {
+    if (v.tw % 32 != 0) return false;
+    bw = 32, bh = 1, bt = 1;
+  } else if (plane >= 32) {
+    if (32 % v.tw != 0 || v.th % (32 / v.tw) != 0) return false;
+    bw = v.tw, bh = 32 / v.tw, bt = 1;
+  } else {
+    if (32 % plane != 0 || v.tt % (32 / plane) != 0) return false;
+    bw = v.tw, bh = v.th, bt = 32 / plane;
+  }
+  return true;
+}
 
 struct AttnArgs {
   const void* q;  // codes
@@ -33,6 +62,9 @@ struct AttnArgs {
   bool qk_fp4;
   bool causal;
   float softmax_scale;
+  // Non-null: Q, K, V are in tile-major order and out / lse are written back
+  // in raster order of this video layout (validated by video_chunk_box).
+  const VideoLayout* video;
 };
 
 // Returns cudaErrorNotSupported when the driver's tensor-map encoder is

@@ -7,6 +7,10 @@
 // itself stored in FP8). FP8 follows the FPSAttention conversion formula
 // (section 2.1) and staged granularities (section 3.1).
 //
+// With a video token map the kernels read raster-order (time-major) input
+// and write codes and scales in tile-major order, so the permutation costs no
+// pass of its own (FPSAttention page, section 3.3, item 1).
+//
 // All kernels are bandwidth-bound streams: 16-byte loads per thread,
 // consecutive threads on consecutive 16-byte chunks, warp-shuffle reductions.
 // Every scale step is one correctly rounded fp32 operation (__fdiv_rn,
@@ -19,6 +23,7 @@
 
 #include "fpattn_internal.h"
 #include "sm100.cuh"
+#include "token_map.cuh"
 
 namespace fpattn {
 
@@ -87,20 +92,27 @@ __device__ __forceinline__ uint2 quant8_e4m3(const uint4& v, float s) {
 // ---------------------------------------------------------------------------
 // FP8, one scale per (b, h, 128-token tile). grid = (ceil(N/128), B*H).
 // The tile (<= 128 x 128 bf16 = 32 KiB) stays in registers between the amax
-// reduction and the conversion, so x is read from HBM exactly once.
+// reduction and the conversion, so x is read from HBM exactly once. With a
+// token map (kMap) the tile's 128 source rows are looked up once into shared
+// memory.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kMap>
 __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restrict__ x, int N,
                                                             uint2* __restrict__ codes, float* __restrict__ scales,
-                                                            int* nonfinite) {
+                                                            int* nonfinite, TokenMap tmap) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int kChunks = 128 * kChunksPerRow;  // 16-byte chunks per full tile
   constexpr int kPer = kChunks / kThreads;
   __shared__ float red[kThreads / 32];
+  __shared__ int src_row[kMap ? 128 : 1];
   const int tile = blockIdx.x;
   const size_t bh = blockIdx.y;
   const int rows = min(128, N - tile * 128);
   const size_t base = (bh * N + static_cast<size_t>(tile) * 128) * kChunksPerRow;
+  if (kMap) {
+    if (threadIdx.x < rows) src_row[threadIdx.x] = to_raster(tmap, tile * 128 + threadIdx.x);
+    __syncthreads();
+  }
   uint4 v[kPer];
   float m = 0.f;
   bool bad = false;
@@ -108,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restr
   for (int i = 0; i < kPer; ++i) {
     const int c = threadIdx.x + i * kThreads;
     if (c / kChunksPerRow < rows) {
-      v[i] = x[base + c];
+      v[i] = kMap ? x[(bh * N + src_row[c / kChunksPerRow]) * kChunksPerRow + c % kChunksPerRow] : x[base + c];
       m = fmaxf(m, amax8(v[i], &bad));
     }
   }
@@ -170,23 +182,31 @@ __global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4*
   }
 }
 
-template <int D>
+// The amax pass is order-free, so only the conversion pass reads through the
+// token map (output row r, tile-major, from source row to_raster(r)).
+template <int D, bool kMap>
 __global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4* __restrict__ x, int N,
                                                                      const float* __restrict__ amax,
-                                                                     uint2* __restrict__ codes) {
+                                                                     uint2* __restrict__ codes, TokenMap tmap) {
   constexpr int kCpr = D / 8;
   constexpr int kRowsPerIter = kThreads / kCpr;
+  static_assert(kRowsPerCta == kThreads, "one source-row lookup per thread");
+  __shared__ int src_row[kMap ? kRowsPerCta : 1];
   const size_t bh = blockIdx.y;
   const int r0 = blockIdx.x * kRowsPerCta;
   const int cg = threadIdx.x % kCpr;
   const int rr = threadIdx.x / kCpr;
+  const int rend = min(N, r0 + kRowsPerCta);
+  if (kMap) {
+    if (r0 + static_cast<int>(threadIdx.x) < rend) src_row[threadIdx.x] = to_raster(tmap, r0 + threadIdx.x);
+    __syncthreads();
+  }
   float s[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) s[i] = fp8_scale_from_amax(amax[bh * D + cg * 8 + i]);
-  const int rend = min(N, r0 + kRowsPerCta);
   for (int r = r0 + rr; r < rend; r += kRowsPerIter) {
     const size_t idx = (bh * N + r) * kCpr + cg;
-    const uint4 v = x[idx];
+    const uint4 v = kMap ? x[(bh * N + src_row[r - r0]) * kCpr + cg] : x[idx];
     float f[8];
     unpack8(v, f);
     uint2 o;
@@ -236,11 +256,12 @@ __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
   return amax == 0.f ? 1.f : __fdiv_rn(amax, 2688.f);
 }
 
-template <int D>
+template <int D, bool kMap>
 __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __restrict__ x, int N, int nblk,
                                                                const float* __restrict__ amax_ptr,
                                                                uint4* __restrict__ codes,
-                                                               uint32_t* __restrict__ sf, size_t total_groups) {
+                                                               uint32_t* __restrict__ sf, size_t total_groups,
+                                                               TokenMap tmap) {
   constexpr int kGroups = D / 64;  // 64-element groups per row
   const size_t g = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x;
   if (g >= total_groups) return;
@@ -261,7 +282,8 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __re
   const float s_t = nvfp4_tensor_scale(*amax_ptr);
   const float six_st = __fmul_rn(6.f, s_t);
   const size_t row = bh * N + r;
-  const uint4* src = x + (row * D + grp * 64) / 8;
+  const size_t src_row = kMap ? bh * N + to_raster(tmap, r) : row;
+  const uint4* src = x + (src_row * D + grp * 64) / 8;
   uint4* dst = codes + (row * D + grp * 64) / 32;
   uint32_t sfw = 0;
   uint32_t out[8];
@@ -309,30 +331,37 @@ inline int num_sms() {
 // Host launchers (arguments already validated by the C ABI layer).
 // ---------------------------------------------------------------------------
 cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
-                                     int* nonfinite, cudaStream_t st) {
+                                     int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
   dim3 grid((N + 127) / 128, BH);
-  if (d == 128)
-    fp8_tile_kernel<128><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(x), N,
-                                                    reinterpret_cast<uint2*>(codes), scales, nonfinite);
-  else
-    fp8_tile_kernel<64><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(x), N,
-                                                   reinterpret_cast<uint2*>(codes), scales, nonfinite);
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint2* cv = reinterpret_cast<uint2*>(codes);
+  const TokenMap tm = tmap ? *tmap : TokenMap{};
+  if (d == 128) {
+    if (tmap) fp8_tile_kernel<128, true><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+    else fp8_tile_kernel<128, false><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+  } else {
+    if (tmap) fp8_tile_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+    else fp8_tile_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
-                                        int* nonfinite, cudaStream_t st) {
+                                        int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(scales, 0, sizeof(float) * BH * d, st);
   if (e != cudaSuccess) return e;
   dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, BH);
   const uint4* xv = static_cast<const uint4*>(x);
   uint2* cv = reinterpret_cast<uint2*>(codes);
+  const TokenMap tm = tmap ? *tmap : TokenMap{};
   if (d == 128) {
     fp8_channel_amax_kernel<128><<<grid, kThreads, 0, st>>>(xv, N, scales, nonfinite);
-    fp8_channel_quant_kernel<128><<<grid, kThreads, 0, st>>>(xv, N, scales, cv);
+    if (tmap) fp8_channel_quant_kernel<128, true><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
+    else fp8_channel_quant_kernel<128, false><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
   } else {
     fp8_channel_amax_kernel<64><<<grid, kThreads, 0, st>>>(xv, N, scales, nonfinite);
-    fp8_channel_quant_kernel<64><<<grid, kThreads, 0, st>>>(xv, N, scales, cv);
+    if (tmap) fp8_channel_quant_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
+    else fp8_channel_quant_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
   }
   const int n = BH * d;
   fp8_channel_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(scales, n);
@@ -341,7 +370,7 @@ cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uin
 
 cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const float* static_amax,
                                   uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
-                                  cudaStream_t st) {
+                                  const TokenMap* tmap, cudaStream_t st) {
   const float* amax_ptr = static_amax;
   if (!static_amax) {
     // tensor_scale doubles as the amax accumulator until pass 3 overwrites it.
@@ -356,14 +385,17 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
   const int nblk = (N + 127) / 128;
   const size_t groups = static_cast<size_t>(BH) * nblk * 128 * (d / 64);
   const unsigned blocks = static_cast<unsigned>((groups + kThreads - 1) / kThreads);
-  if (d == 128)
-    nvfp4_quant_kernel<128><<<blocks, kThreads, 0, st>>>(static_cast<const uint4*>(x), N, nblk, amax_ptr,
-                                                         reinterpret_cast<uint4*>(codes),
-                                                         reinterpret_cast<uint32_t*>(block_sf), groups);
-  else
-    nvfp4_quant_kernel<64><<<blocks, kThreads, 0, st>>>(static_cast<const uint4*>(x), N, nblk, amax_ptr,
-                                                        reinterpret_cast<uint4*>(codes),
-                                                        reinterpret_cast<uint32_t*>(block_sf), groups);
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint4* cv = reinterpret_cast<uint4*>(codes);
+  uint32_t* sv = reinterpret_cast<uint32_t*>(block_sf);
+  const TokenMap tm = tmap ? *tmap : TokenMap{};
+  if (d == 128) {
+    if (tmap) nvfp4_quant_kernel<128, true><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
+    else nvfp4_quant_kernel<128, false><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
+  } else {
+    if (tmap) nvfp4_quant_kernel<64, true><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
+    else nvfp4_quant_kernel<64, false><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
+  }
   nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax_ptr, tensor_scale);
   return cudaGetLastError();
 }

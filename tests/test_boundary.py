@@ -134,3 +134,75 @@ def test_library_missing_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         _lib.load()
+
+
+def _chunks_are_boxes(grid, tile):
+    """Brute force on the oracle's permutation: every 32 consecutive
+    tile-major tokens fill an axis-aligned box of the grid in raster order,
+    and no 128-token block crosses a tile."""
+    if (tile[0] * tile[1] * tile[2]) % 128:
+        return False
+    perm = sta.raster_index_of_tile_major(grid, tile)
+    T, Hs, W = grid
+    t, h, w = perm // (Hs * W), (perm // W) % Hs, perm % W
+    for i0 in range(0, len(perm), 32):
+        sl = slice(i0, i0 + 32)
+        ext = [(a.max() - a.min() + 1) for a in (t[sl], h[sl], w[sl])]
+        if ext[0] * ext[1] * ext[2] != 32:
+            return False
+        # the box in raster order is what a 3D box copy reads or writes
+        tt, hh, ww = np.meshgrid(np.arange(t[sl].min(), t[sl].min() + ext[0]),
+                                 np.arange(h[sl].min(), h[sl].min() + ext[1]),
+                                 np.arange(w[sl].min(), w[sl].min() + ext[2]), indexing="ij")
+        if not np.array_equal((tt * Hs + hh) * W + ww, perm[sl].reshape(ext)):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("tile", [(6, 8, 8), (4, 8, 8), (6, 16, 16), (2, 4, 16), (1, 4, 32), (2, 8, 8),
+                                  (4, 4, 8), (8, 2, 8), (1, 2, 64), (2, 16, 4), (6, 12, 8), (3, 8, 8),
+                                  (2, 2, 32), (4, 4, 4), (1, 1, 128), (2, 8, 16), (4, 8, 4), (2, 32, 2),
+                                  (8, 3, 16), (16, 1, 24), (4, 2, 48), (2, 6, 32)])
+def test_video_layout_rule_matches_bruteforce(lib, tile):
+    grid = (tile[0] * 2, tile[1] * 2, tile[2] * 3)
+    N = grid[0] * grid[1] * grid[2]
+    lay = _lib.VideoLayout(*grid, *tile)
+    st = lib.fpattn_video_layout_check(ctypes.byref(lay), N)
+    assert st in (_lib.OK, _lib.ERR_UNSUPPORTED)
+    assert (st == _lib.OK) == _chunks_are_boxes(grid, tile)
+
+
+def test_video_argument_errors(lib):
+    buf = (ctypes.c_uint8 * 4096)()
+    p16 = (ctypes.addressof(buf) + 15) & ~15
+    good = _lib.VideoLayout(1, 8, 16, 1, 8, 16)          # N = 128
+    assert lib.fpattn_video_layout_check(ctypes.byref(good), 128) == _lib.OK
+    assert lib.fpattn_video_layout_check(None, 128) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_video_layout_check(ctypes.byref(good), 256) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_video_layout_check(ctypes.byref(_lib.VideoLayout(1, 8, 16, 1, 0, 16)), 128) == _lib.ERR_INVALID_ARG
+    ragged = _lib.VideoLayout(1, 8, 16, 1, 3, 16)         # Hs not a multiple of th
+    assert lib.fpattn_video_layout_check(ctypes.byref(ragged), 128) == _lib.ERR_UNSUPPORTED
+    x = _t(p16, _lib.BF16, N=128)
+    for ok in [(1, 4, 32, 1, 4, 32),     # a chunk is one w-row of 32
+               (1, 16, 8, 1, 16, 8),     # a chunk is 4 w-rows of 8
+               (1, 1, 128, 1, 1, 128),   # a chunk is a quarter w-row
+               (1, 2, 64, 1, 2, 64)]:    # a chunk is half a w-row
+        assert lib.fpattn_video_layout_check(ctypes.byref(_lib.VideoLayout(*ok)), 128) == _lib.OK
+    rej = _lib.VideoLayout(3, 8, 8, 3, 8, 8)              # tile volume 192: not a multiple of 128
+    assert lib.fpattn_video_layout_check(ctypes.byref(rej), 192) == _lib.ERR_UNSUPPORTED
+    # the entry points reject before any CUDA call
+    assert lib.fpattn_quantize_fp8_video(ctypes.byref(x), None, 0, p16, p16, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_quantize_fp8_video(ctypes.byref(x), ctypes.byref(ragged), 0, p16, p16, None,
+                                         None) == _lib.ERR_UNSUPPORTED
+    assert lib.fpattn_quantize_nvfp4_video(ctypes.byref(x), ctypes.byref(ragged), None, p16, p16, p16, None,
+                                           None) == _lib.ERR_UNSUPPORTED
+    assert lib.fpattn_quantize_nvfp4_video(ctypes.byref(x), None, None, p16, p16, p16, None,
+                                           None) == _lib.ERR_INVALID_ARG
+    q = _t(p16, _lib.E4M3, N=128)
+    sc = _lib.Scales(p16, p16, p16, None, None, 1.0 / 448.0, 0.0)
+    assert lib.fpattn_fwd_video(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(sc), None, 0,
+                                None, p16, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_fwd_video(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(sc), None, 0,
+                                ctypes.byref(rej), p16, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_fwd_video(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(sc), None, 0,
+                                ctypes.byref(ragged), p16, None, None) == _lib.ERR_UNSUPPORTED

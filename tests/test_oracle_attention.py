@@ -153,3 +153,30 @@ def test_sta_block_lists_match_token_bruteforce():
         for kb in blocks[p // 128]:
             from_blocks[kb * 128:(kb + 1) * 128] = True
         assert np.array_equal(from_blocks, tok[i])
+
+
+def test_tile_major_raster_index_worked_example():
+    # 2 x 2 x 4 grid in 1 x 2 x 2 tiles, worked out by hand: tiles in raster
+    # order (0,0,0), (0,0,1), (1,0,0), (1,0,1); each lists its 2 x 2 tokens
+    # (h, w) in raster order; raster row = t*8 + h*4 + w.
+    perm = sta.raster_index_of_tile_major((2, 2, 4), (1, 2, 2))
+    assert perm.tolist() == [0, 1, 4, 5, 2, 3, 6, 7, 8, 9, 12, 13, 10, 11, 14, 15]
+
+
+def test_tile_major_raster_index_is_tile_contiguous_bijection():
+    grid, tile = (12, 16, 24), (6, 8, 8)
+    perm = sta.raster_index_of_tile_major(grid, tile)
+    N = 12 * 16 * 24
+    assert sorted(perm.tolist()) == list(range(N))
+    vol = 6 * 8 * 8
+    t, h, w = perm // (16 * 24), (perm // 24) % 16, perm % 24
+    for i0 in range(0, N, vol):
+        # one tile per vol consecutive positions, full extent on every axis
+        sl = slice(i0, i0 + vol)
+        assert len({(a // 6, b // 8, c // 8) for a, b, c in zip(t[sl], h[sl], w[sl])}) == 1
+        # raster order inside the tile: (t, h, w) ascend lexicographically
+        key = (t[sl] * 1000 + h[sl]) * 1000 + w[sl]
+        assert np.all(np.diff(key) > 0)
+    # tiles themselves in raster order over the 2 x 2 x 3 tile grid
+    firsts = [(t[i] // 6, h[i] // 8, w[i] // 8) for i in range(0, N, vol)]
+    assert firsts == [(a, b, c) for a in range(2) for b in range(2) for c in range(3)]

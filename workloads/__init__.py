@@ -135,11 +135,13 @@ def _video_bias(gen: torch.Generator, grid, d: int) -> torch.Tensor:
 
 
 def make_qkv(w: Workload, *, heads: Optional[int] = None, batch: Optional[int] = None,
-             N: Optional[int] = None):
+             N: Optional[int] = None, tile_major: bool = True):
     """Return bf16 CPU tensors q, k, v of shape [B, H, N, d] for workload ``w``.
 
     ``heads``/``batch``/``N`` override the sizes for reduced parity cases; the
-    seed and recipe stay the workload's.
+    seed and recipe stay the workload's. Sliding-tile workloads come in
+    tile-major token order unless ``tile_major`` is False (raster order, as a
+    video model holds its tokens).
     """
     B = w.B if batch is None else batch
     H = w.H if heads is None else heads
@@ -159,7 +161,7 @@ def make_qkv(w: Workload, *, heads: Optional[int] = None, batch: Optional[int] =
         q += bias
         k += bias
         v += bias
-        if w.sta_tile is not None:
+        if w.sta_tile is not None and tile_major:
             perm = video_tile_major_perm(w.video, w.sta_tile)
             q, k, v = q[:, :, perm], k[:, :, perm], v[:, :, perm]
     return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(),
