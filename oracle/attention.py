@@ -20,6 +20,18 @@ What is computed (per query row i of one (batch, head)):
 A tile with no allowed key leaves the state unchanged. A row with no allowed
 key at all gives out = 0 and lse = -inf.
 
+Conditional rescale (FlashAttention-4 article, co-design list, online-softmax
+item: rescale only once the running max has moved past a threshold),
+``rescale_threshold`` = tau >= 0 in log2 units. The reference max m moves only
+when it must:
+      m_c  = max(m, max_j S_j)
+      m'   = m_c   if m = -inf or (m_c - m) * log2(e) > tau,   else m
+and the rest of the step is unchanged, except that P_j = exp(S_j - m') may
+now reach 2^tau, so P is rounded at the scale 448 * 2^-tau, which keeps every
+code below the E4M3 maximum:
+      Ph_j = E4M3(448 * 2^-tau * P_j) / (448 * 2^-tau).
+tau = 0 is the exact running max above.
+
 Allowed keys: all keys < N; under ``causal`` only j <= i; under a tile mask
 only keys whose 128-key block is listed for the query's 128-row block.
 
@@ -42,24 +54,29 @@ from . import codec
 
 TILE = 128
 P_SCALE_INV = 448.0
+LOG2E = 1.0 / math.log(2.0)
 
 
-def _quantize_p(p: np.ndarray) -> np.ndarray:
-    return codec.e4m3_decode(codec.e4m3_encode(p * P_SCALE_INV)) / P_SCALE_INV
+def _quantize_p(p: np.ndarray, tau: float = 0.0) -> np.ndarray:
+    s = P_SCALE_INV * 2.0 ** -tau
+    return codec.e4m3_decode(codec.e4m3_encode(p * s)) / s
 
 
 def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray,
                    *, softmax_scale: Optional[float] = None, causal: bool = False,
                    key_blocks: Optional[Sequence[Sequence[int]]] = None,
-                   quantize_p: bool = True):
+                   quantize_p: bool = True, rescale_threshold: float = 0.0):
     """Attention output and lse for the query ``rows`` of one (batch, head).
 
     q, k, v     float64 [N, d] dequantized operands
     rows        int array of query indices (all in one 128-row block, or any)
     key_blocks  optional list: key_blocks[qb] = allowed 128-key block indices
                 for query block qb (the tile mask); None = dense
+    rescale_threshold  tau of the conditional rescale (log2 units), 0 = exact
     Returns (out float64 [len(rows), d], lse float64 [len(rows)]).
     """
+    tau = float(rescale_threshold)
+    assert tau >= 0.0
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -89,12 +106,15 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray
             continue
         S = softmax_scale * (q[rows] @ k[keys].T)
         S = np.where(allowed, S, -np.inf)
-        m_new = np.where(live, np.maximum(m, S.max(axis=1)), m)
+        m_cand = np.where(live, np.maximum(m, S.max(axis=1)), m)
+        with np.errstate(invalid="ignore"):
+            move = np.isneginf(m) | ((m_cand - m) * LOG2E > tau)
+        m_new = np.where(move, m_cand, m)
         with np.errstate(invalid="ignore"):
             alpha = np.where(live, np.exp(m - m_new), 1.0)
             P = np.where(allowed, np.exp(S - m_new[:, None]), 0.0)
         l = l * alpha + P.sum(axis=1)
-        Ph = _quantize_p(P) if quantize_p else P
+        Ph = _quantize_p(P, tau) if quantize_p else P
         O = O * alpha[:, None] + Ph @ v[keys]
         m = m_new
     with np.errstate(invalid="ignore", divide="ignore"):
@@ -104,14 +124,15 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray
 
 
 def attention(q, k, v, *, softmax_scale=None, causal=False, key_blocks=None,
-              quantize_p=True):
+              quantize_p=True, rescale_threshold=0.0):
     """Whole (batch, head) attention, 128 rows at a time. Returns (out, lse)."""
     N = q.shape[0]
     outs, lses = [], []
     for b0 in range(0, N, TILE):
         rows = np.arange(b0, min(b0 + TILE, N))
         o, s = attention_rows(q, k, v, rows, softmax_scale=softmax_scale, causal=causal,
-                              key_blocks=key_blocks, quantize_p=quantize_p)
+                              key_blocks=key_blocks, quantize_p=quantize_p,
+                              rescale_threshold=rescale_threshold)
         outs.append(o)
         lses.append(s)
     return np.concatenate(outs), np.concatenate(lses)

@@ -8,6 +8,9 @@
 * Causal row 0 is v_0.
 * Worked examples pin the E4M3 rounding of P against the running max and the
   rescale across tiles.
+* The conditional rescale with threshold tau: unquantized, it equals the
+  textbook softmax for any tau; worked examples pin the stale-max decision and
+  the 448 * 2^-tau rounding scale on both sides of the threshold.
 * The STA block lists agree with a brute-force token-level window test and
   with the pair counts of the (6,8,8)-tile, (3,3,5)-window video workload.
 """
@@ -153,6 +156,73 @@ def test_sta_block_lists_match_token_bruteforce():
         for kb in blocks[p // 128]:
             from_blocks[kb * 128:(kb + 1) * 128] = True
         assert np.array_equal(from_blocks, tok[i])
+
+
+@pytest.mark.parametrize("tau", [1.0, 3.5, 8.0])
+@pytest.mark.parametrize("causal", [False, True])
+def test_threshold_rescale_unquantized_matches_sdpa(tau, causal):
+    # A stale reference max cancels in O / l when P is not rounded, so any
+    # threshold must reproduce the textbook softmax exactly.
+    rng = np.random.default_rng(int(tau * 10) + causal)
+    N, d = 300, 64
+    q, k, v = (rng.standard_normal((N, d)) * 2 for _ in range(3))
+    # raise the later keys' scores so the max keeps growing across tiles
+    k[128:] *= 1.5
+    out, lse = A.attention(q, k, v, causal=causal, quantize_p=False, rescale_threshold=tau)
+    assert np.max(np.abs(out - _sdpa(q, k, v, causal=causal))) < 1e-12
+    ref_out, ref_lse = A.attention(q, k, v, causal=causal, quantize_p=False)
+    assert np.max(np.abs(lse - ref_lse)) < 1e-12
+
+
+def _threshold_example(tau):
+    # one query; key 0 (tile 0) scores 0; keys 128 and 129 (tile 1) score
+    # 1.5 ln 2 and 1.5 ln 2 + ln 0.3; every other key -1000 (P = 0 exactly)
+    N = 256
+    q = np.ones((1, 1))
+    k = np.full((N, 1), -1000.0)
+    k[0, 0] = 0.0
+    k[128, 0] = 1.5 * math.log(2.0)
+    k[129, 0] = 1.5 * math.log(2.0) + math.log(0.3)
+    v = np.zeros((N, 3))
+    v[0, 0] = v[128, 1] = v[129, 2] = 1.0
+    return A.attention_rows(q, k, v, np.array([0]), softmax_scale=1.0, rescale_threshold=tau)
+
+
+def test_threshold_rescale_worked_example_keeps_stale_max():
+    # tau = 3: the max grows by 1.5 (log2) <= 3, so m stays 0 and tile 1's P
+    # reach 2^1.5. P is rounded at the scale 448 / 8 = 56:
+    #   1 -> 56 (exact); 2^1.5 * 56 = 158.39 -> 160; 0.3 * 2^1.5 * 56 = 47.52 -> 48
+    out, lse = _threshold_example(3.0)
+    r = 2.0 ** 1.5
+    l = 1.0 + r + 0.3 * r
+    assert out[0].tolist() == pytest.approx([1.0 / l, (160.0 / 56.0) / l, (48.0 / 56.0) / l], rel=1e-14)
+    assert lse[0] == pytest.approx(math.log(l), rel=1e-14)
+
+
+def test_threshold_rescale_worked_example_moves_max():
+    # tau = 1: 1.5 > 1, so m moves to 1.5 ln 2 and O, l scale by 2^-1.5. P is
+    # rounded at 448 / 2 = 224: tile 0's 1 -> 224 (exact); tile 1: 1 -> 224,
+    # 0.3 * 224 = 67.2 -> 64.
+    out, lse = _threshold_example(1.0)
+    a = 2.0 ** -1.5
+    l = a + 1.0 + 0.3
+    assert out[0].tolist() == pytest.approx([a / l, 1.0 / l, (64.0 / 224.0) / l], rel=1e-14)
+    assert lse[0] == pytest.approx(1.5 * math.log(2.0) + math.log(l), rel=1e-14)
+    # the same keys at tau = 0 round tile 1 at 448: 0.3 * 448 = 134.4 -> 128
+    out0, _ = _threshold_example(0.0)
+    assert out0[0, 2] == pytest.approx((128.0 / 448.0) / l, rel=1e-14)
+
+
+def test_threshold_is_in_log2_units():
+    # tau = 1.25 lies between the growth in log2 units (1.5) and in natural
+    # units (1.04): the max must move. Rounding scale s = 448 * 2^-1.25 =
+    # 188.36: 1 * s -> 192 (step 16 in [128, 256)); 0.3 * s = 56.51 -> 56
+    # (step 4 in [32, 64)).
+    out, _ = _threshold_example(1.25)
+    s = 448.0 * 2.0 ** -1.25
+    a = 2.0 ** -1.5
+    l = a + 1.3
+    assert out[0].tolist() == pytest.approx([a * (192.0 / s) / l, (192.0 / s) / l, (56.0 / s) / l], rel=1e-14)
 
 
 def test_tile_major_raster_index_worked_example():
