@@ -338,6 +338,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--rescale-threshold", type=float, default=0.0,
+                    help="conditional softmax rescale threshold tau (log2 units); 0 = exact running max")
     args = ap.parse_args()
     if args.sweep:
         return run_sweep(args)
@@ -381,7 +383,8 @@ def main():
         vq = fp.quantize_fp8(v, "channel", video=video)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask, video=video)
+        out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask, video=video,
+                                    rescale_threshold=args.rescale_threshold)
         if ev_pair is not None:
             ev_pair[1].record(stream)
         return out
@@ -434,14 +437,14 @@ def main():
         out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
         lse_h = torch.empty(q_h.shape[:3], dtype=torch.float32, pin_memory=True)
         fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
-                     lse_host=lse_h, video=video)
+                     lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         e0.record(stream)
         for _ in range(args.e2e_steps):
             fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
-                         lse_host=lse_h, video=video)
+                         lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold)
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = rank_max(e0.elapsed_time(e1) / args.e2e_steps)
@@ -470,7 +473,8 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e2m1/e4m3 MMA, f32 accumulate", "data": "synthetic",
-            "config": config_dict(w),
+            "config": dict(config_dict(w), **({"rescale_threshold": args.rescale_threshold}
+                                              if args.rescale_threshold else {})),
             "attn_ms": attn_ms, "attn_tflops_algorithmic": attn_tflops,
             "attn_tflops_dense_eq": w.dense_flops() / (attn_ms * 1e-3) / 1e12,
             "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,

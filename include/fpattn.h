@@ -149,6 +149,16 @@ typedef struct {
   float p_scale;
   /* Multiplier of Q K^T before the softmax; 0 selects 1/sqrt(d). */
   float softmax_scale;
+  /* Conditional softmax rescale (FlashAttention-4 article, co-design list,
+     online-softmax item: rescale only once the running max has moved past a
+     threshold). tau in [0, 8], log2 units; 0 (the default of a zeroed struct)
+     is the exact running max. With tau > 0 a row's reference max m moves to
+     the running max only when that exceeds m by more than tau; otherwise O
+     and l are not rescaled, P = 2^(s - m) may reach 2^tau, and P is stored
+     in E4M3 at the scale 448 * 2^-tau (p_scale above stays 1/448: the
+     2^-tau is applied inside the kernel and cancels in O / l). Outside
+     [0, 8]: FPATTN_ERR_INVALID_ARG. */
+  float rescale_threshold;
 } fpattn_scales;
 
 /*

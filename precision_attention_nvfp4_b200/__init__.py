@@ -185,13 +185,14 @@ def sta_plan(tile_grid: Sequence[int], tile: Sequence[int], window: Sequence[int
 def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, return_lse: bool = True,
-                  video: Optional[VideoLayout] = None):
+                  video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0):
     """Fused attention on quantized operands.
 
     q, k: both Nvfp4Tensor or both Fp8Tensor (tile128); v: Fp8Tensor (channel).
     Returns (out bf16 [B,H,N,d], lse float32 [B,H,N] or None). With ``video``
     the operands are in tile-major order and out / lse come back in raster
-    order.
+    order. ``rescale_threshold`` (tau, log2 units, 0..8) skips the O / l
+    rescale until a row's max has grown by more than tau; 0 is exact.
     """
     B, H, N, d = v.shape
     lib = library()
@@ -199,12 +200,13 @@ def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Option
         qd = _desc(q.codes, _lib.NVFP4, B, H, N, d)
         kd = _desc(k.codes, _lib.NVFP4, B, H, N, d)
         sc = _lib.Scales(q.tensor_scale.data_ptr(), k.tensor_scale.data_ptr(), v.scales.data_ptr(),
-                         q.block_sf.data_ptr(), k.block_sf.data_ptr(), 1.0 / 448.0, softmax_scale)
+                         q.block_sf.data_ptr(), k.block_sf.data_ptr(), 1.0 / 448.0, softmax_scale,
+                         rescale_threshold)
     elif isinstance(q, Fp8Tensor) and isinstance(k, Fp8Tensor):
         qd = _desc(q.codes, _lib.E4M3, B, H, N, d)
         kd = _desc(k.codes, _lib.E4M3, B, H, N, d)
         sc = _lib.Scales(q.scales.data_ptr(), k.scales.data_ptr(), v.scales.data_ptr(), None, None,
-                         1.0 / 448.0, softmax_scale)
+                         1.0 / 448.0, softmax_scale, rescale_threshold)
     else:
         raise TypeError("q and k must both be Nvfp4Tensor or both Fp8Tensor")
     vd = _desc(v.codes, _lib.E4M3, B, H, N, d)
@@ -227,7 +229,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
               causal: bool = False, tile_mask: Optional[DeviceTileMask] = None, softmax_scale: float = 0.0,
               return_lse: bool = True, device: Optional[torch.device] = None,
               out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None,
-              video: Optional[VideoLayout] = None):
+              video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0):
     """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
 
     CUDA inputs stay where they are. Host inputs (ideally pinned) are copied
@@ -249,7 +251,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
     vq = quantize_fp8(v, "channel", video=video)
     out, lse = attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
-                             return_lse=return_lse, video=video)
+                             return_lse=return_lse, video=video, rescale_threshold=rescale_threshold)
     if host:
         out_h = out_host if out_host is not None else torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         out_h.copy_(out, non_blocking=True)

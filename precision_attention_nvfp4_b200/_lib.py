@@ -20,7 +20,8 @@ class Tensor(ctypes.Structure):
 class Scales(ctypes.Structure):
     _fields_ = [("q_scale", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("q_block_sf", ctypes.c_void_p), ("k_block_sf", ctypes.c_void_p),
-                ("p_scale", ctypes.c_float), ("softmax_scale", ctypes.c_float)]
+                ("p_scale", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("rescale_threshold", ctypes.c_float)]
 
 
 class TileMask(ctypes.Structure):

@@ -113,6 +113,7 @@ fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_t
   // P is stored in E4M3 at the fixed scale 1/448.
   if (!(scales->p_scale > 0.f) || std::abs(scales->p_scale * 448.f - 1.f) > 1e-6f) return FPATTN_ERR_INVALID_ARG;
   if (!(scales->softmax_scale >= 0.f) || scales->softmax_scale > 1e30f) return FPATTN_ERR_INVALID_ARG;
+  if (!(scales->rescale_threshold >= 0.f && scales->rescale_threshold <= 8.f)) return FPATTN_ERR_INVALID_ARG;
   const int nblk = (q->N + 127) / 128;
   if (tile_mask) {
     if (tile_mask->nblk_q != nblk || !tile_mask->row_ptr || !tile_mask->col_idx || tile_mask->nnz < 0)
@@ -139,6 +140,7 @@ fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_t
   a.qk_fp4 = fp4;
   a.causal = causal != 0;
   a.softmax_scale = scales->softmax_scale > 0.f ? scales->softmax_scale : 1.0f / std::sqrt(static_cast<float>(q->d));
+  a.rescale_threshold = scales->rescale_threshold;
   a.video = layout ? &vl : nullptr;
   return from_cuda(fpattn::launch_attn_fwd(a, reinterpret_cast<cudaStream_t>(stream)));
 }

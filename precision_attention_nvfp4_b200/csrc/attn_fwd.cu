@@ -139,6 +139,8 @@ struct __align__(64) Params {
   int N, nblk, BH, num_items;
   int causal, sparse;
   float sm_scale_log2;
+  float tau;           // conditional-rescale threshold, log2 units (0: exact running max)
+  float p_log2_scale;  // log2 of the P scale: log2(448) - tau
   TokenMap tmap;  // on: rows are tile-major, out and lse go to raster positions
 };
 
@@ -542,10 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ok = __all_sync(0xffffffffu, got) && ok;
         const float rawmax = w == 0 ? fmaxf(half_max, other_max) : fmaxf(other_max, half_max);
         const float c = FP4 ? c_fp4 : inv_sq / p.k_scale[static_cast<size_t>(bh) * p.nblk + kb];
-        // m_ref: exact running max (-inf while every key so far is masked);
-        // m_use: the offset the exponentials use (0 in that case).
+        // m_ref: reference max (-inf while every key so far is masked). It
+        // moves to the running max only when that exceeds it by more than tau
+        // (log2 units; tau = 0: the exact running max), and P then reaches at
+        // most 2^tau, which the P scale 448 * 2^-tau absorbs. m_use: the
+        // offset the exponentials use (0 while m_ref is -inf).
         const float m_prev = m_ref;
-        const float m_new = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
+        const float cand = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
+        const float m_new = (m_prev == -INFINITY || cand - m_prev > p.tau) ? cand : m_prev;
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
         // Rescale factor of O and of the row sum; a row that has seen no key
         // yet (m_prev = -inf) has O = 0 and l = 0, scaled by 2^-inf = 0.
@@ -560,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         m_ref = m_new;
         // P = 2^(c s - m + log2 448) -> E4M3, this half's 16 columns of P
         // buffer g % kPBufs.
-        const float nbias = kLog2_448 - m_use;
+        const float nbias = p.p_log2_scale - m_use;
         const int pb = g % C::kPBufs;
         const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32 + 16 * w;
         uint32_t pk0[8], pk1[8];
@@ -707,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       if (store && p.lse)
         p.lse[static_cast<size_t>(bh) * p.N + to_raster(p.tmap, qrow)] =
-            ltot > 0.f ? (m + __log2f(ltot) - kLog2_448) * kLn2 : -INFINITY;
+            ltot > 0.f ? (m + __log2f(ltot) - p.p_log2_scale) * kLn2 : -INFINITY;
       tc_fence_before();
     }
     if (lane == 0) bulk_wait_all();
@@ -845,6 +851,8 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   p.causal = a.causal ? 1 : 0;
   p.sparse = a.row_ptr ? 1 : 0;
   p.sm_scale_log2 = a.softmax_scale * 1.4426950408889634f;
+  p.tau = a.rescale_threshold;
+  p.p_log2_scale = kLog2_448 - a.rescale_threshold;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -62,6 +62,7 @@ struct AttnArgs {
   bool qk_fp4;
   bool causal;
   float softmax_scale;
+  float rescale_threshold;  // tau in [0, 8], log2 units
   // Non-null: Q, K, V are in tile-major order and out / lse are written back
   // in raster order of this video layout (validated by video_chunk_box).
   const VideoLayout* video;

@@ -61,10 +61,10 @@ def oracle_operands(q, k, v, qk_format, heads=None):
 
 
 def compare_attention(out_gpu: np.ndarray, lse_gpu: np.ndarray, qh, kh, vh, rows, *, causal=False,
-                      key_blocks=None, softmax_scale=None):
+                      key_blocks=None, softmax_scale=None, rescale_threshold=0.0):
     """Oracle rows vs GPU rows for one (b,h). Returns a dict of errors."""
     ref, ref_lse = oatt.attention_rows(qh, kh, vh, rows, causal=causal, key_blocks=key_blocks,
-                                       softmax_scale=softmax_scale)
+                                       softmax_scale=softmax_scale, rescale_threshold=rescale_threshold)
     got = out_gpu[rows].astype(np.float64)
     err = np.abs(got - ref)
     vmax = np.abs(vh).max()

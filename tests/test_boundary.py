@@ -99,6 +99,10 @@ def test_fwd_argument_errors(lib):
     assert lib.fpattn_fwd(ctypes.byref(qbf), ctypes.byref(qbf), *ok_args[2:]) == _lib.ERR_UNSUPPORTED
     # misaligned output, tile mask of the wrong size
     assert lib.fpattn_fwd(*ok_args[:6], p16 + 4, None, None) == _lib.ERR_ALIGNMENT
+    for tau in (-0.5, 8.5, float("nan"), float("inf")):
+        bad_tau = _lib.Scales(p16, p16, p16, None, None, 1.0 / 448.0, 0.0, tau)
+        assert lib.fpattn_fwd(ctypes.byref(q), ctypes.byref(q), ctypes.byref(v), ctypes.byref(bad_tau), None, 0,
+                              p16, None, None) == _lib.ERR_INVALID_ARG
     tm = _lib.TileMask(5, 0, p16, p16, None)
     assert lib.fpattn_fwd(*ok_args[:4], ctypes.byref(tm), 0, p16, None, None) == _lib.ERR_INVALID_ARG
 
