@@ -137,6 +137,34 @@ def quantize_fp8_tile(x, tile: int = FP8_TILE):
     return codes, s
 
 
+def quantize_fp8_group(x, group: int, tile: int = FP8_TILE):
+    """Q/K quantization with one scale per group of ``group`` consecutive
+    128-token tiles of one (batch, head): the coarser granularities of the
+    FPSAttention page's denoising-step-aware schedule (section 3.2: coarse,
+    intermediate and fine granularities by phase). group = 1 is the per-tile
+    quantization; a group of all tiles is one scale per (batch, head); a
+    group of the tiles of one 3D video tile is one scale per video tile.
+    A is the amax over the group's tokens (a last partial group over its
+    valid tokens); s = 448 / A; code = E4M3(x * s).
+
+    Returns (codes uint8 [..., N, d], scales float32 [..., ceil(N/tile)]): the
+    scale of each tile, i.e. its group's scale repeated, so the result
+    dequantizes with dequantize_fp8_tile.
+    """
+    assert group >= 1
+    x = _f32(x)
+    N = x.shape[-2]
+    nt = -(-N // tile)
+    span = group * tile
+    s = np.zeros(x.shape[:-2] + (nt,), dtype=F32)
+    for g0 in range(0, nt, group):
+        a = np.max(np.abs(x[..., g0 * tile:g0 * tile + span, :]), axis=(-2, -1)).astype(F32)
+        s[..., g0:g0 + group] = fp8_scale(a)[..., None]
+    s_tok = np.repeat(s, tile, axis=-1)[..., :N]
+    codes = codec.e4m3_encode(x * s_tok[..., None])
+    return codes, s
+
+
 def quantize_fp8_channel(x):
     """Per-(batch, head) per-channel quantization of ``x`` [..., N, d].
 

@@ -155,3 +155,48 @@ def test_fp8_roundtrip_idempotent_and_zero():
     assert np.allclose(s1, s2, rtol=3e-7, atol=0)
     cz, sz = quant.quantize_fp8_channel(np.zeros((1, 1, 10, 16), dtype=F32))
     assert np.all(cz == 0) and np.all(sz == 1.0)
+
+
+@pytest.mark.parametrize("group", [1, 2, 3, 5])
+def test_fp8_group_scales_and_torch_cast(group):
+    # N = 600: 5 tiles, the last one ragged (88 tokens). Each group's scale is
+    # 448 / amax over exactly its tokens, repeated for its tiles; codes equal
+    # torch's E4M3 cast of x * s.
+    rng = np.random.default_rng(10 + group)
+    x = _bf16(rng.standard_normal((2, 2, 600, 64)) * 3)
+    x[0, 1, 590, 5] = 40.0                       # an outlier in the ragged tail
+    codes, s = quant.quantize_fp8_group(x, group)
+    assert s.shape == (2, 2, 5)
+    for t in range(5):
+        g0 = (t // group) * group
+        tokens = x[:, :, g0 * 128:min(600, (g0 + group) * 128)]
+        A = np.abs(tokens).max(axis=(-2, -1)).astype(F32)
+        assert np.array_equal(s[:, :, t], F32(448.0) / A), t
+    s_tok = np.repeat(s, 128, axis=-1)[..., :600]
+    prod = (x * s_tok[..., None]).astype(F32)
+    ref = torch.from_numpy(np.clip(prod, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+    # the amax element of every group maps to +-448
+    dec = np.abs(codec.e4m3_decode(codes))
+    for g0 in range(0, 5, group):
+        assert np.all(dec[:, :, g0 * 128:(g0 + group) * 128].max(axis=(-2, -1)) == 448.0)
+
+
+def test_fp8_group_of_one_tile_is_per_tile_and_whole_head_is_one_scale():
+    rng = np.random.default_rng(12)
+    x = _bf16(rng.standard_normal((1, 3, 300, 128)))
+    c1, s1 = quant.quantize_fp8_group(x, 1)
+    c0, s0 = quant.quantize_fp8_tile(x)
+    assert np.array_equal(c1, c0) and np.array_equal(s1, s0)
+    ch, sh = quant.quantize_fp8_group(x, 3)
+    A = np.abs(x).max(axis=(-2, -1)).astype(F32)
+    assert np.all(sh == (F32(448.0) / A)[..., None])
+
+
+def test_step_phase_worked_example():
+    # D = 50 steps with the page's alpha1 = 0.2, alpha2 = 0.7: t1 = 10, t2 = 35
+    from oracle import schedule
+    got = [schedule.step_phase(t, 50) for t in range(1, 51)]
+    assert got == [schedule.EARLY] * 10 + [schedule.MIDDLE] * 25 + [schedule.LATE] * 15
+    # D = 7: t1 = 1.4, t2 = 4.9 -> steps 1 | 2..4 | 5..7
+    assert [schedule.step_phase(t, 7) for t in range(1, 8)] == [0, 1, 1, 1, 2, 2, 2]
