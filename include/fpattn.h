@@ -133,6 +133,41 @@ fpattn_status fpattn_quantize_nvfp4(const fpattn_tensor* x, const float* static_
 fpattn_status fpattn_quantize_fp8(const fpattn_tensor* x, int32_t granularity, uint8_t* codes,
                                   float* scales, int32_t* nonfinite_flag, fpattn_stream_t stream);
 
+/*
+ * FP8 E4M3 quantization of Q or K with one scale per group of `group_tiles`
+ * consecutive 128-token tiles of each (b, h): the coarser Q/K granularities
+ * of the FPSAttention page's denoising-step-aware schedule (section 3.2).
+ * group_tiles = 1 is FPATTN_FP8_TILE128; ceil(N/128) (or more) is one scale
+ * per (b, h); the tiles of one 3D video tile (tt*th*tw/128) is one scale per
+ * video tile.
+ *
+ *   A = amax over the group's tokens (a last partial group: its valid
+ *       tokens); s = 448 / A (1 when A == 0); code = E4M3(x * s).
+ *
+ * scales receives B*H*ceil(N/128) floats, the scale of every tile (its
+ * group's scale, repeated), so fpattn_fwd takes them as per-tile scales
+ * unchanged. layout: NULL for x in kernel order, else x is in raster order
+ * and codes / scales come out tile-major, as in fpattn_quantize_fp8_video.
+ * group_tiles < 1: FPATTN_ERR_INVALID_ARG; other arguments as
+ * fpattn_quantize_fp8. x is read twice when group_tiles > 1 (amax pass,
+ * then conversion).
+ */
+fpattn_status fpattn_quantize_fp8_group(const fpattn_tensor* x, const struct fpattn_video_layout_s* layout,
+                                        int32_t group_tiles, uint8_t* codes, float* scales,
+                                        int32_t* nonfinite_flag, fpattn_stream_t stream);
+
+/*
+ * Phase of denoising step t of num_steps (FPSAttention page, section 3.2):
+ * with t1 = alpha1 * num_steps and t2 = alpha2 * num_steps (the page deploys
+ * alpha1 = 0.2, alpha2 = 0.7), t <= t1 is early (coarse granularity, sparse
+ * window), t1 < t <= t2 middle (fine, dense), later steps late
+ * (intermediate, medium). t counts steps in run order, 1 .. num_steps;
+ * comparisons in double. HOST-only. Errors: t outside 1..num_steps, or not
+ * 0 <= alpha1 <= alpha2 <= 1: FPATTN_ERR_INVALID_ARG.
+ */
+typedef enum { FPATTN_PHASE_EARLY = 0, FPATTN_PHASE_MIDDLE = 1, FPATTN_PHASE_LATE = 2 } fpattn_phase;
+fpattn_status fpattn_step_phase(int32_t t, int32_t num_steps, double alpha1, double alpha2, int32_t* phase);
+
 /* Scales consumed by fpattn_fwd. */
 typedef struct {
   /* NVFP4 Q/K: device pointer to the one-float tensor scale s_t.
@@ -245,7 +280,7 @@ fpattn_status fpattn_fwd(const fpattn_tensor* q, const fpattn_tensor* k, const f
  * (6,16,16) qualify. Other tiles give FPATTN_ERR_UNSUPPORTED; a layout with
  * T*Hs*W != N gives FPATTN_ERR_INVALID_ARG.
  */
-typedef struct {
+typedef struct fpattn_video_layout_s {
   int32_t T, Hs, W;    /* grid, in tokens */
   int32_t tt, th, tw;  /* tile, in tokens */
 } fpattn_video_layout;

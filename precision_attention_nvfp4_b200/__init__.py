@@ -7,10 +7,13 @@ computes any part of the method on the host.
 
 Public calls
   quantize_nvfp4(x)            -> Nvfp4Tensor(codes, block_sf, tensor_scale)
-  quantize_fp8(x, granularity) -> Fp8Tensor(codes, scales)
+  quantize_fp8(x, granularity) -> Fp8Tensor(codes, scales); granularity
+                                  "tile128", "channel", or "group" with
+                                  group_tiles tiles per scale
                                   (with video=VideoLayout: x in raster order,
                                   codes and scales in tile-major order)
   sta_plan(grid, tile, window) -> StaPlan (host CSR over 128-token blocks)
+  step_phase(t, num_steps)     -> 0 early / 1 middle / 2 late denoising phase
   attention_fwd(q, k, v, ...)  -> (out, lse) on quantized operands
   attention(q, k, v, ...)      -> (out, lse) from bf16 inputs: quantize + fwd;
                                   host (pinned) inputs are copied in and the
@@ -33,7 +36,7 @@ from . import _lib
 from ._lib import FpattnError
 
 __all__ = ["Nvfp4Tensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_fp8", "sta_plan",
-           "attention_fwd", "attention", "device_error", "library", "FpattnError"]
+           "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError"]
 
 
 def library() -> ctypes.CDLL:
@@ -113,7 +116,7 @@ def quantize_nvfp4(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
 
 def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
                  nonfinite_flag: Optional[torch.Tensor] = None,
-                 video: Optional[VideoLayout] = None) -> Fp8Tensor:
+                 video: Optional[VideoLayout] = None, group_tiles: int = 1) -> Fp8Tensor:
     B, H, N, d = _check_bf16(x)
     lib = library()
     codes = torch.empty((B, H, N, d), dtype=torch.uint8, device=x.device)
@@ -121,9 +124,16 @@ def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
         g, scales = _lib.FP8_TILE128, torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
     elif granularity == "channel":
         g, scales = _lib.FP8_CHANNEL, torch.empty((B, H, d), dtype=torch.float32, device=x.device)
+    elif granularity == "group":
+        g, scales = None, torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
     else:
-        raise ValueError("granularity must be 'tile128' or 'channel'")
+        raise ValueError("granularity must be 'tile128', 'channel' or 'group'")
     xd = ctypes.byref(_desc(x, _lib.BF16, B, H, N, d))
+    if g is None:
+        st = lib.fpattn_quantize_fp8_group(xd, _video_ref(video), int(group_tiles), codes.data_ptr(),
+                                           scales.data_ptr(), _ptr(nonfinite_flag), _stream())
+        _lib.check(st, "fpattn_quantize_fp8_group")
+        return Fp8Tensor(codes, scales, "tile128", (B, H, N, d))
     if video is None:
         st = lib.fpattn_quantize_fp8(xd, g, codes.data_ptr(), scales.data_ptr(), _ptr(nonfinite_flag), _stream())
     else:
@@ -182,6 +192,14 @@ def sta_plan(tile_grid: Sequence[int], tile: Sequence[int], window: Sequence[int
     return StaPlan(row_ptr, col_idx[:nnz.value], row_order)
 
 
+def step_phase(t: int, num_steps: int, alpha1: float = 0.2, alpha2: float = 0.7) -> int:
+    """Denoising phase of step t (1-based): 0 early, 1 middle, 2 late."""
+    ph = ctypes.c_int32(0)
+    _lib.check(library().fpattn_step_phase(int(t), int(num_steps), float(alpha1), float(alpha2), ctypes.byref(ph)),
+               "fpattn_step_phase")
+    return ph.value
+
+
 def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, return_lse: bool = True,
@@ -229,8 +247,13 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
               causal: bool = False, tile_mask: Optional[DeviceTileMask] = None, softmax_scale: float = 0.0,
               return_lse: bool = True, device: Optional[torch.device] = None,
               out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None,
-              video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0):
+              video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0,
+              qk_group_tiles: int = 1):
     """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
+
+    ``qk_group_tiles`` > 1 (FP8 Q/K only) shares one Q/K scale across that
+    many consecutive 128-token tiles (the coarser granularities of the
+    denoising-step schedule).
 
     CUDA inputs stay where they are. Host inputs (ideally pinned) are copied
     to ``device`` (default cuda:0) on the current stream, and the output (and
@@ -246,7 +269,9 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
     if qk_format == "nvfp4":
         qq, kq = quantize_nvfp4(q, video=video), quantize_nvfp4(k, video=video)
     elif qk_format == "fp8":
-        qq, kq = quantize_fp8(q, "tile128", video=video), quantize_fp8(k, "tile128", video=video)
+        gran = "group" if qk_group_tiles > 1 else "tile128"
+        qq = quantize_fp8(q, gran, video=video, group_tiles=qk_group_tiles)
+        kq = quantize_fp8(k, gran, video=video, group_tiles=qk_group_tiles)
     else:
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
     vq = quantize_fp8(v, "channel", video=video)

@@ -89,6 +89,21 @@ fpattn_status quantize_fp8(const fpattn_tensor* x, const fpattn_video_layout* la
   return FPATTN_ERR_INVALID_ARG;
 }
 
+fpattn_status quantize_fp8_group(const fpattn_tensor* x, const fpattn_video_layout* layout, int32_t group,
+                                 uint8_t* codes, float* scales, int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  if (layout && (s = check_layout(layout, x->N, &vl, &tm)) != FPATTN_OK) return s;
+  if (group < 1 || !codes || !scales) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FPATTN_ERR_ALIGNMENT;
+  const int nblk = (x->N + 127) / 128;
+  return from_cuda(fpattn::launch_quantize_fp8_group(x->data, x->B * x->H, x->N, x->d, std::min<int>(group, nblk),
+                                                     codes, scales, nonfinite_flag, layout ? &tm : nullptr,
+                                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
                   const fpattn_scales* scales, const fpattn_tile_mask_desc* tile_mask, int32_t causal,
                   const fpattn_video_layout* layout, void* out, float* lse, fpattn_stream_t stream) {
@@ -183,6 +198,21 @@ fpattn_status fpattn_quantize_fp8_video(const fpattn_tensor* x, const fpattn_vid
                                         fpattn_stream_t stream) {
   if (!layout) return FPATTN_ERR_INVALID_ARG;
   return quantize_fp8(x, layout, granularity, codes, scales, nonfinite_flag, stream);
+}
+
+fpattn_status fpattn_quantize_fp8_group(const fpattn_tensor* x, const fpattn_video_layout* layout,
+                                        int32_t group_tiles, uint8_t* codes, float* scales,
+                                        int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  return quantize_fp8_group(x, layout, group_tiles, codes, scales, nonfinite_flag, stream);
+}
+
+fpattn_status fpattn_step_phase(int32_t t, int32_t num_steps, double alpha1, double alpha2, int32_t* phase) {
+  if (!phase || num_steps < 1 || t < 1 || t > num_steps) return FPATTN_ERR_INVALID_ARG;
+  if (!(alpha1 >= 0.0 && alpha1 <= alpha2 && alpha2 <= 1.0)) return FPATTN_ERR_INVALID_ARG;
+  const double td = static_cast<double>(t);
+  *phase = td <= alpha1 * num_steps ? FPATTN_PHASE_EARLY
+                                    : (td <= alpha2 * num_steps ? FPATTN_PHASE_MIDDLE : FPATTN_PHASE_LATE);
+  return FPATTN_OK;
 }
 
 fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, int32_t th, int32_t tw, int32_t wt,

@@ -13,6 +13,9 @@ namespace fpattn {
 // read in raster order and the codes are written in tile-major order.
 cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                      int* nonfinite, const TokenMap* tmap, cudaStream_t st);
+// One scale per group of `group` consecutive 128-token tiles (group 1: per tile).
+cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int group, uint8_t* codes,
+                                      float* scales, int* nonfinite, const TokenMap* tmap, cudaStream_t st);
 cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                         int* nonfinite, const TokenMap* tmap, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const float* static_amax,

@@ -95,8 +95,14 @@ __device__ __forceinline__ uint2 quant8_e4m3(const uint4& v, float s) {
 // reduction and the conversion, so x is read from HBM exactly once. With a
 // token map (kMap) the tile's 128 source rows are looked up once into shared
 // memory.
+//
+// Grouped scales (one scale for several consecutive tiles) run the same
+// kernel twice around fp8_group_finalize_kernel: kAmaxOnly writes each tile's
+// amax into its scale slot, kConvert converts with the scale found there.
 // ---------------------------------------------------------------------------
-template <int D, bool kMap>
+enum TileMode { kFused = 0, kAmaxOnly = 1, kConvert = 2 };
+
+template <int D, bool kMap, int kMode = kFused>
 __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restrict__ x, int N,
                                                             uint2* __restrict__ codes, float* __restrict__ scales,
                                                             int* nonfinite, TokenMap tmap) {
@@ -121,18 +127,43 @@ __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restr
     const int c = threadIdx.x + i * kThreads;
     if (c / kChunksPerRow < rows) {
       v[i] = kMap ? x[(bh * N + src_row[c / kChunksPerRow]) * kChunksPerRow + c % kChunksPerRow] : x[base + c];
-      m = fmaxf(m, amax8(v[i], &bad));
+      if (kMode != kConvert) m = fmaxf(m, amax8(v[i], &bad));
     }
   }
-  if (bad && nonfinite) atomicExch(nonfinite, 1);
-  const float a = block_max(m, red);
-  const float s = fp8_scale_from_amax(a);
-  if (threadIdx.x == 0) scales[bh * gridDim.x + tile] = s;
+  float s;
+  if (kMode == kConvert) {
+    s = scales[bh * gridDim.x + tile];
+  } else {
+    if (bad && nonfinite) atomicExch(nonfinite, 1);
+    const float a = block_max(m, red);
+    if (kMode == kAmaxOnly) {
+      if (threadIdx.x == 0) scales[bh * gridDim.x + tile] = a;
+      return;
+    }
+    s = fp8_scale_from_amax(a);
+    if (threadIdx.x == 0) scales[bh * gridDim.x + tile] = s;
+  }
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int c = threadIdx.x + i * kThreads;
     if (c / kChunksPerRow < rows) codes[base + c] = quant8_e4m3(v[i], s);
   }
+}
+
+// One thread per (b*h, group of `group` tiles): the group's amax is the max of
+// its tiles' amaxes (left in the scale slots by the kAmaxOnly pass); every
+// tile of the group gets s = 448 / amax.
+__global__ void fp8_group_finalize_kernel(float* __restrict__ scales, int nblk, int group, int ngroups,
+                                          int total) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  float* sc = scales + static_cast<size_t>(i / ngroups) * nblk;
+  const int b0 = (i % ngroups) * group;
+  const int b1 = min(nblk, b0 + group);
+  float a = 0.f;
+  for (int b = b0; b < b1; ++b) a = fmaxf(a, sc[b]);
+  const float s = fp8_scale_from_amax(a);
+  for (int b = b0; b < b1; ++b) sc[b] = s;
 }
 
 // ---------------------------------------------------------------------------
@@ -342,6 +373,34 @@ cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_
   } else {
     if (tmap) fp8_tile_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
     else fp8_tile_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+  }
+  return cudaGetLastError();
+}
+
+template <int D, bool kMap>
+void launch_fp8_grouped(const uint4* xv, int BH, int N, int group, uint2* cv, float* scales, int* nonfinite,
+                        const TokenMap& tm, cudaStream_t st) {
+  const int nblk = (N + 127) / 128;
+  dim3 grid(nblk, BH);
+  fp8_tile_kernel<D, kMap, kAmaxOnly><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+  const int ngroups = (nblk + group - 1) / group;
+  const int total = BH * ngroups;
+  fp8_group_finalize_kernel<<<(total + 255) / 256, 256, 0, st>>>(scales, nblk, group, ngroups, total);
+  fp8_tile_kernel<D, kMap, kConvert><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+}
+
+cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int group, uint8_t* codes,
+                                      float* scales, int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
+  if (group <= 1) return launch_quantize_fp8_tile(x, BH, N, d, codes, scales, nonfinite, tmap, st);
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint2* cv = reinterpret_cast<uint2*>(codes);
+  const TokenMap tm = tmap ? *tmap : TokenMap{};
+  if (d == 128) {
+    if (tmap) launch_fp8_grouped<128, true>(xv, BH, N, group, cv, scales, nonfinite, tm, st);
+    else launch_fp8_grouped<128, false>(xv, BH, N, group, cv, scales, nonfinite, tm, st);
+  } else {
+    if (tmap) launch_fp8_grouped<64, true>(xv, BH, N, group, cv, scales, nonfinite, tm, st);
+    else launch_fp8_grouped<64, false>(xv, BH, N, group, cv, scales, nonfinite, tm, st);
   }
   return cudaGetLastError();
 }

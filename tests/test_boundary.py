@@ -210,3 +210,35 @@ def test_video_argument_errors(lib):
                                 ctypes.byref(rej), p16, None, None) == _lib.ERR_INVALID_ARG
     assert lib.fpattn_fwd_video(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(sc), None, 0,
                                 ctypes.byref(ragged), p16, None, None) == _lib.ERR_UNSUPPORTED
+
+
+def test_step_phase_matches_oracle(lib):
+    from oracle import schedule
+    ph = ctypes.c_int32(-1)
+    cases = [(t, D, a1, a2) for D in (1, 7, 10, 49, 50, 1000) for t in sorted({1, 2, D // 5, D // 5 + 1, D // 2,
+                                                                               (7 * D) // 10, (7 * D) // 10 + 1,
+                                                                               D - 1, D} - {0})
+             for a1, a2 in ((0.2, 0.7), (0.0, 1.0), (0.5, 0.5), (0.1, 0.3), (1 / 3, 2 / 3))]
+    for t, D, a1, a2 in cases:
+        if not 1 <= t <= D:
+            continue
+        assert lib.fpattn_step_phase(t, D, a1, a2, ctypes.byref(ph)) == _lib.OK
+        assert ph.value == schedule.step_phase(t, D, a1, a2), (t, D, a1, a2)
+    for bad in ((0, 10, 0.2, 0.7), (11, 10, 0.2, 0.7), (1, 0, 0.2, 0.7), (1, 10, 0.8, 0.7),
+                (1, 10, -0.1, 0.7), (1, 10, 0.2, 1.5), (1, 10, float("nan"), 0.7)):
+        assert lib.fpattn_step_phase(*bad, ctypes.byref(ph)) == _lib.ERR_INVALID_ARG, bad
+    assert lib.fpattn_step_phase(1, 10, 0.2, 0.7, None) == _lib.ERR_INVALID_ARG
+
+
+def test_quantize_fp8_group_argument_errors(lib):
+    buf = (ctypes.c_uint8 * 4096)()
+    p16 = (ctypes.addressof(buf) + 15) & ~15
+    x = _t(p16, _lib.BF16)
+    assert lib.fpattn_quantize_fp8_group(ctypes.byref(x), None, 0, p16, p16, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_quantize_fp8_group(ctypes.byref(x), None, 2, None, p16, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_quantize_fp8_group(ctypes.byref(x), None, 2, p16 + 4, p16, None, None) == _lib.ERR_ALIGNMENT
+    assert lib.fpattn_quantize_fp8_group(ctypes.byref(_t(p16, _lib.BF16, d=96)), None, 2, p16, p16, None,
+                                         None) == _lib.ERR_UNSUPPORTED
+    ragged = _lib.VideoLayout(1, 8, 16, 1, 3, 16)
+    assert lib.fpattn_quantize_fp8_group(ctypes.byref(x), ctypes.byref(ragged), 2, p16, p16, None,
+                                         None) == _lib.ERR_UNSUPPORTED
