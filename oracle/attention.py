@@ -32,6 +32,15 @@ code below the E4M3 maximum:
       Ph_j = E4M3(448 * 2^-tau * P_j) / (448 * 2^-tau).
 tau = 0 is the exact running max above.
 
+All-NVFP4 variant (``p_format="nvfp4"``): P is quantized with the NVFP4
+recipe of oracle.quant (Blackwell FP4 page, section 1: blocks of 16 along the
+keys of the tile, E4M3 block scales) with its tensor amax fixed at 2^tau, the
+bound of P under the reference max. This is the 4-bit counterpart of the fixed
+FP8 P scale; the pages give no P rule for FP4, so this is the reading:
+      Ph_j = NVFP4(P_j; A_t = 2^tau)   (P widened to float32 first)
+V is then quantized along the sequence (oracle.quant.quantize_nvfp4_tokens),
+which only changes the dequantized v passed in.
+
 Allowed keys: all keys < N; under ``causal`` only j <= i; under a tile mask
 only keys whose 128-key block is listed for the query's 128-row block.
 
@@ -50,14 +59,22 @@ from typing import Optional, Sequence
 
 import numpy as np
 
-from . import codec
+from . import codec, quant
 
 TILE = 128
 P_SCALE_INV = 448.0
 LOG2E = 1.0 / math.log(2.0)
 
 
-def _quantize_p(p: np.ndarray, tau: float = 0.0) -> np.ndarray:
+def _quantize_p(p: np.ndarray, tau: float = 0.0, fmt: str = "e4m3") -> np.ndarray:
+    if fmt == "nvfp4":
+        R, K = p.shape
+        Kp = -(-K // quant.NVFP4_BLOCK) * quant.NVFP4_BLOCK
+        pp = np.zeros((R, Kp), dtype=np.float32)
+        pp[:, :K] = p.astype(np.float32)
+        codes, sb, s_t = quant.quantize_nvfp4(pp, static_amax=2.0 ** tau)
+        return quant.dequantize_nvfp4(codes, sb, s_t)[:, :K]
+    assert fmt == "e4m3"
     s = P_SCALE_INV * 2.0 ** -tau
     return codec.e4m3_decode(codec.e4m3_encode(p * s)) / s
 
@@ -65,7 +82,7 @@ def _quantize_p(p: np.ndarray, tau: float = 0.0) -> np.ndarray:
 def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray,
                    *, softmax_scale: Optional[float] = None, causal: bool = False,
                    key_blocks: Optional[Sequence[Sequence[int]]] = None,
-                   quantize_p: bool = True, rescale_threshold: float = 0.0):
+                   quantize_p: bool = True, rescale_threshold: float = 0.0, p_format: str = "e4m3"):
     """Attention output and lse for the query ``rows`` of one (batch, head).
 
     q, k, v     float64 [N, d] dequantized operands
@@ -73,6 +90,7 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray
     key_blocks  optional list: key_blocks[qb] = allowed 128-key block indices
                 for query block qb (the tile mask); None = dense
     rescale_threshold  tau of the conditional rescale (log2 units), 0 = exact
+    p_format    "e4m3" (fixed 1/448 scale) or "nvfp4" (see the module notes)
     Returns (out float64 [len(rows), d], lse float64 [len(rows)]).
     """
     tau = float(rescale_threshold)
@@ -114,7 +132,7 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray
             alpha = np.where(live, np.exp(m - m_new), 1.0)
             P = np.where(allowed, np.exp(S - m_new[:, None]), 0.0)
         l = l * alpha + P.sum(axis=1)
-        Ph = _quantize_p(P, tau) if quantize_p else P
+        Ph = _quantize_p(P, tau, p_format) if quantize_p else P
         O = O * alpha[:, None] + Ph @ v[keys]
         m = m_new
     with np.errstate(invalid="ignore", divide="ignore"):
@@ -124,7 +142,7 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray
 
 
 def attention(q, k, v, *, softmax_scale=None, causal=False, key_blocks=None,
-              quantize_p=True, rescale_threshold=0.0):
+              quantize_p=True, rescale_threshold=0.0, p_format="e4m3"):
     """Whole (batch, head) attention, 128 rows at a time. Returns (out, lse)."""
     N = q.shape[0]
     outs, lses = [], []
@@ -132,7 +150,7 @@ def attention(q, k, v, *, softmax_scale=None, causal=False, key_blocks=None,
         rows = np.arange(b0, min(b0 + TILE, N))
         o, s = attention_rows(q, k, v, rows, softmax_scale=softmax_scale, causal=causal,
                               key_blocks=key_blocks, quantize_p=quantize_p,
-                              rescale_threshold=rescale_threshold)
+                              rescale_threshold=rescale_threshold, p_format=p_format)
         outs.append(o)
         lses.append(s)
     return np.concatenate(outs), np.concatenate(lses)

@@ -87,6 +87,29 @@ def dequantize_nvfp4(codes, block_scales, s_t) -> np.ndarray:
     return v * sbv * float(s_t)
 
 
+def quantize_nvfp4_tokens(v, pad_to: int = 128):
+    """NVFP4 for V as the second operand of a block-scaled P V product: the
+    same recipe as quantize_nvfp4 (tensor amax over all of ``v``), with the
+    16-element blocks running along the sequence (the contraction axis of
+    P V) instead of along d.
+
+    ``v`` [..., N, d]. The sequence is zero-padded to a multiple of
+    ``pad_to`` tokens. Returns (codes uint8 [..., d, Np], block_scales uint8
+    [..., d, Np/16], s_t): channel-major, tokens along the last axis.
+    """
+    v = _f32(v)
+    N = v.shape[-2]
+    Np = -(-N // pad_to) * pad_to
+    vt = np.zeros(v.shape[:-2] + (v.shape[-1], Np), dtype=F32)
+    vt[..., :N] = np.swapaxes(v, -1, -2)
+    return quantize_nvfp4(vt)
+
+
+def dequantize_nvfp4_tokens(codes, block_scales, s_t, N: int) -> np.ndarray:
+    """Inverse arrangement of quantize_nvfp4_tokens: float64 [..., N, d]."""
+    return np.swapaxes(dequantize_nvfp4(codes, block_scales, s_t), -1, -2)[..., :N, :]
+
+
 def nvfp4_sf_swizzle(block_scales: np.ndarray, N: int, d: int) -> np.ndarray:
     """Arrange logical block scales [BH, N, d/16] into the tensor-core layout.
 

@@ -250,3 +250,40 @@ def test_tile_major_raster_index_is_tile_contiguous_bijection():
     # tiles themselves in raster order over the 2 x 2 x 3 tile grid
     firsts = [(t[i] // 6, h[i] // 8, w[i] // 8) for i in range(0, N, vol)]
     assert firsts == [(a, b, c) for a in range(2) for b in range(2) for c in range(3)]
+
+
+def test_nvfp4_p_worked_example():
+    # One tile, keys 0 and 1 score 0 and ln 0.3, the rest -1000 (P = 0).
+    # P's tensor amax is fixed at 1: s_t = 1/2688, and the first 16-key block
+    # has A_b = 1 -> sb = E4M3(448) = 448, den = 448/2688 = 1/6.
+    # Codes: 1 * 6 = 6 -> 6; 0.3 * 6 = 1.8 -> 2 (E2M1 grid 1.5, 2).
+    # P_hat = [1, 2/6]; l uses the unquantized P.
+    N = 128
+    q = np.ones((1, 1))
+    k = np.full((N, 1), -1000.0)
+    k[0, 0] = 0.0
+    k[1, 0] = math.log(0.3)
+    v = np.zeros((N, 2))
+    v[0, 0] = v[1, 1] = 1.0
+    out, lse = A.attention_rows(q, k, v, np.array([0]), softmax_scale=1.0, p_format="nvfp4")
+    assert out[0].tolist() == pytest.approx([1.0 / 1.3, (1.0 / 3.0) / 1.3], rel=1e-6)
+    assert lse[0] == pytest.approx(math.log(1.3), rel=1e-12)
+
+
+def test_nvfp4_p_small_block_scale():
+    # Tile 0: key 0 at score 0 (P = 1). Keys 16 and 17 (the second 16-key
+    # block) at ln 0.01 and ln 0.004: that block's A_b = 0.01, sb =
+    # E4M3(4.48) = 4.5 (grid step 0.5 in [4, 8)), den = 4.5/2688.
+    # Codes: 0.01 * 2688/4.5 = 5.973 -> 6; 0.004 * 2688/4.5 = 2.389 -> 2.
+    N = 128
+    q = np.ones((1, 1))
+    k = np.full((N, 1), -1000.0)
+    k[0, 0] = 0.0
+    k[16, 0] = math.log(0.01)
+    k[17, 0] = math.log(0.004)
+    v = np.zeros((N, 3))
+    v[0, 0] = v[16, 1] = v[17, 2] = 1.0
+    out, _ = A.attention_rows(q, k, v, np.array([0]), softmax_scale=1.0, p_format="nvfp4")
+    l = 1.0 + 0.01 + 0.004
+    step = 4.5 / 2688.0
+    assert out[0].tolist() == pytest.approx([1.0 / l, 6 * step / l, 2 * step / l], rel=1e-6)

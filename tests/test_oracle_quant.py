@@ -200,3 +200,32 @@ def test_step_phase_worked_example():
     assert got == [schedule.EARLY] * 10 + [schedule.MIDDLE] * 25 + [schedule.LATE] * 15
     # D = 7: t1 = 1.4, t2 = 4.9 -> steps 1 | 2..4 | 5..7
     assert [schedule.step_phase(t, 7) for t in range(1, 8)] == [0, 1, 1, 1, 2, 2, 2]
+
+
+def test_nvfp4_tokens_grid_values_survive_and_padding_is_zero():
+    # V [N = 40, d = 32]: in channel c, token block b (16 tokens) holds E2M1
+    # grid values times a scale that E4M3 represents exactly, with one element
+    # at 6 * scale so the block's amax is 6 * scale. Channel 0, block 0 has
+    # scale 448, which puts the tensor amax at 2688 and s_t at exactly 1. Then
+    # every block scale encodes exactly and dequantize(quantize(v)) == v.
+    # Tokens 40..127 are padding: zero codes and zero scales.
+    rng = np.random.default_rng(21)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    N, d = 40, 32
+    v = np.zeros((N, d), dtype=np.float64)
+    scale = np.zeros((d, 3))
+    for c in range(d):
+        for b in range(3):
+            t0, t1 = 16 * b, min(N, 16 * b + 16)
+            vals = rng.choice(grid, t1 - t0) * rng.choice([-1, 1], t1 - t0)
+            vals[0] = 6.0
+            scale[c, b] = 448.0 if (c, b) == (0, 0) else 2.0 ** -(c % 5) * (b + 1)
+            v[t0:t1, c] = vals * scale[c, b]
+    codes, sb, s_t = quant.quantize_nvfp4_tokens(v.astype(np.float32))
+    assert codes.shape == (d, 128) and sb.shape == (d, 8)
+    assert s_t == np.float32(1.0)
+    back = quant.dequantize_nvfp4_tokens(codes, sb, s_t, N)
+    assert np.array_equal(back, v)
+    assert np.all(codes[:, 48:] == 0) and np.all(sb[:, 3:] == 0)
+    # blocks run along tokens: (channel c, token block b) has scale[c, b]
+    assert np.array_equal(codec.e4m3_decode(sb[:, :3]), scale)
