@@ -81,14 +81,17 @@ def executed_block_pairs(w: workloads.Workload) -> int:
     return nblk * (nblk + 1) // 2 if w.causal else nblk * nblk
 
 
-def quant_bytes(w: workloads.Workload) -> float:
+def quant_bytes(w: workloads.Workload, pv_format: str = "fp8") -> float:
     """Algorithmic HBM bytes of one step's quantization (two-pass amax)."""
     n = w.B * w.H * w.N * w.d
     if w.qk_format == "nvfp4":
         qk = 2 * n * (2 + 2 + 0.5 + 1.0 / 16)   # amax read + quant read + codes + scales
     else:
         qk = 2 * n * (2 + 1)                    # single pass per 128-token tile
-    v = n * (2 + 2 + 1)                         # channel amax pass + quant pass
+    if pv_format == "nvfp4":
+        v = n * (2 + 2 + 0.5 + 1.0 / 16)        # tensor amax pass + quant pass (codes + scales)
+    else:
+        v = n * (2 + 2 + 1)                     # channel amax pass + quant pass
     return qk + v
 
 
@@ -338,6 +341,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--pv-format", default="fp8", choices=["fp8", "nvfp4"],
+                    help="P and V in E4M3 (default) or both in NVFP4 with P V on FP4 tensor cores")
     ap.add_argument("--rescale-threshold", type=float, default=0.0,
                     help="conditional softmax rescale threshold tau (log2 units); 0 = exact running max")
     args = ap.parse_args()
@@ -380,7 +385,10 @@ def main():
             qq, kq = fp.quantize_nvfp4(q, video=video), fp.quantize_nvfp4(k, video=video)
         else:
             qq, kq = fp.quantize_fp8(q, "tile128", video=video), fp.quantize_fp8(k, "tile128", video=video)
-        vq = fp.quantize_fp8(v, "channel", video=video)
+        if args.pv_format == "nvfp4":
+            vq = fp.quantize_nvfp4_v(v, video=video)
+        else:
+            vq = fp.quantize_fp8(v, "channel", video=video)
         if ev_pair is not None:
             ev_pair[0].record(stream)
         out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask, video=video,
@@ -425,10 +433,13 @@ def main():
     peaks, peak_src = load_peaks()
     bf16 = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
-    peak = 2.0 / (1.0 / p4 + 1.0 / p8) if w.qk_format == "nvfp4" else p8
+    # both MMAs do 2d flops per score: the peak is the harmonic mean of theirs
+    p_qk = p4 if w.qk_format == "nvfp4" else p8
+    p_pv = p4 if args.pv_format == "nvfp4" else p8
+    peak = 2.0 / (1.0 / p_qk + 1.0 / p_pv)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     quant_ms = ms_step - attn_ms
-    quant_gbs = quant_bytes(w) / (quant_ms * 1e-3) / 1e9
+    quant_gbs = quant_bytes(w, args.pv_format) / (quant_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host bf16 in, host bf16 out
     e2e = None
@@ -437,14 +448,16 @@ def main():
         out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
         lse_h = torch.empty(q_h.shape[:3], dtype=torch.float32, pin_memory=True)
         fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
-                     lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold)
+                     lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold,
+                     pv_format=args.pv_format)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         e0.record(stream)
         for _ in range(args.e2e_steps):
             fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
-                         lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold)
+                         lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold,
+                         pv_format=args.pv_format)
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = rank_max(e0.elapsed_time(e1) / args.e2e_steps)
@@ -467,6 +480,8 @@ def main():
                          f"{sorted(set(h for h, _ in done))} x query blocks {qblocks} in that order (fp64 "
                          f"numpy oracle, its quantization of those heads included), {s:.1f} s"}
 
+    # Q/K: NVFP4 amax + quantize + finalize each, or one FP8 kernel each; V: three kernels
+    # (FP8 channel or NVFP4); attention: one
     launches_per_step = (6 if w.qk_format == "nvfp4" else 2) + 3 + 1
     if rank == 0:
         line = {
@@ -474,7 +489,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e2m1/e4m3 MMA, f32 accumulate", "data": "synthetic",
             "config": dict(config_dict(w), **({"rescale_threshold": args.rescale_threshold}
-                                              if args.rescale_threshold else {})),
+                                              if args.rescale_threshold else {}),
+                           **({"pv": "nvfp4"} if args.pv_format == "nvfp4" else {})),
             "attn_ms": attn_ms, "attn_tflops_algorithmic": attn_tflops,
             "attn_tflops_dense_eq": w.dense_flops() / (attn_ms * 1e-3) / 1e12,
             "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,
@@ -483,7 +499,8 @@ def main():
                          "frac": attn_tflops / peak,
                          "traffic": profiled_traffic() if w.name == "llm_prefill_causal" else None,
                          "peak_source": f"{peak_src} bf16 sustained {bf16} x nominal fp8 2x / fp4 4x; "
-                                        f"{'harmonic mix of fp4 QK and fp8 PV' if w.qk_format == 'nvfp4' else 'fp8'}"},
+                                        f"QK {'fp4' if w.qk_format == 'nvfp4' else 'fp8'}, "
+                                        f"PV {'fp4' if args.pv_format == 'nvfp4' else 'fp8'}, harmonic mean"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk, "device_error": err,
         }

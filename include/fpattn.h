@@ -168,13 +168,41 @@ fpattn_status fpattn_quantize_fp8_group(const fpattn_tensor* x, const struct fpa
 typedef enum { FPATTN_PHASE_EARLY = 0, FPATTN_PHASE_MIDDLE = 1, FPATTN_PHASE_LATE = 2 } fpattn_phase;
 fpattn_status fpattn_step_phase(int32_t t, int32_t num_steps, double alpha1, double alpha2, int32_t* phase);
 
+/*
+ * NVFP4 quantization of V for the all-NVFP4 attention (P and V in NVFP4, P V
+ * on block-scaled FP4 tensor cores). Same two-level recipe as
+ * fpattn_quantize_nvfp4 (Blackwell FP4 practice page, section 1; tensor amax
+ * over all of V, or *static_amax), but the 16-element blocks run along the
+ * sequence, the contraction axis of P V, and the result is channel-major:
+ *
+ *   codes     device, fpattn_nvfp4_v_bytes() bytes: [B, H, d, Np/2] with
+ *             Np = 128 * ceil(N/128); byte t/2 of row (b, h, c) holds
+ *             tokens t (low nibble) and t+1; tokens >= N are 0
+ *   block_sf  device, *block_sf_bytes bytes: per (b, h) and 128-token block
+ *             kb, two 512-byte groups g (tokens 64g .. 64g+63): the E4M3
+ *             scale of channel c = 32j + i and token block 4g + s at byte
+ *             16i + 4j + s (the tensor-core scale layout with channels as
+ *             rows; rows >= d are 0)
+ *   tensor_scale  device float: s_t = A_t / 2688
+ *
+ * layout: NULL, or x in raster order of a video (tokens permuted to
+ * tile-major order on the way, as in fpattn_quantize_fp8_video). Pass the
+ * codes as an FPATTN_NVFP4 tensor [B, H, N, d] to fpattn_fwd with
+ * scales.v_scale = tensor_scale and scales.v_block_sf = block_sf.
+ */
+size_t fpattn_nvfp4_v_bytes(int32_t B, int32_t H, int32_t N, int32_t d, size_t* block_sf_bytes);
+fpattn_status fpattn_quantize_nvfp4_v(const fpattn_tensor* x, const struct fpattn_video_layout_s* layout,
+                                      const float* static_amax, uint8_t* codes, uint8_t* block_sf,
+                                      float* tensor_scale, int32_t* nonfinite_flag, fpattn_stream_t stream);
+
 /* Scales consumed by fpattn_fwd. */
 typedef struct {
   /* NVFP4 Q/K: device pointer to the one-float tensor scale s_t.
      E4M3 Q/K: device pointer to B*H*ceil(N/128) per-tile multipliers. */
   const float* q_scale;
   const float* k_scale;
-  /* E4M3 V: device pointer to B*H*d per-channel multipliers. */
+  /* E4M3 V: device pointer to B*H*d per-channel multipliers.
+     NVFP4 V: device pointer to its one-float tensor scale s_t. */
   const float* v_scale;
   /* NVFP4 Q/K: device block scales in the tensor-core scale layout; else NULL. */
   const uint8_t* q_block_sf;
@@ -194,6 +222,8 @@ typedef struct {
      2^-tau is applied inside the kernel and cancels in O / l). Outside
      [0, 8]: FPATTN_ERR_INVALID_ARG. */
   float rescale_threshold;
+  /* NVFP4 V (fpattn_quantize_nvfp4_v): device block scales; else NULL. */
+  const uint8_t* v_block_sf;
 } fpattn_scales;
 
 /*
@@ -241,7 +271,12 @@ fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, in
  * q, k        both FPATTN_NVFP4 (QK^T on block-scaled FP4 tensor cores) or
  *             both FPATTN_E4M3 (FP8 tensor cores)
  * v           FPATTN_E4M3 with per-channel scales (PV on FP8 tensor cores,
- *             P in E4M3 at scale 1/448)
+ *             P in E4M3 at scale 1/448), or FPATTN_NVFP4 from
+ *             fpattn_quantize_nvfp4_v: all-NVFP4 attention, P quantized to
+ *             NVFP4 in 16-key blocks with its tensor amax fixed at 2^tau (the
+ *             bound of P under the reference max; the pages give no P rule
+ *             for FP4, this is the library's reading) and P V on block-scaled
+ *             FP4 tensor cores
  * scales      as described in fpattn_scales
  * tile_mask   NULL for dense, else a block mask (may be combined with causal)
  * causal      nonzero: key j attends query i only when j <= i

@@ -12,6 +12,8 @@ Public calls
                                   group_tiles tiles per scale
                                   (with video=VideoLayout: x in raster order,
                                   codes and scales in tile-major order)
+  quantize_nvfp4_v(x)          -> Nvfp4VTensor: V in NVFP4 with 16-token
+                                  blocks, channel-major (all-NVFP4 attention)
   sta_plan(grid, tile, window) -> StaPlan (host CSR over 128-token blocks)
   step_phase(t, num_steps)     -> 0 early / 1 middle / 2 late denoising phase
   attention_fwd(q, k, v, ...)  -> (out, lse) on quantized operands
@@ -35,7 +37,8 @@ import torch
 from . import _lib
 from ._lib import FpattnError
 
-__all__ = ["Nvfp4Tensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_fp8", "sta_plan",
+__all__ = ["Nvfp4Tensor", "Nvfp4VTensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4",
+           "quantize_nvfp4_v", "quantize_fp8", "sta_plan",
            "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError"]
 
 
@@ -88,6 +91,14 @@ class Nvfp4Tensor:
 
 
 @dataclasses.dataclass
+class Nvfp4VTensor:
+    codes: torch.Tensor         # uint8 [B, H, d, 64*ceil(N/128)], packed E2M1 along tokens
+    block_sf: torch.Tensor      # uint8 [B*H*ceil(N/128)*1024], tensor-core layout, channels as rows
+    tensor_scale: torch.Tensor  # float32 [1]
+    shape: Tuple[int, int, int, int]
+
+
+@dataclasses.dataclass
 class Fp8Tensor:
     codes: torch.Tensor         # uint8 [B, H, N, d] (E4M3 bits)
     scales: torch.Tensor        # float32 [B, H, ceil(N/128)] or [B, H, d]
@@ -112,6 +123,24 @@ def quantize_nvfp4(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
                                              sf.data_ptr(), ts.data_ptr(), _ptr(nonfinite_flag), _stream())
     _lib.check(st, "fpattn_quantize_nvfp4" + ("_video" if video is not None else ""))
     return Nvfp4Tensor(codes, sf, ts, (B, H, N, d))
+
+
+def quantize_nvfp4_v(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
+                     nonfinite_flag: Optional[torch.Tensor] = None,
+                     video: Optional[VideoLayout] = None) -> Nvfp4VTensor:
+    """V for the all-NVFP4 attention: NVFP4 blocks of 16 tokens, channel-major."""
+    B, H, N, d = _check_bf16(x)
+    lib = library()
+    sfb = ctypes.c_size_t(0)
+    nbytes = lib.fpattn_nvfp4_v_bytes(B, H, N, d, ctypes.byref(sfb))
+    codes = torch.empty((B, H, d, nbytes // (B * H * d)), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(sfb.value, dtype=torch.uint8, device=x.device)
+    ts = torch.empty(1, dtype=torch.float32, device=x.device)
+    st = lib.fpattn_quantize_nvfp4_v(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), _video_ref(video),
+                                     _ptr(static_amax), codes.data_ptr(), sf.data_ptr(), ts.data_ptr(),
+                                     _ptr(nonfinite_flag), _stream())
+    _lib.check(st, "fpattn_quantize_nvfp4_v")
+    return Nvfp4VTensor(codes, sf, ts, (B, H, N, d))
 
 
 def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
@@ -200,13 +229,14 @@ def step_phase(t: int, num_steps: int, alpha1: float = 0.2, alpha2: float = 0.7)
     return ph.value
 
 
-def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
+def attention_fwd(q, k, v, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, return_lse: bool = True,
                   video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0):
     """Fused attention on quantized operands.
 
-    q, k: both Nvfp4Tensor or both Fp8Tensor (tile128); v: Fp8Tensor (channel).
+    q, k: both Nvfp4Tensor or both Fp8Tensor (tile128); v: Fp8Tensor
+    (channel), or Nvfp4VTensor for the all-NVFP4 attention (P and V in NVFP4).
     Returns (out bf16 [B,H,N,d], lse float32 [B,H,N] or None). With ``video``
     the operands are in tile-major order and out / lse come back in raster
     order. ``rescale_threshold`` (tau, log2 units, 0..8) skips the O / l
@@ -214,20 +244,23 @@ def attention_fwd(q, k, v: Fp8Tensor, *, causal: bool = False, tile_mask: Option
     """
     B, H, N, d = v.shape
     lib = library()
+    if isinstance(v, Nvfp4VTensor):
+        vd, v_scale, v_sf = _desc(v.codes, _lib.NVFP4, B, H, N, d), v.tensor_scale.data_ptr(), v.block_sf.data_ptr()
+    else:
+        vd, v_scale, v_sf = _desc(v.codes, _lib.E4M3, B, H, N, d), v.scales.data_ptr(), None
     if isinstance(q, Nvfp4Tensor) and isinstance(k, Nvfp4Tensor):
         qd = _desc(q.codes, _lib.NVFP4, B, H, N, d)
         kd = _desc(k.codes, _lib.NVFP4, B, H, N, d)
-        sc = _lib.Scales(q.tensor_scale.data_ptr(), k.tensor_scale.data_ptr(), v.scales.data_ptr(),
+        sc = _lib.Scales(q.tensor_scale.data_ptr(), k.tensor_scale.data_ptr(), v_scale,
                          q.block_sf.data_ptr(), k.block_sf.data_ptr(), 1.0 / 448.0, softmax_scale,
-                         rescale_threshold)
+                         rescale_threshold, v_sf)
     elif isinstance(q, Fp8Tensor) and isinstance(k, Fp8Tensor):
         qd = _desc(q.codes, _lib.E4M3, B, H, N, d)
         kd = _desc(k.codes, _lib.E4M3, B, H, N, d)
-        sc = _lib.Scales(q.scales.data_ptr(), k.scales.data_ptr(), v.scales.data_ptr(), None, None,
-                         1.0 / 448.0, softmax_scale, rescale_threshold)
+        sc = _lib.Scales(q.scales.data_ptr(), k.scales.data_ptr(), v_scale, None, None,
+                         1.0 / 448.0, softmax_scale, rescale_threshold, v_sf)
     else:
         raise TypeError("q and k must both be Nvfp4Tensor or both Fp8Tensor")
-    vd = _desc(v.codes, _lib.E4M3, B, H, N, d)
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.codes.device)
     if lse is None and return_lse:
@@ -248,12 +281,13 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
               return_lse: bool = True, device: Optional[torch.device] = None,
               out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None,
               video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0,
-              qk_group_tiles: int = 1):
+              qk_group_tiles: int = 1, pv_format: str = "fp8"):
     """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
 
     ``qk_group_tiles`` > 1 (FP8 Q/K only) shares one Q/K scale across that
     many consecutive 128-token tiles (the coarser granularities of the
-    denoising-step schedule).
+    denoising-step schedule). ``pv_format="nvfp4"`` quantizes P and V to
+    NVFP4 and runs P V on the block-scaled FP4 tensor cores.
 
     CUDA inputs stay where they are. Host inputs (ideally pinned) are copied
     to ``device`` (default cuda:0) on the current stream, and the output (and
@@ -274,7 +308,12 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
         kq = quantize_fp8(k, gran, video=video, group_tiles=qk_group_tiles)
     else:
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
-    vq = quantize_fp8(v, "channel", video=video)
+    if pv_format == "fp8":
+        vq = quantize_fp8(v, "channel", video=video)
+    elif pv_format == "nvfp4":
+        vq = quantize_nvfp4_v(v, video=video)
+    else:
+        raise ValueError("pv_format must be 'fp8' or 'nvfp4'")
     out, lse = attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
                              return_lse=return_lse, video=video, rescale_threshold=rescale_threshold)
     if host:

@@ -21,7 +21,7 @@ class Scales(ctypes.Structure):
     _fields_ = [("q_scale", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("q_block_sf", ctypes.c_void_p), ("k_block_sf", ctypes.c_void_p),
                 ("p_scale", ctypes.c_float), ("softmax_scale", ctypes.c_float),
-                ("rescale_threshold", ctypes.c_float)]
+                ("rescale_threshold", ctypes.c_float), ("v_block_sf", ctypes.c_void_p)]
 
 
 class TileMask(ctypes.Structure):
@@ -47,6 +47,9 @@ _SIGNATURES = {
                                                    ctypes.c_void_p]),
     "fpattn_quantize_fp8_video": (ctypes.c_int, [_P(Tensor), _P(VideoLayout), ctypes.c_int32, ctypes.c_void_p,
                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "fpattn_nvfp4_v_bytes": (ctypes.c_size_t, [ctypes.c_int32] * 4 + [_P(ctypes.c_size_t)]),
+    "fpattn_quantize_nvfp4_v": (ctypes.c_int, [_P(Tensor), _P(VideoLayout), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "fpattn_quantize_fp8_group": (ctypes.c_int, [_P(Tensor), _P(VideoLayout), ctypes.c_int32, ctypes.c_void_p,
                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "fpattn_step_phase": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_double, ctypes.c_double,

@@ -89,6 +89,23 @@ fpattn_status quantize_fp8(const fpattn_tensor* x, const fpattn_video_layout* la
   return FPATTN_ERR_INVALID_ARG;
 }
 
+fpattn_status quantize_nvfp4_v(const fpattn_tensor* x, const fpattn_video_layout* layout, const float* static_amax,
+                              uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int32_t* nonfinite_flag,
+                              fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  if (layout && (s = check_layout(layout, x->N, &vl, &tm)) != FPATTN_OK) return s;
+  if (!codes || !block_sf || !tensor_scale) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(block_sf) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+    return FPATTN_ERR_ALIGNMENT;
+  return from_cuda(fpattn::launch_quantize_nvfp4_tokens(x->data, x->B * x->H, x->N, x->d, static_amax, codes,
+                                                        block_sf, tensor_scale, nonfinite_flag,
+                                                        layout ? &tm : nullptr,
+                                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fpattn_status quantize_fp8_group(const fpattn_tensor* x, const fpattn_video_layout* layout, int32_t group,
                                  uint8_t* codes, float* scales, int32_t* nonfinite_flag, fpattn_stream_t stream) {
   fpattn_status s = check_tensor(x, FPATTN_BF16);
@@ -113,7 +130,8 @@ fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_t
   fpattn_status s;
   if ((s = check_tensor(q, qk_dtype)) != FPATTN_OK) return s;
   if ((s = check_tensor(k, qk_dtype)) != FPATTN_OK) return s;
-  if ((s = check_tensor(v, FPATTN_E4M3)) != FPATTN_OK) return s;
+  const bool pv4 = v->dtype == FPATTN_NVFP4;
+  if ((s = check_tensor(v, pv4 ? FPATTN_NVFP4 : FPATTN_E4M3)) != FPATTN_OK) return s;
   if (k->B != q->B || k->H != q->H || k->N != q->N || k->d != q->d || v->B != q->B || v->H != q->H ||
       v->N != q->N || v->d != q->d)
     return FPATTN_ERR_INVALID_ARG;
@@ -125,6 +143,8 @@ fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_t
   const bool fp4 = qk_dtype == FPATTN_NVFP4;
   if (fp4 && (!scales->q_block_sf || !scales->k_block_sf)) return FPATTN_ERR_INVALID_ARG;
   if (fp4 && (!aligned16(scales->q_block_sf) || !aligned16(scales->k_block_sf))) return FPATTN_ERR_ALIGNMENT;
+  if (pv4 && !scales->v_block_sf) return FPATTN_ERR_INVALID_ARG;
+  if (pv4 && !aligned16(scales->v_block_sf)) return FPATTN_ERR_ALIGNMENT;
   // P is stored in E4M3 at the fixed scale 1/448.
   if (!(scales->p_scale > 0.f) || std::abs(scales->p_scale * 448.f - 1.f) > 1e-6f) return FPATTN_ERR_INVALID_ARG;
   if (!(scales->softmax_scale >= 0.f) || scales->softmax_scale > 1e30f) return FPATTN_ERR_INVALID_ARG;
@@ -140,6 +160,8 @@ fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_t
   a.v = v->data;
   a.q_sf = fp4 ? scales->q_block_sf : nullptr;
   a.k_sf = fp4 ? scales->k_block_sf : nullptr;
+  a.v_sf = pv4 ? scales->v_block_sf : nullptr;
+  a.pv_fp4 = pv4;
   a.q_scale = scales->q_scale;
   a.k_scale = scales->k_scale;
   a.v_scale = scales->v_scale;
@@ -198,6 +220,22 @@ fpattn_status fpattn_quantize_fp8_video(const fpattn_tensor* x, const fpattn_vid
                                         fpattn_stream_t stream) {
   if (!layout) return FPATTN_ERR_INVALID_ARG;
   return quantize_fp8(x, layout, granularity, codes, scales, nonfinite_flag, stream);
+}
+
+size_t fpattn_nvfp4_v_bytes(int32_t B, int32_t H, int32_t N, int32_t d, size_t* block_sf_bytes) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || d % 64 != 0) {
+    if (block_sf_bytes) *block_sf_bytes = 0;
+    return 0;
+  }
+  const size_t nkb = static_cast<size_t>((N + 127) / 128);
+  if (block_sf_bytes) *block_sf_bytes = static_cast<size_t>(B) * H * nkb * 1024;
+  return static_cast<size_t>(B) * H * d * nkb * 64;
+}
+
+fpattn_status fpattn_quantize_nvfp4_v(const fpattn_tensor* x, const fpattn_video_layout* layout,
+                                      const float* static_amax, uint8_t* codes, uint8_t* block_sf,
+                                      float* tensor_scale, int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  return quantize_nvfp4_v(x, layout, static_amax, codes, block_sf, tensor_scale, nonfinite_flag, stream);
 }
 
 fpattn_status fpattn_quantize_fp8_group(const fpattn_tensor* x, const fpattn_video_layout* layout,

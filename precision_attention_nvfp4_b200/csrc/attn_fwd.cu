@@ -59,6 +59,7 @@ constexpr int kThreads = 512;
 constexpr int kStages = 3;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
 
 // error codes recorded on a wait timeout (which wait gave up)
 enum : int {
@@ -67,16 +68,22 @@ enum : int {
   kErrAlpha = 0x305, kErrSFree = 0x306, kErrODone = 0x302, kErrDrain = 0x401
 };
 
-template <int D, bool FP4>
+// FP4: Q, K in NVFP4 (else E4M3). PV4: P and V in NVFP4 and P V on the
+// block-scaled FP4 tensor cores (else E4M3 P and V).
+template <int D, bool FP4, bool PV4>
 struct Cfg {
   static constexpr int kQKRow = FP4 ? D / 2 : D;          // bytes per Q/K row
   static constexpr int kQKTile = 128 * kQKRow;            // bytes per 128-row Q/K tile
-  static constexpr int kVTile = 128 * D;                  // bytes per 128-row V tile
+  // V tile of one 128-key block: E4M3 [128 keys][D], or NVFP4 transposed
+  // [D channels][64 bytes = 128 keys]
+  static constexpr int kVTile = PV4 ? D * 64 : 128 * D;
   static constexpr int kSF = FP4 ? 512 * (D / 64) : 0;    // block-scale bytes per 128 rows
+  static constexpr int kSFV = PV4 ? 1024 : 0;             // V block scales per key block (2 k-steps)
+  static constexpr int kSFP = PV4 ? 1024 : 0;             // P block scales per P buffer
   static constexpr uint32_t kQKSwz = kQKRow == 128 ? 2u : (kQKRow == 64 ? 4u : 6u);
   static constexpr uint32_t kQKSbo = 8 * kQKRow;
-  static constexpr uint32_t kVSwz = D == 128 ? 2u : 4u;
-  static constexpr uint32_t kVSbo = 8 * D;
+  static constexpr uint32_t kVSwz = PV4 ? 4u : (D == 128 ? 2u : 4u);
+  static constexpr uint32_t kVSbo = PV4 ? 8 * 64 : 8 * D;
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
   // of the 16 exp2 pairs of a 32-score chunk, how many take the FMA-pipe
   // polynomial (measured best: 3 next to the cheaper FP4 QK^T, 4 with FP8)
@@ -89,16 +96,23 @@ struct Cfg {
   // the buffer without a barrier of its own.
   static constexpr int kPBufs = kStages;
   static constexpr uint32_t kColP = 384;
-  static constexpr uint32_t kColSFQ = kColP + 32 * kPBufs;
+  static constexpr uint32_t kPCols = PV4 ? 16 : 32;       // per P buffer: 128 keys of E2M1 or E4M3
+  static constexpr uint32_t kColSFQ = kColP + kPCols * kPBufs;
   static constexpr uint32_t kSFCols = 4 * (D / 64);
   static constexpr uint32_t kColSFK = kColSFQ + kSFCols;  // + buf * kSFCols
+  // P and V block scales of PV4, two buffers of 2 k-steps x 4 columns each
+  static constexpr uint32_t kColSFP = kColSFK + (FP4 ? 2 * kSFCols : 0);  // + (g & 1) * 8
+  static constexpr uint32_t kColSFV = kColSFP + 16;                       // + (g & 1) * 8
+  static_assert(!PV4 || kColSFV + 16 <= 512, "tensor memory columns");
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQKTile;
   static constexpr int kOffV = kOffK + kStages * kQKTile;
   static constexpr int kOffSFQ = kOffV + kStages * kVTile;
   static constexpr int kOffSFK = kOffSFQ + kSF;
-  static constexpr int kOffBar = kOffSFK + kStages * kSF;
+  static constexpr int kOffSFV = kOffSFK + kStages * kSF;   // [stage][1024]
+  static constexpr int kOffSFP = kOffSFV + kStages * kSFV;  // [P buffer][1024], written by the softmax
+  static constexpr int kOffBar = kOffSFP + kPBufs * kSFP;
   // mbarrier indices (one chain, so the pointers and the count cannot drift)
   static constexpr int kBarQFull = 0, kBarQEmpty = 1, kBarKFull = 2;
   static constexpr int kBarVFull = kBarKFull + kStages, kBarKVEmpty = kBarVFull + kStages;
@@ -128,6 +142,7 @@ struct __align__(64) Params {
   CUtensorMap tm_out;
   const uint8_t* q_sf;
   const uint8_t* k_sf;
+  const uint8_t* v_sf;  // NVFP4 V block scales [BH][nblk][1024] (PV4)
   const float* q_scale;
   const float* k_scale;
   const float* v_scale;
@@ -241,6 +256,64 @@ __device__ __forceinline__ float exp_pack32(const uint32_t (&r)[32], float c, fl
   return lo + hi;
 }
 
+// NVFP4 P for 32 scores: two 16-key blocks, each with an E4M3 block scale
+// taken from its largest P. This is the NVFP4 recipe with P's tensor amax fixed
+// at its bound: in units where P carries the factor 448 * 2^-tau, as nbias
+// gives it, sb = E4M3(P_max) and the codes are E2M1(6 P / dec(sb)). The
+// 6 / dec(sb) is folded into the block's exponent bias, so each exp2 lands on
+// the E2M1 grid directly. A block whose scale underflows to 0 keeps the plain
+// bias; its P are then far below the smallest E2M1 step and encode as 0.
+// Returns the sum of the unquantized P (in nbias units) for the row sum.
+// pk: key 8j + b in nibble b of pk[j]; sfw receives the two scale bytes at
+// byte positions shift and shift + 1.
+template <int kPoly>
+__device__ __forceinline__ float exp_pack32_fp4(const uint32_t (&r)[32], float c, float nbias, uint32_t (&pk)[4],
+                                                uint32_t& sfw, int shift) {
+  const uint64_t c2 = f2_pack(c, c);
+  float total = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t* rb = r + 16 * h;
+    const float bm =
+        fmax3(fmax3(fmax3(__uint_as_float(rb[0]), __uint_as_float(rb[1]), __uint_as_float(rb[2])),
+                    fmax3(__uint_as_float(rb[3]), __uint_as_float(rb[4]), __uint_as_float(rb[5])),
+                    fmax3(__uint_as_float(rb[6]), __uint_as_float(rb[7]), __uint_as_float(rb[8]))),
+              fmax3(__uint_as_float(rb[9]), __uint_as_float(rb[10]), __uint_as_float(rb[11])),
+              fmax3(fmax3(__uint_as_float(rb[12]), __uint_as_float(rb[13]), __uint_as_float(rb[14])),
+                    __uint_as_float(rb[15]), -INFINITY));
+    const uint32_t sb = cvt_e4m3x2(ex2_approx(fmaf(bm, c, nbias)), 0.f) & 0xFFu;
+    const float dec = e4m3_to_float(sb);
+    const float bias = sb ? nbias + (kLog2_6 - __log2f(dec)) : nbias;
+    const float back = sb ? dec * (1.f / 6.f) : 1.f;  // from the E2M1 grid back to P
+    const uint64_t nb2 = f2_pack(bias, bias);
+    uint64_t acc = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = 8 * h + i;  // pair of keys 2q, 2q + 1 of the chunk
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), c2, nb2);
+      uint64_t pr;
+      if (((q * kPoly) % 16) < kPoly) {
+        pr = exp2_poly2(x);
+      } else {
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        pr = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      }
+      acc = f2_add(acc, pr);
+      float p0, p1;
+      f2_unpack(pr, p0, p1);
+      const uint32_t byte = cvt_e2m1x2(p0, p1);
+      if ((q & 3) == 0) pk[q >> 2] = byte;
+      else pk[q >> 2] |= byte << (8 * (q & 3));
+    }
+    float lo, hi;
+    f2_unpack(acc, lo, hi);
+    total += (lo + hi) * back;
+    sfw |= sb << (8 * (shift + h));
+  }
+  return total;
+}
+
 // Every lane polls the barrier (one broadcast shared-memory access per poll),
 // so the warp never diverges around the wait.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
@@ -278,9 +351,9 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-template <int D, bool FP4>
+template <int D, bool FP4, bool PV4>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
-  using C = Cfg<D, FP4>;
+  using C = Cfg<D, FP4, PV4>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -385,8 +458,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           if (FP4)
             bulk_load(smem + C::kOffSFK + st * C::kSF,
                       p.k_sf + (static_cast<size_t>(bh) * p.nblk + kb) * C::kSF, C::kSF, k_full + st);
-          mbar_arrive_expect_tx(v_full + st, C::kVTile);
-          tma_load_3d(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, 0, kb * 128, bh);
+          mbar_arrive_expect_tx(v_full + st, C::kVTile + C::kSFV);
+          if (PV4) {
+            tma_load_3d(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, kb * 64, 0, bh);
+            bulk_load(smem + C::kOffSFV + st * C::kSFV, p.v_sf + (static_cast<size_t>(bh) * p.nblk + kb) * C::kSFV,
+                      C::kSFV, v_full + st);
+          } else {
+            tma_load_3d(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, 0, kb * 128, bh);
+          }
           *issued_cnt = g + 1;
         }
       }
@@ -394,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   } else if (warp == 1) {
     // ------------------------------------------------------------ PV issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescPV = idesc_e4m3(128, D, true);
+      constexpr uint32_t kIdescPV = PV4 ? idesc_nvf4(128, D) : idesc_e4m3(128, D, true);
       int g = 0;
       bool ok = true;
       for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
@@ -411,10 +490,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           tc_fence_after();
           const uint64_t v_desc =
               make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
+          if (PV4) {
+            // block scales of P (written by the softmax) and of V into tensor
+            // memory, then two K = 64 block-scaled MMAs with P from tensor memory
+            const uint32_t sb = (g & 1) * 8;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
-                          v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int a = 0; a < 2; ++a) {
+              tmem_cp_32x128_warpx4(tmem + C::kColSFP + sb + 4 * a,
+                                    make_smem_desc(smem_u32(smem + C::kOffSFP + pb * C::kSFP + 512 * a), 128, 128, 0));
+              tmem_cp_32x128_warpx4(tmem + C::kColSFV + sb + 4 * a,
+                                    make_smem_desc(smem_u32(smem + C::kOffSFV + st * C::kSFV + 512 * a), 128, 128, 0));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_nvf4_ts(tmem + C::kColO, tmem + C::kColP + pb * C::kPCols + 8 * kk, v_desc + 2 * kk, kIdescPV,
+                          tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk, (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
+                            v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(kv_empty + st);
           mma_commit(o_done + st);
           *consumed_cnt = g + 1;
@@ -568,12 +664,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // buffer g % kPBufs.
         const float nbias = p.p_log2_scale - m_use;
         const int pb = g % C::kPBufs;
-        const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32 + 16 * w;
-        uint32_t pk0[8], pk1[8];
-        float psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
-        tmem_st8(p_addr, pk0);
-        psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
-        tmem_st8(p_addr + 8, pk1);
+        float psum;
+        if (PV4) {
+          // NVFP4 P: this half's 64 keys are one K = 64 step of the P V
+          // product: 8 columns of E2M1 and 4 block scales, which go through
+          // shared memory (in the tensor-core scale layout) to the PV issuer.
+          const uint32_t p_addr = tmem + lane_off + C::kColP + pb * C::kPCols + 8 * w;
+          uint32_t pk0[4], pk1[4], sfw = 0u;
+          psum = exp_pack32_fp4<C::kPolyPairs>(r0, c, nbias, pk0, sfw, 0);
+          tmem_st4(p_addr, pk0);
+          psum += exp_pack32_fp4<C::kPolyPairs>(r1, c, nbias, pk1, sfw, 2);
+          tmem_st4(p_addr + 4, pk1);
+          reinterpret_cast<uint32_t*>(smem + C::kOffSFP + pb * C::kSFP + 512 * w)[(row & 31) * 4 + (row >> 5)] = sfw;
+          fence_proxy_async_shared();
+        } else {
+          const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32 + 16 * w;
+          uint32_t pk0[8], pk1[8];
+          psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
+          tmem_st8(p_addr, pk0);
+          psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
+          tmem_st8(p_addr + 8, pk1);
+        }
         l += psum;
         tmem_wait_st();
         tc_fence_before();
@@ -601,9 +712,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const KList L = key_list(p, qb);
       // this head's V scales, loaded now so their latency hides behind the
       // item's blocks (lane t holds channels t, t + 32, ...)
+      // (NVFP4 V: every channel takes 6 / s_t, the P scale's 1/2688 against
+      // the 1/448 the row sum is kept in)
       float vsv[D / 32];
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) vsv[i] = __ldg(p.v_scale + static_cast<size_t>(bh) * D + lane + 32 * i);
+      for (int i = 0; i < D / 32; ++i)
+        vsv[i] = PV4 ? __fdiv_rn(6.f, __ldg(p.v_scale)) : __ldg(p.v_scale + static_cast<size_t>(bh) * D + lane + 32 * i);
       for (int j = 0; j < L.count; ++j, ++g) {
         const int slot = g % kStages;
         if (!(ok = warp_wait(a_bar + q4 * kStages + slot, (g / kStages) & 1, abort_flag, &g_error_word, kErrAlpha)))
@@ -817,15 +931,31 @@ int sm_count() {
   return n;
 }
 
-template <int D, bool FP4>
+// NVFP4 V, transposed: bytes [BH][D][nkb * 64] with box [1][D][64] (one
+// 128-key block of every channel), 64-byte swizzle.
+bool make_map_vt(CUtensorMap* m, const void* base, int D, int nkb, int BH) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  const cuuint64_t pitch = static_cast<cuuint64_t>(nkb) * 64;
+  cuuint64_t dims[3] = {pitch, static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {pitch, pitch * static_cast<cuuint64_t>(D)};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(D), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool FP4, bool PV4>
 cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
-  using C = Cfg<D, FP4>;
+  using C = Cfg<D, FP4, PV4>;
   Params p;
   const int BH = a.B * a.H;
   const int qk_row = C::kQKRow;
+  const int nkb = (a.N + 127) / 128;
   if (!make_map(&p.tm_q, a.q, qk_row, a.N, BH, swizzle_for(qk_row)) ||
       !make_map(&p.tm_k, a.k, qk_row, a.N, BH, swizzle_for(qk_row)) ||
-      !make_map(&p.tm_v, a.v, D, a.N, BH, swizzle_for(D)))
+      !(PV4 ? make_map_vt(&p.tm_v, a.v, D, nkb, BH) : make_map(&p.tm_v, a.v, D, a.N, BH, swizzle_for(D))))
     return cudaErrorNotSupported;
   if (a.video) {
     if (!make_out_map_video(&p.tm_out, a.out, D, *a.video, BH)) return cudaErrorNotSupported;
@@ -836,6 +966,7 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   }
   p.q_sf = a.q_sf;
   p.k_sf = a.k_sf;
+  p.v_sf = a.v_sf;
   p.q_scale = a.q_scale;
   p.k_scale = a.k_scale;
   p.v_scale = a.v_scale;
@@ -855,21 +986,25 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   p.p_log2_scale = kLog2_448 - a.rescale_threshold;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, FP4, PV4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemRequest);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const int grid = p.num_items < sm_count() ? p.num_items : sm_count();
-  attn_fwd_kernel<D, FP4><<<grid, kThreads, C::kSmemRequest, st>>>(p);
+  attn_fwd_kernel<D, FP4, PV4><<<grid, kThreads, C::kSmemRequest, st>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {
-  if (a.d == 128) return a.qk_fp4 ? launch_t<128, true>(a, st) : launch_t<128, false>(a, st);
-  return a.qk_fp4 ? launch_t<64, true>(a, st) : launch_t<64, false>(a, st);
+  if (a.pv_fp4) {
+    if (a.d == 128) return a.qk_fp4 ? launch_t<128, true, true>(a, st) : launch_t<128, false, true>(a, st);
+    return a.qk_fp4 ? launch_t<64, true, true>(a, st) : launch_t<64, false, true>(a, st);
+  }
+  if (a.d == 128) return a.qk_fp4 ? launch_t<128, true, false>(a, st) : launch_t<128, false, false>(a, st);
+  return a.qk_fp4 ? launch_t<64, true, false>(a, st) : launch_t<64, false, false>(a, st);
 }
 
 cudaError_t read_device_error(cudaStream_t st, int clear, int* code) {

@@ -13,6 +13,11 @@ namespace fpattn {
 // read in raster order and the codes are written in tile-major order.
 cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                      int* nonfinite, const TokenMap* tmap, cudaStream_t st);
+// NVFP4 V with 16-token blocks along the sequence, transposed: codes
+// [BH][d][ceil(N/128)*64] bytes, scales [BH][ceil(N/128)][2][512].
+cudaError_t launch_quantize_nvfp4_tokens(const void* x, int BH, int N, int d, const float* static_amax,
+                                         uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
+                                         const TokenMap* tmap, cudaStream_t st);
 // One scale per group of `group` consecutive 128-token tiles (group 1: per tile).
 cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int group, uint8_t* codes,
                                       float* scales, int* nonfinite, const TokenMap* tmap, cudaStream_t st);
@@ -53,6 +58,7 @@ struct AttnArgs {
   const void* v;
   const uint8_t* q_sf;  // NVFP4 block scales (tensor-core layout) or null
   const uint8_t* k_sf;
+  const uint8_t* v_sf;  // NVFP4 V block scales [BH][nkb][2][512] (pv_fp4)
   const float* q_scale;
   const float* k_scale;
   const float* v_scale;
@@ -63,6 +69,7 @@ struct AttnArgs {
   const int32_t* row_order;
   int B, H, N, d;
   bool qk_fp4;
+  bool pv_fp4;  // P and V in NVFP4: v is transposed NVFP4 codes, v_scale its tensor scale
   bool causal;
   float softmax_scale;
   float rescale_threshold;  // tau in [0, 8], log2 units

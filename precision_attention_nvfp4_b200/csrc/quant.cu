@@ -342,6 +342,80 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __re
   sf[sf_word] = sfw;
 }
 
+// NVFP4 V for a block-scaled P V product: 16-token blocks along the sequence.
+// grid = (ceil(N/128), B*H), D threads. Thread t takes channels 2*(t % (D/2))
+// and +1 over tokens 64*(t / (D/2)) .. +63 of the key block: per channel four
+// 16-token blocks -> 32 code bytes of the transposed row and one 32-bit word
+// of block scales. Output, per (b, h): codes [D][nkb*64] (channel-major, two
+// tokens per byte, zero past N) and scales [nkb][2][512] in the tensor-core
+// scale layout with channels as rows. Same fp32 operation sequence as
+// nvfp4_quant_kernel, so the codes are bit-exact against the oracle.
+template <int D, bool kMap>
+__global__ void __launch_bounds__(D) nvfp4_tokens_quant_kernel(const uint32_t* __restrict__ x, int N, int nkb,
+                                                              const float* __restrict__ amax_ptr,
+                                                              uint8_t* __restrict__ codes,
+                                                              uint32_t* __restrict__ sf, TokenMap tmap) {
+  constexpr int kPairs = D / 2;
+  __shared__ int src_row[kMap ? 128 : 1];
+  const int kb = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int pair = threadIdx.x % kPairs;
+  const int half = threadIdx.x / kPairs;
+  if (kMap) {
+    for (int i = threadIdx.x; i < 128; i += D) src_row[i] = kb * 128 + i < N ? to_raster(tmap, kb * 128 + i) : 0;
+    __syncthreads();
+  }
+  const float s_t = nvfp4_tensor_scale(*amax_ptr);
+  const float six_st = __fmul_rn(6.f, s_t);
+  uint32_t cw[2][8];  // [channel of the pair][word]: 4 blocks x 8 codes each = 32 bytes per channel
+  uint32_t sfw[2] = {0u, 0u};
+#pragma unroll
+  for (int blk = 0; blk < 4; ++blk) {
+    float f[2][16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int tl = half * 64 + blk * 16 + k;  // token within the key block
+      const int n = kb * 128 + tl;
+      uint32_t w = 0u;
+      if (n < N) {
+        const size_t row = bh * N + (kMap ? src_row[tl] : n);
+        w = x[row * kPairs + pair];
+      }
+      f[0][k] = bf16_lo(w);
+      f[1][k] = bf16_hi(w);
+    }
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      float a = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) a = fmaxf(a, fabsf(f[ch][k]));
+      const uint32_t sb = cvt_e4m3x2(__fdiv_rn(a, six_st), 0.f) & 0xFFu;
+      const float den = __fmul_rn(e4m3_to_float(sb), s_t);
+      const float inv = __fdiv_rn(1.f, den);
+      const bool usable = (den != 0.f) && (fabsf(inv) <= FLT_MAX);
+      float y[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) y[k] = usable ? __fmul_rn(f[ch][k], inv) : 0.f;
+      cw[ch][2 * blk] = usable ? cvt_e2m1x8(y) : 0u;
+      cw[ch][2 * blk + 1] = usable ? cvt_e2m1x8(y + 8) : 0u;
+      sfw[ch] |= sb << (8 * blk);
+    }
+  }
+  const size_t pitch = static_cast<size_t>(nkb) * 64;
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int c = 2 * pair + ch;
+    uint4* dst = reinterpret_cast<uint4*>(codes + (bh * D + c) * pitch + kb * 64 + half * 32);
+    dst[0] = make_uint4(cw[ch][0], cw[ch][1], cw[ch][2], cw[ch][3]);
+    dst[1] = make_uint4(cw[ch][4], cw[ch][5], cw[ch][6], cw[ch][7]);
+    // channel c = 32 j + i, scale columns 4*half .. +3 of the key block:
+    // bytes 16 i + 4 j .. +3 of the block's 512-byte group `half`
+    uint32_t* group = sf + ((bh * nkb + kb) * 2 + half) * 128;
+    group[(c & 31) * 4 + (c >> 5)] = sfw[ch];
+    if (D == 64) group[(c & 31) * 4 + (c >> 5) + 2] = 0u;  // rows 64..127 of the layout are zero
+  }
+}
+
 __global__ void nvfp4_finalize_kernel(const float* __restrict__ amax_ptr, float* __restrict__ tensor_scale) {
   if (threadIdx.x == 0 && blockIdx.x == 0) *tensor_scale = nvfp4_tensor_scale(*amax_ptr);
 }
@@ -360,6 +434,36 @@ inline int num_sms() {
 
 // ---------------------------------------------------------------------------
 // Host launchers (arguments already validated by the C ABI layer).
+// ---------------------------------------------------------------------------
+cudaError_t launch_quantize_nvfp4_tokens(const void* x, int BH, int N, int d, const float* static_amax,
+                                         uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
+                                         const TokenMap* tmap, cudaStream_t st) {
+  const float* amax_ptr = static_amax;
+  if (!static_amax) {
+    cudaError_t e = cudaMemsetAsync(tensor_scale, 0, sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
+    tensor_amax_kernel<<<num_sms() * 8, kThreads, 0, st>>>(static_cast<const uint4*>(x), nchunks, tensor_scale,
+                                                           nonfinite);
+    amax_ptr = tensor_scale;
+  }
+  const int nkb = (N + 127) / 128;
+  dim3 grid(nkb, BH);
+  const uint32_t* xv = static_cast<const uint32_t*>(x);
+  uint32_t* sv = reinterpret_cast<uint32_t*>(block_sf);
+  const TokenMap tm = tmap ? *tmap : TokenMap{};
+  if (d == 128) {
+    if (tmap) nvfp4_tokens_quant_kernel<128, true><<<grid, 128, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
+    else nvfp4_tokens_quant_kernel<128, false><<<grid, 128, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
+  } else {
+    if (tmap) nvfp4_tokens_quant_kernel<64, true><<<grid, 64, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
+    else nvfp4_tokens_quant_kernel<64, false><<<grid, 64, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
+  }
+  nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax_ptr, tensor_scale);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
 cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                      int* nonfinite, const TokenMap* tmap, cudaStream_t st) {

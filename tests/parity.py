@@ -34,7 +34,7 @@ def f32(x: torch.Tensor) -> np.ndarray:
     return x.detach().float().cpu().numpy()
 
 
-def oracle_operands(q, k, v, qk_format, heads=None):
+def oracle_operands(q, k, v, qk_format, heads=None, pv_format="fp8"):
     """Quantize with the oracle and return dequantized fp64 operands
     [len(heads), N, d] for the (b*h) indices in ``heads`` (all by default).
     Only the selected heads are widened; the NVFP4 tensor scale still comes
@@ -55,16 +55,33 @@ def oracle_operands(q, k, v, qk_format, heads=None):
         ck, sk = quant.quantize_fp8_tile(kf)
         qh = quant.dequantize_fp8_tile(cq, sq)
         kh = quant.dequantize_fp8_tile(ck, sk)
-    cv, sv = quant.quantize_fp8_channel(vf)
-    vh = quant.dequantize_fp8_channel(cv, sv)
+    if pv_format == "nvfp4":
+        # the layout of quantize_nvfp4_tokens, with the tensor amax taken over
+        # every head (as the kernel does), not only the selected ones
+        av = float(v.abs().max().float())
+        cv, sbv, stv = quant.quantize_nvfp4(_pad_tokens_t(vf), static_amax=av)
+        vh = quant.dequantize_nvfp4_tokens(cv, sbv, stv, N)
+    else:
+        cv, sv = quant.quantize_fp8_channel(vf)
+        vh = quant.dequantize_fp8_channel(cv, sv)
     return qh, kh, vh
 
 
+def _pad_tokens_t(vf):
+    """[..., N, d] -> [..., d, Np] zero-padded to 128 tokens (the NVFP4 V layout)."""
+    N = vf.shape[-2]
+    Np = -(-N // 128) * 128
+    out = np.zeros(vf.shape[:-2] + (vf.shape[-1], Np), dtype=np.float32)
+    out[..., :N] = np.swapaxes(vf, -1, -2)
+    return out
+
+
 def compare_attention(out_gpu: np.ndarray, lse_gpu: np.ndarray, qh, kh, vh, rows, *, causal=False,
-                      key_blocks=None, softmax_scale=None, rescale_threshold=0.0):
+                      key_blocks=None, softmax_scale=None, rescale_threshold=0.0, p_format="e4m3"):
     """Oracle rows vs GPU rows for one (b,h). Returns a dict of errors."""
     ref, ref_lse = oatt.attention_rows(qh, kh, vh, rows, causal=causal, key_blocks=key_blocks,
-                                       softmax_scale=softmax_scale, rescale_threshold=rescale_threshold)
+                                       softmax_scale=softmax_scale, rescale_threshold=rescale_threshold,
+                                       p_format=p_format)
     got = out_gpu[rows].astype(np.float64)
     err = np.abs(got - ref)
     vmax = np.abs(vh).max()

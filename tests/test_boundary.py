@@ -242,3 +242,27 @@ def test_quantize_fp8_group_argument_errors(lib):
     ragged = _lib.VideoLayout(1, 8, 16, 1, 3, 16)
     assert lib.fpattn_quantize_fp8_group(ctypes.byref(x), ctypes.byref(ragged), 2, p16, p16, None,
                                          None) == _lib.ERR_UNSUPPORTED
+
+
+def test_nvfp4_v_sizes_and_argument_errors(lib):
+    sf = ctypes.c_size_t(0)
+    assert lib.fpattn_nvfp4_v_bytes(2, 3, 300, 128, ctypes.byref(sf)) == 2 * 3 * 128 * 3 * 64
+    assert sf.value == 2 * 3 * 3 * 1024
+    assert lib.fpattn_nvfp4_v_bytes(1, 1, 0, 64, ctypes.byref(sf)) == 0 and sf.value == 0
+    buf = (ctypes.c_uint8 * 4096)()
+    p16 = (ctypes.addressof(buf) + 15) & ~15
+    x = _t(p16, _lib.BF16)
+    assert lib.fpattn_quantize_nvfp4_v(ctypes.byref(x), None, None, None, p16, p16, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.fpattn_quantize_nvfp4_v(ctypes.byref(x), None, None, p16 + 8, p16, p16, None,
+                                       None) == _lib.ERR_ALIGNMENT
+    assert lib.fpattn_quantize_nvfp4_v(ctypes.byref(_t(p16, _lib.BF16, d=48)), None, None, p16, p16, p16, None,
+                                       None) == _lib.ERR_UNSUPPORTED
+    # an NVFP4 V needs its block scales
+    q = _t(p16, _lib.E4M3)
+    v4 = _t(p16, _lib.NVFP4)
+    sc = _lib.Scales(p16, p16, p16, None, None, 1.0 / 448.0, 0.0, 0.0, None)
+    assert lib.fpattn_fwd(ctypes.byref(q), ctypes.byref(q), ctypes.byref(v4), ctypes.byref(sc), None, 0, p16, None,
+                          None) == _lib.ERR_INVALID_ARG
+    sc_bad = _lib.Scales(p16, p16, p16, None, None, 1.0 / 448.0, 0.0, 0.0, p16 + 4)
+    assert lib.fpattn_fwd(ctypes.byref(q), ctypes.byref(q), ctypes.byref(v4), ctypes.byref(sc_bad), None, 0, p16,
+                          None, None) == _lib.ERR_ALIGNMENT
