@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4*
   for (int i = 0; i < 8; ++i) m[i] = 0.f;
   bool bad = false;
   const int rend = min(N, r0 + kRowsPerCta);
+#pragma unroll 4
   for (int r = r0 + rr; r < rend; r += kRowsPerIter) {
     const uint4 v = x[(bh * N + r) * kCpr + cg];
     float f[8];
@@ -257,12 +258,12 @@ __global__ void fp8_channel_finalize_kernel(float* __restrict__ s, int n) {
 // ---------------------------------------------------------------------------
 // NVFP4.
 // Pass 1 (dynamic only): tensor amax -> *amax_out via integer atomicMax.
-// Pass 2: one thread per (row, group of 64 elements = four 16-element blocks):
+// Pass 2 (nvfp4_quant_kernel), per 16-element block along d:
 //   s_t = A_t / 2688 (1 if A_t == 0)
 //   sb  = E4M3(A_b / (6 * s_t)), den = dec(sb) * s_t, inv = 1 / den,
 //   code = E2M1(x * inv)   (all zero when den == 0 or inv is not finite)
-//   32 code bytes + 4 scale bytes (one aligned 32-bit store into the
-//   tensor-core scale layout). Threads past N write the zero scale padding.
+//   codes in place of x's elements, scales in the tensor-core scale layout
+//   (zero for the rows that pad N up to 128).
 // Pass 3: *tensor_scale = s_t.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __restrict__ x, size_t nchunks,
@@ -287,59 +288,65 @@ __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
   return amax == 0.f ? 1.f : __fdiv_rn(amax, 2688.f);
 }
 
+// One warp per 128 consecutive 16-byte chunks (8 rows at D = 128, 16 at
+// D = 64): every load instruction covers 512 contiguous bytes. Lane i holds
+// chunks 32k + i; the two chunks of a 16-element block sit in adjacent
+// lanes, which combine their maxima with one shuffle and then take the same
+// scale decisions. Each lane writes the 4 code bytes of its chunk (a warp
+// store covers 128 contiguous bytes); even lanes write the block's scale byte.
+// grid = (nblk * 128 / kRowsPerCta, B*H): rows are padded to 128 per (b, h),
+// and the padding rows only write zero scales.
 template <int D, bool kMap>
 __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __restrict__ x, int N, int nblk,
                                                                const float* __restrict__ amax_ptr,
-                                                               uint4* __restrict__ codes,
-                                                               uint32_t* __restrict__ sf, size_t total_groups,
-                                                               TokenMap tmap) {
-  constexpr int kGroups = D / 64;  // 64-element groups per row
-  const size_t g = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x;
-  if (g >= total_groups) return;
-  // g enumerates (bh, padded row, group) with rows padded to 128 per (b, h).
-  const int grp = static_cast<int>(g % kGroups);
-  const size_t prow = g / kGroups;                // padded row over all (b, h)
-  const size_t rows_pad = static_cast<size_t>(nblk) * 128;
-  const size_t bh = prow / rows_pad;
-  const int r = static_cast<int>(prow % rows_pad);
-  // scale-layout offset (in 32-bit words): [bh][nb][grp] x 512 bytes, then
-  // byte 16*i + 4*j for row 32*j + i of the 128-row block.
-  const int nb = r >> 7, rr = r & 127;
-  const size_t sf_word = ((bh * nblk + nb) * kGroups + grp) * 128 + (rr & 31) * 4 + (rr >> 5);
-  if (r >= N) {
-    sf[sf_word] = 0u;
-    return;
+                                                               uint32_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ sf, TokenMap tmap) {
+  constexpr int kCpr = D / 8;                // 16-byte chunks per row
+  constexpr int kRowsPerWarp = 128 / kCpr;   // 8 or 16
+  constexpr int kGroups = D / 64;            // 512-byte scale groups per 128-row block
+  const int bh = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int r0 = (blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp;
+  int src = 0;
+  if (kMap && lane < kRowsPerWarp && r0 + lane < N) src = to_raster(tmap, r0 + lane);
+  uint4 v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = 32 * k + lane;
+    const int rl = c / kCpr;
+    const int srow = kMap ? __shfl_sync(0xffffffffu, src, rl) : r0 + rl;
+    v[k] = r0 + rl < N ? x[(static_cast<size_t>(bh) * N + srow) * kCpr + c % kCpr] : make_uint4(0u, 0u, 0u, 0u);
   }
   const float s_t = nvfp4_tensor_scale(*amax_ptr);
   const float six_st = __fmul_rn(6.f, s_t);
-  const size_t row = bh * N + r;
-  const size_t src_row = kMap ? bh * N + to_raster(tmap, r) : row;
-  const uint4* src = x + (src_row * D + grp * 64) / 8;
-  uint4* dst = codes + (row * D + grp * 64) / 32;
-  uint32_t sfw = 0;
-  uint32_t out[8];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {  // four 16-element blocks
-    float f[16];
-    unpack8(src[2 * b], f);
-    unpack8(src[2 * b + 1], f + 8);
+  for (int k = 0; k < 4; ++k) {
+    const int c = 32 * k + lane;
+    const int r = r0 + c / kCpr;
+    const int cc = c % kCpr;
+    float f[8];
+    unpack8(v[k], f);
     float a = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(f[i]));
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
     const uint32_t sb = cvt_e4m3x2(__fdiv_rn(a, six_st), 0.f) & 0xFFu;
     const float den = __fmul_rn(e4m3_to_float(sb), s_t);
     const float inv = __fdiv_rn(1.f, den);
     const bool usable = (den != 0.f) && (fabsf(inv) <= FLT_MAX);
-    float y[16];
+    float y[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = usable ? __fmul_rn(f[i], inv) : 0.f;
-    out[2 * b] = usable ? cvt_e2m1x8(y) : 0u;
-    out[2 * b + 1] = usable ? cvt_e2m1x8(y + 8) : 0u;
-    sfw |= sb << (8 * b);
+    for (int i = 0; i < 8; ++i) y[i] = usable ? __fmul_rn(f[i], inv) : 0.f;
+    if (r < N) codes[(static_cast<size_t>(bh) * N + r) * (D / 8) + cc] = usable ? cvt_e2m1x8(y) : 0u;
+    if ((lane & 1) == 0) {
+      // row r = 128 nb + 32 j + i, scale column col = 4 grp + s: byte
+      // 16 i + 4 j + s of the 512-byte group (bh, nb, grp)
+      const int col = cc >> 1, rr = r & 127;
+      const size_t byte = ((static_cast<size_t>(bh) * nblk + (r >> 7)) * kGroups + (col >> 2)) * 512 +
+                          16 * (rr & 31) + 4 * (rr >> 5) + (col & 3);
+      sf[byte] = r < N ? static_cast<uint8_t>(sb) : 0u;
+    }
   }
-  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-  sf[sf_word] = sfw;
 }
 
 // NVFP4 V for a block-scaled P V product: 16-token blocks along the sequence.
@@ -546,18 +553,18 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
     amax_ptr = tensor_scale;
   }
   const int nblk = (N + 127) / 128;
-  const size_t groups = static_cast<size_t>(BH) * nblk * 128 * (d / 64);
-  const unsigned blocks = static_cast<unsigned>((groups + kThreads - 1) / kThreads);
+  // rows per CTA: 8 warps x 128 chunks; 128 divides by it, so CTAs tile the padded rows
+  const int rows_per_cta = (kThreads / 32) * (128 / (d / 8));
+  dim3 grid(nblk * 128 / rows_per_cta, BH);
   const uint4* xv = static_cast<const uint4*>(x);
-  uint4* cv = reinterpret_cast<uint4*>(codes);
-  uint32_t* sv = reinterpret_cast<uint32_t*>(block_sf);
+  uint32_t* cv = reinterpret_cast<uint32_t*>(codes);
   const TokenMap tm = tmap ? *tmap : TokenMap{};
   if (d == 128) {
-    if (tmap) nvfp4_quant_kernel<128, true><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
-    else nvfp4_quant_kernel<128, false><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
+    if (tmap) nvfp4_quant_kernel<128, true><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
+    else nvfp4_quant_kernel<128, false><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
   } else {
-    if (tmap) nvfp4_quant_kernel<64, true><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
-    else nvfp4_quant_kernel<64, false><<<blocks, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, sv, groups, tm);
+    if (tmap) nvfp4_quant_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
+    else nvfp4_quant_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
   }
   nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax_ptr, tensor_scale);
   return cudaGetLastError();
