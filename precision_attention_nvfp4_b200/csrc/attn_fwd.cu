@@ -434,6 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
+      // K and V blocks are read by every query block of their head; Q once
+      const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
       int g = 0, it = 0;
       bool ok = true;
       for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
@@ -443,10 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (it > 0) ok = mbar_wait(q_empty, (it - 1) & 1, abort_flag, &g_error_word, kErrQEmpty);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, C::kQKTile + C::kSF);
-        tma_load_3d(smem + C::kOffQ, &p.tm_q, q_full, 0, qb * 128, bh);
+        tma_load_3d_hint(smem + C::kOffQ, &p.tm_q, q_full, 0, qb * 128, bh, stream);
         if (FP4)
-          bulk_load(smem + C::kOffSFQ, p.q_sf + (static_cast<size_t>(bh) * p.nblk + qb) * C::kSF, C::kSF,
-                    q_full);
+          bulk_load_hint(smem + C::kOffSFQ, p.q_sf + (static_cast<size_t>(bh) * p.nblk + qb) * C::kSF, C::kSF,
+                         q_full, stream);
         for (int j = 0; j < L.count; ++j, ++g) {
           const int st = g % kStages;
           const int use = g / kStages;
@@ -454,17 +456,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             break;
           const int kb = key_block(p, L, j);
           mbar_arrive_expect_tx(k_full + st, C::kQKTile + C::kSF);
-          tma_load_3d(smem + C::kOffK + st * C::kQKTile, &p.tm_k, k_full + st, 0, kb * 128, bh);
+          tma_load_3d_hint(smem + C::kOffK + st * C::kQKTile, &p.tm_k, k_full + st, 0, kb * 128, bh, keep);
           if (FP4)
-            bulk_load(smem + C::kOffSFK + st * C::kSF,
-                      p.k_sf + (static_cast<size_t>(bh) * p.nblk + kb) * C::kSF, C::kSF, k_full + st);
+            bulk_load_hint(smem + C::kOffSFK + st * C::kSF,
+                           p.k_sf + (static_cast<size_t>(bh) * p.nblk + kb) * C::kSF, C::kSF, k_full + st, keep);
           mbar_arrive_expect_tx(v_full + st, C::kVTile + C::kSFV);
           if (PV4) {
-            tma_load_3d(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, kb * 64, 0, bh);
-            bulk_load(smem + C::kOffSFV + st * C::kSFV, p.v_sf + (static_cast<size_t>(bh) * p.nblk + kb) * C::kSFV,
-                      C::kSFV, v_full + st);
+            tma_load_3d_hint(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, kb * 64, 0, bh, keep);
+            bulk_load_hint(smem + C::kOffSFV + st * C::kSFV,
+                           p.v_sf + (static_cast<size_t>(bh) * p.nblk + kb) * C::kSFV, C::kSFV, v_full + st, keep);
           } else {
-            tma_load_3d(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, 0, kb * 128, bh);
+            tma_load_3d_hint(smem + C::kOffV + st * C::kVTile, &p.tm_v, v_full + st, 0, kb * 128, bh, keep);
           }
           *issued_cnt = g + 1;
         }
@@ -820,8 +822,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
           for (int h = 0; h < D / 64; ++h) tma_store_5d(&p.tm_out, tile + h * 4096, h * 64, w0, h0, t0, bh);
         } else {
+          const uint64_t stream = l2_policy_evict_first();  // written once, read by no one here
 #pragma unroll
-          for (int h = 0; h < D / 64; ++h) tma_store_3d(&p.tm_out, tile + h * 4096, h * 64, qb * 128 + q4 * 32, bh);
+          for (int h = 0; h < D / 64; ++h)
+            tma_store_3d_hint(&p.tm_out, tile + h * 4096, h * 64, qb * 128 + q4 * 32, bh, stream);
         }
         bulk_commit();
       }
