@@ -430,6 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the prologue above touches no global memory; from here on the stream
+  // predecessor's results are read
+  griddep_wait();
   if (warp < 4) {
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
@@ -855,6 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -996,8 +1000,8 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
     configured = true;
   }
   const int grid = p.num_items < sm_count() ? p.num_items : sm_count();
-  attn_fwd_kernel<D, FP4, PV4><<<grid, kThreads, C::kSmemRequest, st>>>(p);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(attn_fwd_kernel<D, FP4, PV4>, dim3(grid), dim3(kThreads), C::kSmemRequest, st, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

@@ -106,6 +106,7 @@ template <int D, bool kMap, int kMode = kFused>
 __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restrict__ x, int N,
                                                             uint2* __restrict__ codes, float* __restrict__ scales,
                                                             int* nonfinite, TokenMap tmap) {
+  griddep_wait();
   constexpr int kChunksPerRow = D / 8;
   constexpr int kChunks = 128 * kChunksPerRow;  // 16-byte chunks per full tile
   constexpr int kPer = kChunks / kThreads;
@@ -148,6 +149,7 @@ __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restr
     const int c = threadIdx.x + i * kThreads;
     if (c / kChunksPerRow < rows) codes[base + c] = quant8_e4m3(v[i], s);
   }
+  griddep_launch_dependents();
 }
 
 // One thread per (b*h, group of `group` tiles): the group's amax is the max of
@@ -155,6 +157,7 @@ __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restr
 // tile of the group gets s = 448 / amax.
 __global__ void fp8_group_finalize_kernel(float* __restrict__ scales, int nblk, int group, int ngroups,
                                           int total) {
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total) return;
   float* sc = scales + static_cast<size_t>(i / ngroups) * nblk;
@@ -164,6 +167,7 @@ __global__ void fp8_group_finalize_kernel(float* __restrict__ scales, int nblk, 
   for (int b = b0; b < b1; ++b) a = fmaxf(a, sc[b]);
   const float s = fp8_scale_from_amax(a);
   for (int b = b0; b < b1; ++b) sc[b] = s;
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -178,6 +182,7 @@ constexpr int kRowsPerCta = 256;
 template <int D>
 __global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4* __restrict__ x, int N,
                                                                     float* __restrict__ amax, int* nonfinite) {
+  griddep_wait();
   constexpr int kCpr = D / 8;                 // chunks per row
   constexpr int kRowsPerIter = kThreads / kCpr;
   __shared__ float part[kRowsPerIter][D];
@@ -212,6 +217,7 @@ __global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4*
     for (int j = 0; j < kRowsPerIter; ++j) a = fmaxf(a, part[j][c]);
     atomicMax(reinterpret_cast<int*>(amax) + bh * D + c, __float_as_int(a));
   }
+  griddep_launch_dependents();
 }
 
 // The amax pass is order-free, so only the conversion pass reads through the
@@ -220,6 +226,7 @@ template <int D, bool kMap>
 __global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4* __restrict__ x, int N,
                                                                      const float* __restrict__ amax,
                                                                      uint2* __restrict__ codes, TokenMap tmap) {
+  griddep_wait();
   constexpr int kCpr = D / 8;
   constexpr int kRowsPerIter = kThreads / kCpr;
   static_assert(kRowsPerCta == kThreads, "one source-row lookup per thread");
@@ -248,11 +255,14 @@ __global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4
           (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[6], s[6]), __fmul_rn(f[7], s[7]))) << 16);
     codes[idx] = o;
   }
+  griddep_launch_dependents();
 }
 
 __global__ void fp8_channel_finalize_kernel(float* __restrict__ s, int n) {
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) s[i] = fp8_scale_from_amax(s[i]);
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -268,6 +278,7 @@ __global__ void fp8_channel_finalize_kernel(float* __restrict__ s, int n) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __restrict__ x, size_t nchunks,
                                                                float* __restrict__ amax_out, int* nonfinite) {
+  griddep_wait();
   __shared__ float red[kThreads / 32];
   float m = 0.f;
   bool bad = false;
@@ -282,6 +293,7 @@ __global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __re
   if (bad && nonfinite) atomicExch(nonfinite, 1);
   m = block_max(m, red);
   if (threadIdx.x == 0) atomicMax(reinterpret_cast<int*>(amax_out), __float_as_int(m));
+  griddep_launch_dependents();
 }
 
 __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
@@ -301,6 +313,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __re
                                                                const float* __restrict__ amax_ptr,
                                                                uint32_t* __restrict__ codes,
                                                                uint8_t* __restrict__ sf, TokenMap tmap) {
+  griddep_wait();
   constexpr int kCpr = D / 8;                // 16-byte chunks per row
   constexpr int kRowsPerWarp = 128 / kCpr;   // 8 or 16
   constexpr int kGroups = D / 64;            // 512-byte scale groups per 128-row block
@@ -347,6 +360,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __re
       sf[byte] = r < N ? static_cast<uint8_t>(sb) : 0u;
     }
   }
+  griddep_launch_dependents();
 }
 
 // NVFP4 V for a block-scaled P V product: 16-token blocks along the sequence.
@@ -362,6 +376,7 @@ __global__ void __launch_bounds__(D) nvfp4_tokens_quant_kernel(const uint32_t* _
                                                               const float* __restrict__ amax_ptr,
                                                               uint8_t* __restrict__ codes,
                                                               uint32_t* __restrict__ sf, TokenMap tmap) {
+  griddep_wait();
   constexpr int kPairs = D / 2;
   __shared__ int src_row[kMap ? 128 : 1];
   const int kb = blockIdx.x;
@@ -421,10 +436,21 @@ __global__ void __launch_bounds__(D) nvfp4_tokens_quant_kernel(const uint32_t* _
     group[(c & 31) * 4 + (c >> 5)] = sfw[ch];
     if (D == 64) group[(c & 31) * 4 + (c >> 5) + 2] = 0u;  // rows 64..127 of the layout are zero
   }
+  griddep_launch_dependents();
+}
+
+// Zeroes n floats (the amax accumulators), as a kernel so that it takes
+// part in the programmatic launch chain like every other step.
+__global__ void zero_kernel(float* __restrict__ p, int n) {
+  griddep_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0.f;
+  griddep_launch_dependents();
 }
 
 __global__ void nvfp4_finalize_kernel(const float* __restrict__ amax_ptr, float* __restrict__ tensor_scale) {
+  griddep_wait();
   if (threadIdx.x == 0 && blockIdx.x == 0) *tensor_scale = nvfp4_tensor_scale(*amax_ptr);
+  griddep_launch_dependents();
 }
 
 inline int num_sms() {
@@ -447,10 +473,10 @@ cudaError_t launch_quantize_nvfp4_tokens(const void* x, int BH, int N, int d, co
                                          const TokenMap* tmap, cudaStream_t st) {
   const float* amax_ptr = static_amax;
   if (!static_amax) {
-    cudaError_t e = cudaMemsetAsync(tensor_scale, 0, sizeof(float), st);
+    cudaError_t e = launch_pdl(zero_kernel, dim3(1), dim3(32), 0, st, tensor_scale, 1);
     if (e != cudaSuccess) return e;
     const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
-    tensor_amax_kernel<<<num_sms() * 8, kThreads, 0, st>>>(static_cast<const uint4*>(x), nchunks, tensor_scale,
+    launch_pdl(tensor_amax_kernel, dim3(num_sms() * 8), dim3(kThreads), 0, st, static_cast<const uint4*>(x), nchunks, tensor_scale,
                                                            nonfinite);
     amax_ptr = tensor_scale;
   }
@@ -460,13 +486,13 @@ cudaError_t launch_quantize_nvfp4_tokens(const void* x, int BH, int N, int d, co
   uint32_t* sv = reinterpret_cast<uint32_t*>(block_sf);
   const TokenMap tm = tmap ? *tmap : TokenMap{};
   if (d == 128) {
-    if (tmap) nvfp4_tokens_quant_kernel<128, true><<<grid, 128, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
-    else nvfp4_tokens_quant_kernel<128, false><<<grid, 128, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
+    if (tmap) launch_pdl(nvfp4_tokens_quant_kernel<128, true>, dim3(grid), dim3(128), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
+    else launch_pdl(nvfp4_tokens_quant_kernel<128, false>, dim3(grid), dim3(128), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
   } else {
-    if (tmap) nvfp4_tokens_quant_kernel<64, true><<<grid, 64, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
-    else nvfp4_tokens_quant_kernel<64, false><<<grid, 64, 0, st>>>(xv, N, nkb, amax_ptr, codes, sv, tm);
+    if (tmap) launch_pdl(nvfp4_tokens_quant_kernel<64, true>, dim3(grid), dim3(64), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
+    else launch_pdl(nvfp4_tokens_quant_kernel<64, false>, dim3(grid), dim3(64), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
   }
-  nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax_ptr, tensor_scale);
+  launch_pdl(nvfp4_finalize_kernel, dim3(1), dim3(32), 0, st, amax_ptr, tensor_scale);
   return cudaGetLastError();
 }
 
@@ -479,11 +505,11 @@ cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_
   uint2* cv = reinterpret_cast<uint2*>(codes);
   const TokenMap tm = tmap ? *tmap : TokenMap{};
   if (d == 128) {
-    if (tmap) fp8_tile_kernel<128, true><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
-    else fp8_tile_kernel<128, false><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+    if (tmap) launch_pdl(fp8_tile_kernel<128, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
+    else launch_pdl(fp8_tile_kernel<128, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
   } else {
-    if (tmap) fp8_tile_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
-    else fp8_tile_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+    if (tmap) launch_pdl(fp8_tile_kernel<64, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
+    else launch_pdl(fp8_tile_kernel<64, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
   }
   return cudaGetLastError();
 }
@@ -493,11 +519,11 @@ void launch_fp8_grouped(const uint4* xv, int BH, int N, int group, uint2* cv, fl
                         const TokenMap& tm, cudaStream_t st) {
   const int nblk = (N + 127) / 128;
   dim3 grid(nblk, BH);
-  fp8_tile_kernel<D, kMap, kAmaxOnly><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+  launch_pdl(fp8_tile_kernel<D, kMap, kAmaxOnly>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
   const int ngroups = (nblk + group - 1) / group;
   const int total = BH * ngroups;
-  fp8_group_finalize_kernel<<<(total + 255) / 256, 256, 0, st>>>(scales, nblk, group, ngroups, total);
-  fp8_tile_kernel<D, kMap, kConvert><<<grid, kThreads, 0, st>>>(xv, N, cv, scales, nonfinite, tm);
+  launch_pdl(fp8_group_finalize_kernel, dim3((total + 255) / 256), dim3(256), 0, st, scales, nblk, group, ngroups, total);
+  launch_pdl(fp8_tile_kernel<D, kMap, kConvert>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
 }
 
 cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int group, uint8_t* codes,
@@ -518,23 +544,23 @@ cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int g
 
 cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                         int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(scales, 0, sizeof(float) * BH * d, st);
+  cudaError_t e = launch_pdl(zero_kernel, dim3((BH * d + 255) / 256), dim3(256), 0, st, scales, BH * d);
   if (e != cudaSuccess) return e;
   dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, BH);
   const uint4* xv = static_cast<const uint4*>(x);
   uint2* cv = reinterpret_cast<uint2*>(codes);
   const TokenMap tm = tmap ? *tmap : TokenMap{};
   if (d == 128) {
-    fp8_channel_amax_kernel<128><<<grid, kThreads, 0, st>>>(xv, N, scales, nonfinite);
-    if (tmap) fp8_channel_quant_kernel<128, true><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
-    else fp8_channel_quant_kernel<128, false><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
+    launch_pdl(fp8_channel_amax_kernel<128>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, nonfinite);
+    if (tmap) launch_pdl(fp8_channel_quant_kernel<128, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
+    else launch_pdl(fp8_channel_quant_kernel<128, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
   } else {
-    fp8_channel_amax_kernel<64><<<grid, kThreads, 0, st>>>(xv, N, scales, nonfinite);
-    if (tmap) fp8_channel_quant_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
-    else fp8_channel_quant_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, scales, cv, tm);
+    launch_pdl(fp8_channel_amax_kernel<64>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, nonfinite);
+    if (tmap) launch_pdl(fp8_channel_quant_kernel<64, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
+    else launch_pdl(fp8_channel_quant_kernel<64, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
   }
   const int n = BH * d;
-  fp8_channel_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(scales, n);
+  launch_pdl(fp8_channel_finalize_kernel, dim3((n + 255) / 256), dim3(256), 0, st, scales, n);
   return cudaGetLastError();
 }
 
@@ -544,11 +570,11 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
   const float* amax_ptr = static_amax;
   if (!static_amax) {
     // tensor_scale doubles as the amax accumulator until pass 3 overwrites it.
-    cudaError_t e = cudaMemsetAsync(tensor_scale, 0, sizeof(float), st);
+    cudaError_t e = launch_pdl(zero_kernel, dim3(1), dim3(32), 0, st, tensor_scale, 1);
     if (e != cudaSuccess) return e;
     const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
     const int blocks = num_sms() * 8;
-    tensor_amax_kernel<<<blocks, kThreads, 0, st>>>(static_cast<const uint4*>(x), nchunks, tensor_scale,
+    launch_pdl(tensor_amax_kernel, dim3(blocks), dim3(kThreads), 0, st, static_cast<const uint4*>(x), nchunks, tensor_scale,
                                                     nonfinite);
     amax_ptr = tensor_scale;
   }
@@ -560,13 +586,13 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
   uint32_t* cv = reinterpret_cast<uint32_t*>(codes);
   const TokenMap tm = tmap ? *tmap : TokenMap{};
   if (d == 128) {
-    if (tmap) nvfp4_quant_kernel<128, true><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
-    else nvfp4_quant_kernel<128, false><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
+    if (tmap) launch_pdl(nvfp4_quant_kernel<128, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
+    else launch_pdl(nvfp4_quant_kernel<128, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
   } else {
-    if (tmap) nvfp4_quant_kernel<64, true><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
-    else nvfp4_quant_kernel<64, false><<<grid, kThreads, 0, st>>>(xv, N, nblk, amax_ptr, cv, block_sf, tm);
+    if (tmap) launch_pdl(nvfp4_quant_kernel<64, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
+    else launch_pdl(nvfp4_quant_kernel<64, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
   }
-  nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax_ptr, tensor_scale);
+  launch_pdl(nvfp4_finalize_kernel, dim3(1), dim3(32), 0, st, amax_ptr, tensor_scale);
   return cudaGetLastError();
 }
 
