@@ -509,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
               mma_nvf4_ts(tmem + C::kColO, tmem + C::kColP + pb * C::kPCols + 8 * kk, v_desc + 2 * kk, kIdescPV,
-                          tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk, (j > 0 || kk > 0) ? 1u : 0u);
+                          tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk,
+                          (j > 0 || kk > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -722,7 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       float vsv[D / 32];
 #pragma unroll
       for (int i = 0; i < D / 32; ++i)
-        vsv[i] = PV4 ? __fdiv_rn(6.f, __ldg(p.v_scale)) : __ldg(p.v_scale + static_cast<size_t>(bh) * D + lane + 32 * i);
+        vsv[i] = PV4 ? __fdiv_rn(6.f, __ldg(p.v_scale))
+                     : __ldg(p.v_scale + static_cast<size_t>(bh) * D + lane + 32 * i);
       for (int j = 0; j < L.count; ++j, ++g) {
         const int slot = g % kStages;
         if (!(ok = warp_wait(a_bar + q4 * kStages + slot, (g / kStages) & 1, abort_flag, &g_error_word, kErrAlpha)))

@@ -466,65 +466,64 @@ inline int num_sms() {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Host launchers (arguments already validated by the C ABI layer).
+// Host launchers (arguments already validated by the C ABI layer). Every
+// launch goes through launch_pdl; the instantiation is picked first.
 // ---------------------------------------------------------------------------
+namespace {
+
+// Zeroes the tensor-amax accumulator, then reduces |x| into it.
+void launch_tensor_amax(const void* x, int BH, int N, int d, float* acc, int* nonfinite, cudaStream_t st) {
+  launch_pdl(zero_kernel, dim3(1), dim3(32), 0, st, acc, 1);
+  const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
+  launch_pdl(tensor_amax_kernel, dim3(num_sms() * 8), dim3(kThreads), 0, st, static_cast<const uint4*>(x), nchunks,
+             acc, nonfinite);
+}
+
+}  // namespace
+
 cudaError_t launch_quantize_nvfp4_tokens(const void* x, int BH, int N, int d, const float* static_amax,
                                          uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
                                          const TokenMap* tmap, cudaStream_t st) {
   const float* amax_ptr = static_amax;
   if (!static_amax) {
-    cudaError_t e = launch_pdl(zero_kernel, dim3(1), dim3(32), 0, st, tensor_scale, 1);
-    if (e != cudaSuccess) return e;
-    const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
-    launch_pdl(tensor_amax_kernel, dim3(num_sms() * 8), dim3(kThreads), 0, st, static_cast<const uint4*>(x), nchunks, tensor_scale,
-                                                           nonfinite);
+    // tensor_scale doubles as the amax accumulator until the finalize overwrites it
+    launch_tensor_amax(x, BH, N, d, tensor_scale, nonfinite, st);
     amax_ptr = tensor_scale;
   }
   const int nkb = (N + 127) / 128;
-  dim3 grid(nkb, BH);
-  const uint32_t* xv = static_cast<const uint32_t*>(x);
-  uint32_t* sv = reinterpret_cast<uint32_t*>(block_sf);
-  const TokenMap tm = tmap ? *tmap : TokenMap{};
-  if (d == 128) {
-    if (tmap) launch_pdl(nvfp4_tokens_quant_kernel<128, true>, dim3(grid), dim3(128), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
-    else launch_pdl(nvfp4_tokens_quant_kernel<128, false>, dim3(grid), dim3(128), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
-  } else {
-    if (tmap) launch_pdl(nvfp4_tokens_quant_kernel<64, true>, dim3(grid), dim3(64), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
-    else launch_pdl(nvfp4_tokens_quant_kernel<64, false>, dim3(grid), dim3(64), 0, st, xv, N, nkb, amax_ptr, codes, sv, tm);
-  }
+  auto kern = d == 128 ? (tmap ? nvfp4_tokens_quant_kernel<128, true> : nvfp4_tokens_quant_kernel<128, false>)
+                       : (tmap ? nvfp4_tokens_quant_kernel<64, true> : nvfp4_tokens_quant_kernel<64, false>);
+  launch_pdl(kern, dim3(nkb, BH), dim3(d), 0, st, static_cast<const uint32_t*>(x), N, nkb, amax_ptr, codes,
+             reinterpret_cast<uint32_t*>(block_sf), tmap ? *tmap : TokenMap{});
   launch_pdl(nvfp4_finalize_kernel, dim3(1), dim3(32), 0, st, amax_ptr, tensor_scale);
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------------------
-// ---------------------------------------------------------------------------
 cudaError_t launch_quantize_fp8_tile(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                      int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
-  dim3 grid((N + 127) / 128, BH);
-  const uint4* xv = static_cast<const uint4*>(x);
-  uint2* cv = reinterpret_cast<uint2*>(codes);
-  const TokenMap tm = tmap ? *tmap : TokenMap{};
-  if (d == 128) {
-    if (tmap) launch_pdl(fp8_tile_kernel<128, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
-    else launch_pdl(fp8_tile_kernel<128, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
-  } else {
-    if (tmap) launch_pdl(fp8_tile_kernel<64, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
-    else launch_pdl(fp8_tile_kernel<64, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
-  }
+  auto kern = d == 128 ? (tmap ? fp8_tile_kernel<128, true> : fp8_tile_kernel<128, false>)
+                       : (tmap ? fp8_tile_kernel<64, true> : fp8_tile_kernel<64, false>);
+  launch_pdl(kern, dim3((N + 127) / 128, BH), dim3(kThreads), 0, st, static_cast<const uint4*>(x), N,
+             reinterpret_cast<uint2*>(codes), scales, nonfinite, tmap ? *tmap : TokenMap{});
   return cudaGetLastError();
 }
+
+namespace {
 
 template <int D, bool kMap>
 void launch_fp8_grouped(const uint4* xv, int BH, int N, int group, uint2* cv, float* scales, int* nonfinite,
                         const TokenMap& tm, cudaStream_t st) {
   const int nblk = (N + 127) / 128;
-  dim3 grid(nblk, BH);
-  launch_pdl(fp8_tile_kernel<D, kMap, kAmaxOnly>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
+  const dim3 grid(nblk, BH);
+  launch_pdl(fp8_tile_kernel<D, kMap, kAmaxOnly>, grid, dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
   const int ngroups = (nblk + group - 1) / group;
   const int total = BH * ngroups;
-  launch_pdl(fp8_group_finalize_kernel, dim3((total + 255) / 256), dim3(256), 0, st, scales, nblk, group, ngroups, total);
-  launch_pdl(fp8_tile_kernel<D, kMap, kConvert>, dim3(grid), dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
+  launch_pdl(fp8_group_finalize_kernel, dim3((total + 255) / 256), dim3(256), 0, st, scales, nblk, group, ngroups,
+             total);
+  launch_pdl(fp8_tile_kernel<D, kMap, kConvert>, grid, dim3(kThreads), 0, st, xv, N, cv, scales, nonfinite, tm);
 }
+
+}  // namespace
 
 cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int group, uint8_t* codes,
                                       float* scales, int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
@@ -544,22 +543,16 @@ cudaError_t launch_quantize_fp8_group(const void* x, int BH, int N, int d, int g
 
 cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uint8_t* codes, float* scales,
                                         int* nonfinite, const TokenMap* tmap, cudaStream_t st) {
-  cudaError_t e = launch_pdl(zero_kernel, dim3((BH * d + 255) / 256), dim3(256), 0, st, scales, BH * d);
-  if (e != cudaSuccess) return e;
-  dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, BH);
-  const uint4* xv = static_cast<const uint4*>(x);
-  uint2* cv = reinterpret_cast<uint2*>(codes);
-  const TokenMap tm = tmap ? *tmap : TokenMap{};
-  if (d == 128) {
-    launch_pdl(fp8_channel_amax_kernel<128>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, nonfinite);
-    if (tmap) launch_pdl(fp8_channel_quant_kernel<128, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
-    else launch_pdl(fp8_channel_quant_kernel<128, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
-  } else {
-    launch_pdl(fp8_channel_amax_kernel<64>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, nonfinite);
-    if (tmap) launch_pdl(fp8_channel_quant_kernel<64, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
-    else launch_pdl(fp8_channel_quant_kernel<64, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, scales, cv, tm);
-  }
   const int n = BH * d;
+  launch_pdl(zero_kernel, dim3((n + 255) / 256), dim3(256), 0, st, scales, n);
+  const dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, BH);
+  const uint4* xv = static_cast<const uint4*>(x);
+  auto amax = d == 128 ? fp8_channel_amax_kernel<128> : fp8_channel_amax_kernel<64>;
+  auto quant = d == 128 ? (tmap ? fp8_channel_quant_kernel<128, true> : fp8_channel_quant_kernel<128, false>)
+                        : (tmap ? fp8_channel_quant_kernel<64, true> : fp8_channel_quant_kernel<64, false>);
+  launch_pdl(amax, grid, dim3(kThreads), 0, st, xv, N, scales, nonfinite);
+  launch_pdl(quant, grid, dim3(kThreads), 0, st, xv, N, static_cast<const float*>(scales),
+             reinterpret_cast<uint2*>(codes), tmap ? *tmap : TokenMap{});
   launch_pdl(fp8_channel_finalize_kernel, dim3((n + 255) / 256), dim3(256), 0, st, scales, n);
   return cudaGetLastError();
 }
@@ -569,29 +562,17 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
                                   const TokenMap* tmap, cudaStream_t st) {
   const float* amax_ptr = static_amax;
   if (!static_amax) {
-    // tensor_scale doubles as the amax accumulator until pass 3 overwrites it.
-    cudaError_t e = launch_pdl(zero_kernel, dim3(1), dim3(32), 0, st, tensor_scale, 1);
-    if (e != cudaSuccess) return e;
-    const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
-    const int blocks = num_sms() * 8;
-    launch_pdl(tensor_amax_kernel, dim3(blocks), dim3(kThreads), 0, st, static_cast<const uint4*>(x), nchunks, tensor_scale,
-                                                    nonfinite);
+    // tensor_scale doubles as the amax accumulator until the finalize overwrites it
+    launch_tensor_amax(x, BH, N, d, tensor_scale, nonfinite, st);
     amax_ptr = tensor_scale;
   }
   const int nblk = (N + 127) / 128;
   // rows per CTA: 8 warps x 128 chunks; 128 divides by it, so CTAs tile the padded rows
   const int rows_per_cta = (kThreads / 32) * (128 / (d / 8));
-  dim3 grid(nblk * 128 / rows_per_cta, BH);
-  const uint4* xv = static_cast<const uint4*>(x);
-  uint32_t* cv = reinterpret_cast<uint32_t*>(codes);
-  const TokenMap tm = tmap ? *tmap : TokenMap{};
-  if (d == 128) {
-    if (tmap) launch_pdl(nvfp4_quant_kernel<128, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
-    else launch_pdl(nvfp4_quant_kernel<128, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
-  } else {
-    if (tmap) launch_pdl(nvfp4_quant_kernel<64, true>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
-    else launch_pdl(nvfp4_quant_kernel<64, false>, dim3(grid), dim3(kThreads), 0, st, xv, N, nblk, amax_ptr, cv, block_sf, tm);
-  }
+  auto kern = d == 128 ? (tmap ? nvfp4_quant_kernel<128, true> : nvfp4_quant_kernel<128, false>)
+                       : (tmap ? nvfp4_quant_kernel<64, true> : nvfp4_quant_kernel<64, false>);
+  launch_pdl(kern, dim3(nblk * 128 / rows_per_cta, BH), dim3(kThreads), 0, st, static_cast<const uint4*>(x), N,
+             nblk, amax_ptr, reinterpret_cast<uint32_t*>(codes), block_sf, tmap ? *tmap : TokenMap{});
   launch_pdl(nvfp4_finalize_kernel, dim3(1), dim3(32), 0, st, amax_ptr, tensor_scale);
   return cudaGetLastError();
 }
