@@ -480,9 +480,9 @@ def main():
                          f"{sorted(set(h for h, _ in done))} x query blocks {qblocks} in that order (fp64 "
                          f"numpy oracle, its quantization of those heads included), {s:.1f} s"}
 
-    # Q/K: NVFP4 amax + quantize + finalize each, or one FP8 kernel each; V: three kernels
-    # (FP8 channel or NVFP4); attention: one
-    launches_per_step = (6 if w.qk_format == "nvfp4" else 2) + 3 + 1
+    # Our kernels per step. Q/K: NVFP4 zero + amax + quantize + finalize each, or one FP8 kernel
+    # each. V: zero + amax + quantize + finalize (FP8 per channel or NVFP4). Attention: one.
+    launches_per_step = (8 if w.qk_format == "nvfp4" else 2) + 4 + 1
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
