@@ -7,16 +7,21 @@
 //   P:    E4M3 at the fixed scale 1/448 (FPSAttention page, section 3.1);
 //   V:    E4M3 with per-channel scales; PV on kind::f8f6f4 with P read
 //         straight from tensor memory.
+// The PV4 variants quantize P to NVFP4 in the softmax (16-key blocks, the
+// tensor amax of P fixed at its bound) and take V in NVFP4 along the
+// sequence; PV then runs on kind::mxf4nvf4 with P from tensor memory.
 // The online softmax follows the FlashAttention tiling the pages describe
 // (FlashAttention-4 article: S and P kept on chip, O accumulated in tensor
-// memory, asynchronous pipeline between loads, MMA and softmax). The running
-// row max is always the exact max of the keys seen so far; O and the row sum
-// are rescaled only for rows whose max moved (a warp skips the tensor-memory
-// round trip when none of its rows moved), which is exact.
+// memory, asynchronous pipeline between loads, MMA and softmax). By default
+// the reference row max is the exact max of the keys seen so far; O and the
+// row sum are rescaled only for rows whose max moved (a warp skips the
+// tensor-memory round trip when none of its rows moved), which is exact. A
+// threshold tau > 0 moves it only when the max grew by more than tau, with P
+// stored at 448 * 2^-tau.
 //
 // CTA organisation (persistent, one CTA per SM, 512 threads):
 //   warp 0        TMA producer: Q once per work item, K/V tiles into a
-//                 4-stage shared-memory ring (plus NVFP4 block scales)
+//                 3-stage shared-memory ring (plus block scales)
 //   warp 1        tensor-memory allocator; issues O += P V (one thread)
 //   warp 2        issues S = Q K^T (one thread)
 //   warp 3        idle
@@ -32,10 +37,16 @@
 // sum of its half; the epilogue adds the two.
 // Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32
 // 128x128, buffer = block parity), O at column 256 (d fp32 columns), a ring
-// of three P buffers (E4M3, 32 columns each) at 384, NVFP4 scale vectors of Q
-// and of two K tiles at 480. S and P having their own buffers lets the S of a block be
-// issued as soon as its buffer's previous tile has been read, independently
-// of the PV of that tile; the two MMA kinds are issued by separate threads.
+// of three P buffers (E4M3: 32 columns each; NVFP4: 16) at 384, then the
+// NVFP4 scale vectors (Q, two K tiles; with PV4 also two each of P and V).
+// S and P having their own buffers lets the S of a block be issued as soon as
+// its buffer's previous tile has been read, independently of the PV of that
+// tile; the two MMA kinds are issued by separate threads.
+// The epilogue stores bf16 rows with TMA tensor stores: 3-D over [BH][N][d],
+// or 5-D over a video's raster grid when the tokens are in tile-major order.
+// K and V are loaded with an L2 evict-last policy, Q and the output with
+// evict-first. The kernel waits for its stream predecessor (programmatic
+// dependent launch) only after its prologue.
 // Work items are (batch*head, 128-query block); causal runs schedule the
 // longest query blocks first, tile-mask runs follow the mask's row order.
 #include <cfloat>

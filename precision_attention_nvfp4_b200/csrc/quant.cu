@@ -11,6 +11,12 @@
 // and write codes and scales in tile-major order, so the permutation costs no
 // pass of its own (FPSAttention page, section 3.3, item 1).
 //
+// Also here: NVFP4 V with its blocks along the sequence (for the all-NVFP4
+// P V product), and FP8 Q/K with one scale per group of tiles (the coarser
+// granularities of the denoising-step schedule, FPSAttention page, section
+// 3.2). Every kernel takes part in the programmatic launch chain (see
+// griddep_wait).
+//
 // All kernels are bandwidth-bound streams: 16-byte loads per thread,
 // consecutive threads on consecutive 16-byte chunks, warp-shuffle reductions.
 // Every scale step is one correctly rounded fp32 operation (__fdiv_rn,

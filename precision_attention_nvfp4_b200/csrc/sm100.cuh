@@ -1,6 +1,7 @@
 // Thin inline-PTX wrappers for the Blackwell (sm_100a) features the kernels
-// use: mbarriers, TMA bulk-tensor loads, tensor memory (TMEM) and the
-// fifth-generation tensor-core MMA (tcgen05), plus FP8/FP4 conversions.
+// use: mbarriers, TMA bulk-tensor loads and stores (with L2 cache policies),
+// tensor memory (TMEM) and the fifth-generation tensor-core MMA (tcgen05),
+// FP8/FP4 conversions, and programmatic dependent launch.
 //
 // Every wait on an mbarrier is bounded: after kWaitTimeoutNs of polling the
 // wait records an error code in the library's device error word, raises the
