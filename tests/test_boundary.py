@@ -123,6 +123,9 @@ def test_sta_planner_matches_oracle(lib, grid, tile, window):
     lens = np.diff(plan.row_ptr)
     assert sorted(plan.row_order.tolist()) == list(range(plan.nblk))
     assert np.all(np.diff(lens[plan.row_order]) <= 0)
+    # rows of equal length keep their index order (a stable longest-first sort)
+    order = plan.row_order.tolist()
+    assert order == sorted(range(plan.nblk), key=lambda r: (-lens[r], r))
 
 
 def test_sta_planner_rejects_unaligned_tiles(lib):
