@@ -28,7 +28,6 @@ from __future__ import annotations
 
 import ctypes
 import dataclasses
-import math
 from typing import Optional, Sequence, Tuple
 
 import numpy as np

@@ -11,13 +11,12 @@ sum near 1e-5 and the fp32 scores carry about 1e-6 relative error, so
 from __future__ import annotations
 
 import functools
-import math
 
 import numpy as np
 import torch
 
 from oracle import attention as oatt
-from oracle import codec, quant
+from oracle import quant
 
 ATOL_FRAC = 2e-2
 REL_L2 = 5e-3

@@ -8,7 +8,6 @@ a ragged tail; full-size workloads are checked on sampled query blocks (first,
 last, middle, causal diagonal, STA edge tiles) in the launch configuration the
 benchmark uses.
 """
-import math
 
 import numpy as np
 import pytest

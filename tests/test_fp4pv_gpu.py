@@ -14,7 +14,6 @@ import pytest
 import torch
 
 import precision_attention_nvfp4_b200 as fp
-import workloads
 from oracle import codec, quant, sta
 import parity
 

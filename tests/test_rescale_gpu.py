@@ -11,7 +11,6 @@ import pytest
 import torch
 
 import precision_attention_nvfp4_b200 as fp
-import workloads
 import parity
 
 pytestmark = pytest.mark.gpu
