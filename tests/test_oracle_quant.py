@@ -4,8 +4,12 @@ Checks: hand-worked examples, exactly representable inputs surviving, the
 amax element mapping to the format maximum, zero blocks, the error bound of
 half a grid step, quantize(dequantize(quantize(x))) == quantize(x), the FP8
 element conversion against torch's float8 cast, and the swizzled scale layout
-against a direct restatement of its byte formula.
+against byte positions worked by hand from NVIDIA's published tensor-core
+scale-factor layout (tests/golden/nvfp4_sf_layout.json).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -13,6 +17,9 @@ import torch
 from oracle import codec, quant
 
 F32 = np.float32
+
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 def _bf16(x):
@@ -93,21 +100,40 @@ def test_nvfp4_roundtrip_idempotent():
     assert np.array_equal(codec.e2m1_decode(c1), codec.e2m1_decode(c2))
 
 
-def test_nvfp4_sf_swizzle_formula():
-    rng = np.random.default_rng(6)
+def test_nvfp4_sf_swizzle_golden_positions():
+    """The scale layout against byte positions worked by hand from NVIDIA's
+    published tensor-core scale-factor layout (tests/golden/nvfp4_sf_layout.json):
+    a single marked scale must land at exactly that byte, nowhere else."""
+    gold = json.load(open(os.path.join(GOLDEN, "nvfp4_sf_layout.json")))
+    for case in gold["cases"]:
+        N, d = case["N"], case["d"]
+        sf = np.zeros((1, N, d // 16), dtype=np.uint8)
+        sf[0, case["row"], case["col"]] = 0xAB
+        sw = quant.nvfp4_sf_swizzle(sf, N, d).reshape(-1)
+        assert sw.size == -(-N // 128) * (d // 64) * 512
+        hit = np.flatnonzero(sw)
+        assert hit.tolist() == [case["byte"]], (case, hit)
+
+
+def test_nvfp4_sf_swizzle_is_a_bijection_with_zero_padding():
+    """Every (row, column) scale of a ragged tensor lands at its own byte,
+    and the bytes of the rows past N that pad the last 128-row block are 0."""
     N, d = 200, 128
-    sf = rng.integers(0, 256, (3, N, d // 16)).astype(np.uint8)
-    sw = quant.nvfp4_sf_swizzle(sf, N, d).reshape(3, -1)
-    for r in (0, 1, 31, 32, 95, 127, 128, 199):
-        for col in range(d // 16):
-            off = ((r // 128) * (d // 64) + col // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + col % 4
-            assert np.array_equal(sw[:, off], sf[:, r, col])
-    # padding rows are zero
-    assert np.all(quant.nvfp4_sf_swizzle(sf, N, d)[:, 1].reshape(3, -1).sum() >= 0)
-    pad_rows = [r for r in range(N, 256)]
-    for r in pad_rows[:5]:
-        off = (1 * (d // 64)) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32)
-        assert np.all(sw[:, off:off + 4] == 0)
+    ncol = d // 16
+    seen = np.zeros((-(-N // 128)) * (d // 64) * 512, dtype=np.int64)
+    for col in range(ncol):  # one column at a time: a uint8 cannot label every scale
+        sf = np.zeros((1, N, ncol), dtype=np.uint8)
+        sf[0, :, col] = 1
+        seen += quant.nvfp4_sf_swizzle(sf, N, d).reshape(-1)
+    assert seen.max() == 1 and seen.sum() == N * ncol
+    rng = np.random.default_rng(6)
+    sf = rng.integers(1, 256, (3, N, ncol)).astype(np.uint8)
+    sw = quant.nvfp4_sf_swizzle(sf, N, d)
+    assert np.count_nonzero(sw) == np.count_nonzero(sf)
+    # the 56 padding rows of the second block (200..255) hold no scale
+    pad = np.zeros_like(seen, dtype=bool)
+    pad[np.flatnonzero(seen == 0)] = True
+    assert np.all(sw.reshape(3, -1)[:, pad] == 0) and pad.sum() == (256 - N) * ncol
 
 
 def test_fp8_tile_amax_maps_to_448_and_matches_torch_cast():
