@@ -1,15 +1,19 @@
 """Benchmark of the quantized attention hot path on B200.
 
 One step = the whole path on one batch of synthetic input already resident
-in HBM: NVFP4 quantization of Q and K, per-channel FP8 quantization of V, and
-the fused attention forward (LLM prefill workload: B=4, H=32, N=4096, d=128,
-causal; QK^T in NVFP4, PV in FP8). W untimed warm-up steps, then exactly K
-timed steps bracketed by a barrier and a device synchronize, timed with CUDA
-events on the launching stream; multi-GPU runs take the max over ranks. Rank 0
-prints one JSON line.
+in HBM: quantization of Q and K (NVFP4, or FP8 per 128-token tile), per-channel
+FP8 quantization of V, and the fused attention forward. The default workload
+is the sequence sweep's longest single-GPU point: B=1, H=32, N=131072, d=128,
+dense, x20 outlier channels, QK^T in NVFP4 and PV in FP8 (2.8e14 flops a
+step). W untimed warm-up steps, then exactly K timed steps bracketed by a
+barrier and a device synchronize, timed with CUDA events on the launching
+stream; multi-GPU runs take the max over ranks. Rank 0 prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
   python bench.py --sweep     # sequence-length sweep, one JSON line per configuration
+
+Workloads: long_seq_128k_nvfp4 (default), long_seq_128k_fp8, llm_prefill_causal,
+video_dense_fp8, video_sta_fp8, tiny_nvfp4.
 
 ``--impl reference`` times the CPU oracle (the only other implementation of
 this path) on a bounded sample of the same workload, on the host cores.
@@ -48,26 +52,31 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def profiled_traffic():
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, or None when the kernel sources changed since that capture."""
+def kernel_source_hash() -> str:
+    """First 16 hex digits of sha256(attn_fwd.cu + sm100.cuh): ties a DRAM
+    traffic record to the kernel source it was captured on."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
-    if not os.path.exists(path):
-        return None
-    kv = {}
-    with open(path) as f:
-        for line in f:
-            if ":" in line and not line.startswith("#"):
-                a, b = line.split(":", 1)
-                kv[a.strip()] = b.strip()
     h = hashlib.sha256()
     for src in ("attn_fwd.cu", "sm100.cuh"):
         with open(os.path.join(ROOT, "precision_attention_nvfp4_b200", "csrc", src), "rb") as f:
             h.update(f.read())
-    if h.hexdigest()[:16] != kv.get("source_sha256_16"):
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """Per-launch DRAM bytes (read + write) of the attention kernel on this
+    workload from the committed ncu record, or None when there is none or the
+    kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+    if not os.path.exists(path):
         return None
-    return float(kv["traffic_bytes"])
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == workload and parts[1] == want:
+                return float(parts[2])
+    return None
 
 
 def executed_block_pairs(w: workloads.Workload) -> int:
@@ -95,7 +104,9 @@ def quant_bytes(w: workloads.Workload, pv_format: str = "fp8") -> float:
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+    """Samples nvidia-smi clocks and throttle reasons (every 100 ms, with a
+    host timestamp per sample) from before the warm-up to the end of the
+    timed region; stop() summarises the samples inside the timed window."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -104,7 +115,7 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (host time, csv line)
 
     def start(self):
         try:
@@ -119,39 +130,62 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.time(), line.strip()))
 
-    def stop(self):
+    def stop(self, t0: float, t1: float):
+        """Summary of the samples taken between host times t0 and t1 (the
+        timed region); when that window holds none (a region shorter than the
+        sampling period), of all samples since start()."""
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)  # let the sample that straddles t1 arrive
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
+        inside = [ln for t, ln in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if not inside:
+            inside = [ln for _, ln in self.samples]
+            window = "warm-up and timed region (timed region shorter than the 100 ms sampling period)"
+        sm, mx, power, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in inside:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
             try:
                 sm.append(float(parts[0]))
                 mx = float(parts[1])
+                power.append(float(parts[2]))
             except ValueError:
                 continue
             for name, val in zip(names, parts[4:8]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_mhz_min": min(sm) if sm else None, "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
 
 
-def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks, budget_s: float = 0.0):
-    """Run the oracle (as it stands) on a bounded sample; returns (flops,
-    seconds, (head, query block) pairs done). With budget_s > 0 the sample
-    stops after the first pair that ends past the budget. q, k, v are in the
-    order the kernel computes in (tile-major for sliding-tile workloads)."""
+def oracle_sample(w: workloads.Workload, q, k, v, heads, row_sets, budget_s: float = 0.0, exact: bool = False,
+                  cache=None):
+    """Run the oracle (as it stands) on a bounded sample of the workload.
+
+    heads: (batch*head) indices; row_sets: arrays of query rows, each within
+    one 128-row block. q, k, v are the full CPU bf16 tensors, in the order the
+    kernel computes in (tile-major for sliding-tile workloads). The oracle
+    quantizes each sampled head once (its K and V serve every query row), then
+    runs the attention rows. With budget_s > 0 the sample stops after the
+    first row set that ends past the budget. With exact, each sampled row set
+    also runs through unquantized fp64 attention (untimed) for the cosine.
+    cache (a dict) keeps each head's quantized operands across calls; a head
+    found there is not quantized (nor timed) again.
+
+    Returns a dict: flops, attn_s, quant_s (seconds for the sampled heads'
+    quantization), done [(head, rows)], out {(head, i): oracle rows}, exact
+    {(head, i): fp64 rows}."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import parity
     from oracle import attention as oatt
@@ -159,23 +193,59 @@ def cpu_oracle_sample(w: workloads.Workload, q, k, v, heads, qblocks, budget_s: 
     if w.sparse:
         from oracle import sta
         kb = sta.block_lists(w.video, w.sta_tile, w.sta_window)
-    t0 = time.perf_counter()
-    flops = 0.0
-    done = []
+    B, H, N, d = q.shape
+    res = {"flops": 0.0, "attn_s": 0.0, "quant_s": 0.0, "done": [], "out": {}, "exact": {}}
+    t_start = time.perf_counter()
     for h in heads:
-        qh, kh, vh = parity.oracle_operands(q, k, v, w.qk_format, [h])
-        for qb in qblocks:
-            rows = np.arange(qb * 128, min(w.N, qb * 128 + 128))
-            oatt.attention_rows(qh[0], kh[0], vh[0], rows, causal=w.causal, key_blocks=kb)
+        if cache is not None and h in cache:
+            qh, kh, vh = cache[h]
+        else:
+            t0 = time.perf_counter()
+            qh, kh, vh = parity.oracle_operands(q, k, v, w.qk_format, [h])
+            res["quant_s"] += time.perf_counter() - t0
+            if cache is not None:
+                cache[h] = (qh, kh, vh)
+        for i, rows in enumerate(row_sets):
+            t0 = time.perf_counter()
+            o, _ = oatt.attention_rows(qh[0], kh[0], vh[0], rows, causal=w.causal, key_blocks=kb)
+            res["attn_s"] += time.perf_counter() - t0
             if kb is not None:
-                keys = np.full(len(rows), 128 * len(kb[qb]))
+                keys = np.full(len(rows), 128 * len(kb[int(rows[0]) // 128]))
             else:
-                keys = (rows + 1) if w.causal else np.full(len(rows), w.N)
-            flops += float(np.sum(4.0 * keys * w.d))
-            done.append((h, qb))
-            if budget_s > 0 and time.perf_counter() - t0 > budget_s:
-                return flops, time.perf_counter() - t0, done
-    return flops, time.perf_counter() - t0, done
+                keys = (rows + 1) if w.causal else np.full(len(rows), N)
+            res["flops"] += float(np.sum(4.0 * keys * d))
+            res["done"].append((h, rows))
+            res["out"][(h, i)] = o
+            if exact:
+                qe, ke, ve = (t.reshape(B * H, N, d)[h].double().numpy() for t in (q, k, v))
+                res["exact"][(h, i)], _ = oatt.attention_rows(qe, ke, ve, rows, causal=w.causal, key_blocks=kb,
+                                                              quantize_p=False)
+            if budget_s > 0 and time.perf_counter() - t_start > budget_s:
+                return res
+    return res
+
+
+def sample_rows(w: workloads.Workload, qblocks, target_flops: float = 2e9):
+    """Query rows per sampled block: as many of the block's first rows as make
+    about target_flops of oracle work (8 to 128 rows)."""
+    keys = w.N if not w.causal else max(1, w.N // 2)
+    n = int(min(128, max(8, target_flops / (4.0 * keys * w.d))))
+    return [np.arange(qb * 128, min(w.N, qb * 128 + n)) for qb in qblocks]
+
+
+def oracle_rate(res, N: int) -> float:
+    """Oracle TFLOPS on a sample: the attention rows' flops over their time
+    plus the sampled rows' share of the per-head quantization time (each
+    head's quantization serves all N of its rows)."""
+    rows = sum(len(r) for _, r in res["done"])
+    heads = len({h for h, _ in res["done"]})
+    t = res["attn_s"] + res["quant_s"] * rows / (heads * N)
+    return res["flops"] / t / 1e12
+
+
+def cosine(a: np.ndarray, b: np.ndarray) -> float:
+    a, b = a.astype(np.float64).ravel(), b.astype(np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
 
 
 def host_cores():
@@ -186,25 +256,35 @@ def host_cores():
 
 
 def run_reference(args, w):
-    """CPU oracle arm: each step a bounded sample of the workload."""
+    """CPU oracle arm: each step a bounded sample of the workload (about 2e9
+    flops of attention rows of one head), on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     q, k, v = workloads.make_qkv(w, heads=1, batch=1)
     nblk = (w.N + 127) // 128
-    qblocks = [nblk - 1, nblk // 2]
+    rows = sample_rows(w, [nblk - 1])
+    # one quantization of the head serves every step (as the inputs of the
+    # native arm stay resident); its time is charged per row sampled
+    tot = {"flops": 0.0, "attn_s": 0.0, "quant_s": 0.0, "done": []}
+    cache = {}
+    quant_s = oracle_sample(w, q, k, v, [0], rows, cache=cache)["quant_s"]
     for _ in range(args.warmup):
-        cpu_oracle_sample(w, q, k, v, [0], qblocks)
-    tot_f, tot_s = 0.0, 0.0
+        oracle_sample(w, q, k, v, [0], rows, cache=cache)
     for _ in range(args.steps):
-        f, s, _ = cpu_oracle_sample(w, q, k, v, [0], qblocks)
-        tot_f += f
-        tot_s += s
-    value = tot_f / tot_s / 1e12
-    sample = f"1 head, query blocks {qblocks} of {w.name} per step (oracle quantization of that head included)"
+        r = oracle_sample(w, q, k, v, [0], rows, cache=cache)
+        for key in ("flops", "attn_s"):
+            tot[key] += r[key]
+        tot["done"] += r["done"]
+    tot["quant_s"] = quant_s
+    value = oracle_rate(tot, w.N)
+    # per step: the sampled rows' attention plus their share of the quantization
+    step_s = tot["flops"] / args.steps / (value * 1e12)
+    sample = (f"{len(rows[0])} query rows of block {nblk - 1} of one head of {w.name} per step (fp64 numpy "
+              f"oracle; the head's quantization, {quant_s:.1f} s, charged per row: it serves all {w.N} rows)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_s,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(w),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
@@ -333,11 +413,11 @@ def run_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="llm_prefill_causal")
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_seq_128k_nvfp4", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--pv-format", default="fp8", choices=["fp8", "nvfp4"],
@@ -375,19 +455,24 @@ def main():
         tg = tuple(a // b for a, b in zip(w.video, w.sta_tile))
         mask = fp.sta_plan(tg, w.sta_tile, w.sta_window).to("cuda")
         video = fp.VideoLayout(w.video, w.sta_tile)
-    q_h, k_h, v_h = workloads.make_qkv(w, tile_major=video is None)
-    q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
+    if w.device_draw:
+        q, k, v = workloads.make_qkv(w, device="cuda")
+        q_h, k_h, v_h = q.cpu(), k.cpu(), v.cpu()
+    else:
+        q_h, k_h, v_h = workloads.make_qkv(w, tile_major=video is None)
+        q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
     stream = torch.cuda.current_stream()
 
     def step(ev_pair=None):
-        if w.qk_format == "nvfp4":
-            qq, kq = fp.quantize_nvfp4(q, video=video), fp.quantize_nvfp4(k, video=video)
+        if args.pv_format == "fp8":
+            # Q, K and V in four fused launches
+            qq, kq, vq = fp.quantize_qkv(q, k, v, w.qk_format, video=video)
         else:
-            qq, kq = fp.quantize_fp8(q, "tile128", video=video), fp.quantize_fp8(k, "tile128", video=video)
-        if args.pv_format == "nvfp4":
+            if w.qk_format == "nvfp4":
+                qq, kq = fp.quantize_nvfp4(q, video=video), fp.quantize_nvfp4(k, video=video)
+            else:
+                qq, kq = fp.quantize_fp8(q, "tile128", video=video), fp.quantize_fp8(k, "tile128", video=video)
             vq = fp.quantize_nvfp4_v(v, video=video)
-        else:
-            vq = fp.quantize_fp8(v, "channel", video=video)
         if ev_pair is not None:
             ev_pair[0].record(stream)
         out, lse = fp.attention_fwd(qq, kq, vq, causal=w.causal, tile_mask=mask, video=video,
@@ -396,30 +481,35 @@ def main():
             ev_pair[1].record(stream)
         return out
 
+    # clocks are sampled from before the warm-up; the summary keeps the
+    # samples inside the timed region
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert fp.device_error() == 0
 
-    clocks = ClockSampler(local)
     attn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    clocks.start()
+    t_host0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        step(attn_events[i])
+        out = step(attn_events[i])
     end.record(stream)
     torch.cuda.synchronize()
+    t_host1 = time.time()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(t_host0, t_host1)
     ms_total = start.elapsed_time(end)
     ms_total = rank_max(ms_total)
     attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_events]))
     attn_ms = rank_max(attn_ms)
     err = fp.device_error()
+    out_last = out.float().cpu() if rank == 0 else None
 
     pairs = executed_block_pairs(w)
     exec_flops = 4.0 * 128 * 128 * w.d * pairs * w.B * w.H
@@ -430,12 +520,18 @@ def main():
     ms_step = ms_total / args.steps
     value = aggregate_value(flops, world, ms_step)
     peaks, peak_src = load_peaks()
-    bf16 = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # A kernel timed inside a seconds-long loop runs under the power cap for
+    # most of it: the sustained bf16 figure applies. A shorter timed region
+    # is a burst.
+    timed_s = ms_total * 1e-3
+    sustained = timed_s >= 1.0 and "bf16_tflops_sustained" in peaks
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
     # both MMAs do 2d flops per score: the peak is the harmonic mean of theirs
     p_qk = p4 if w.qk_format == "nvfp4" else p8
     p_pv = p4 if args.pv_format == "nvfp4" else p8
     peak = 2.0 / (1.0 / p_qk + 1.0 / p_pv)
+    peak_burst = peak * peaks["bf16_tflops"] / bf16
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     quant_ms = ms_step - attn_ms
     quant_gbs = quant_bytes(w, args.pv_format) / (quant_ms * 1e-3) / 1e9
@@ -465,23 +561,51 @@ def main():
         e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    cpu = None
+    cpu, accuracy = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # about 15 s of oracle work: query blocks spread over the rows and heads
+        # a bounded oracle sample: query rows of four blocks spread over the
+        # sequence, of one head (two for short sequences); the same rows also
+        # give the accuracy figures against the kernel and against exact
+        # (unquantized fp64) attention
         nblk = (w.N + 127) // 128
         bh = w.B * w.H
-        heads = list(range(0, bh, max(1, bh // 32)))
-        qblocks = sorted({nblk - 1, (3 * nblk) // 4, nblk // 2, nblk // 4, 1, 0}, reverse=True)
-        qo, ko, vo = (q_h, k_h, v_h) if video is None else workloads.make_qkv(w)
-        f, s, done = cpu_oracle_sample(w, qo, ko, vo, heads, qblocks, budget_s=15.0)
-        cpu = {"value": f / s / 1e12, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
-               "sample": f"{len(done)} (batch*head, 128-query block) pairs of {w.name}: heads "
-                         f"{sorted(set(h for h, _ in done))} x query blocks {qblocks} in that order (fp64 "
-                         f"numpy oracle, its quantization of those heads included), {s:.1f} s"}
+        heads = [bh // 2] if w.N > 16384 else [0, bh - 1]
+        qblocks = sorted({0, nblk // 3, (2 * nblk) // 3, nblk - 1})
+        if w.sparse:
+            qo, ko, vo = workloads.make_qkv(w)     # tile-major, the order the kernel computes in
+        else:
+            qo, ko, vo = q_h, k_h, v_h
+        rows = sample_rows(w, qblocks)
+        res = oracle_sample(w, qo, ko, vo, heads, rows, budget_s=30.0, exact=True)
+        rate = oracle_rate(res, w.N)
+        nrows = sum(len(r) for _, r in res["done"])
+        cpu = {"value": rate, "unit": "TFLOPS", "cores": host_cores(), "kind": "oracle",
+               "sample": f"{nrows} query rows of {w.name}: heads {heads}, blocks {qblocks}, the first "
+                         f"{len(rows[0])} rows of each (fp64 numpy oracle; {res['attn_s']:.1f} s of attention "
+                         f"rows plus the heads' quantization, {res['quant_s']:.1f} s, charged per row)"}
+        # accuracy on the same rows: kernel output (raster order for video
+        # layouts is undone by the same permutation the oracle input used)
+        og = out_last.reshape(bh, w.N, w.d)
+        if video is not None:
+            perm = workloads.video_tile_major_perm(w.video, w.sta_tile)
+            og = og[:, perm]
+        ks, os_, ex = [], [], []
+        for i, (h, r) in enumerate(res["done"]):
+            ks.append(og[h, torch.from_numpy(r)].numpy())
+            os_.append(res["out"][(h, i % len(rows))])
+            ex.append(res["exact"][(h, i % len(rows))])
+        ks, os_, ex = (np.concatenate(x) for x in (ks, os_, ex))
+        accuracy = {"rows": nrows, "cos_vs_exact_kernel": cosine(ks, ex), "cos_vs_exact_oracle": cosine(os_, ex),
+                    "kernel_vs_oracle_rel_l2": float(np.linalg.norm(ks - os_) / np.linalg.norm(os_)),
+                    "kernel_vs_oracle_max_abs": float(np.abs(ks - os_).max())}
 
-    # Our kernels per step. Q/K: NVFP4 zero + amax + quantize + finalize each, or one FP8 kernel
-    # each. V: zero + amax + quantize + finalize (FP8 per channel or NVFP4). Attention: one.
-    launches_per_step = (8 if w.qk_format == "nvfp4" else 2) + 4 + 1
+    # Our kernels per step. FP8 V: the fused quantizer (zero, amax, convert, finalize) and the
+    # attention kernel. NVFP4 V: Q/K NVFP4 zero + amax + quantize + finalize each (or one FP8
+    # kernel each), V zero + amax + quantize + finalize, attention.
+    if args.pv_format == "fp8":
+        launches_per_step = 4 + 1
+    else:
+        launches_per_step = (8 if w.qk_format == "nvfp4" else 2) + 4 + 1
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -495,13 +619,17 @@ def main():
             "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,
             "quant_ms": quant_ms, "quant_gbs": quant_gbs, "quant_frac_hbm": quant_gbs / peaks["hbm_gbs"],
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": attn_tflops / peak,
-                         "traffic": profiled_traffic() if w.name == "llm_prefill_causal" else None,
-                         "peak_source": f"{peak_src} bf16 sustained {bf16} x nominal fp8 2x / fp4 4x; "
-                                        f"QK {'fp4' if w.qk_format == 'nvfp4' else 'fp8'}, "
-                                        f"PV {'fp4' if args.pv_format == 'nvfp4' else 'fp8'}, harmonic mean"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk, "device_error": err,
+                         "frac": attn_tflops / peak, "frac_of_burst_peak": attn_tflops / peak_burst,
+                         "traffic": profiled_traffic(w.name) if args.pv_format == "fp8" and
+                         not args.rescale_threshold else None,
+                         "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} {bf16} "
+                                        f"(timed region {timed_s:.2f} s: "
+                                        f"{'>= 1 s, under the power cap' if sustained else '< 1 s, a burst'}) "
+                                        f"x nominal fp8 2x / fp4 4x; QK "
+                                        f"{'fp4' if w.qk_format == 'nvfp4' else 'fp8'}, PV "
+                                        f"{'fp4' if args.pv_format == 'nvfp4' else 'fp8'}, harmonic mean"},
+            "accuracy": accuracy, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk, "device_error": err,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

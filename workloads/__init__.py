@@ -12,7 +12,8 @@ The workloads restate the ones the pages study:
     section 1: Wan2.1-14B 720p, 3D attention over video tokens),
   * sliding-tile sparse attention over (6,8,8)-token tiles (FPSAttention page,
     section 2.2, "STA"),
-  * a sequence-length sweep.
+  * a sequence-length sweep, and its longest single-GPU point (N = 128K,
+    d = 128, 32 heads) as a workload of its own.
 
 Recipe (all CPU torch.Generator, fp32 draws cast to bf16):
   * one generator per workload, seeded with the workload's seed; Q, then K,
@@ -22,6 +23,11 @@ Recipe (all CPU torch.Generator, fp32 draws cast to bf16):
   * smooth spatial bias for video workloads: for each channel c a frequency
     triple f in {1,2}^3 and a phase phi_c ~ U[0, 2pi); the bias
     ``sin(2pi(f_t t/T + f_h h/Hs + f_w w/W) + phi_c)`` is added to Q, K and V.
+  * ``make_qkv(..., device="cuda")`` draws the same recipe from a seeded CUDA
+    generator on the device (other bits than the CPU stream, same
+    distributions). The long-sequence workloads are defined by that device
+    stream: their three 1 GiB tensors take seconds on the device and about
+    half a minute on host cores.
 """
 from __future__ import annotations
 
@@ -52,6 +58,7 @@ class Workload:
     video: Optional[Tuple[int, int, int]] = None       # (T, Hs, W) token grid
     sta_tile: Optional[Tuple[int, int, int]] = None    # tile size in tokens
     sta_window: Optional[Tuple[int, int, int]] = None  # window size in tiles
+    device_draw: bool = False  # the recipe is drawn on the CUDA device (see make_qkv)
 
     @property
     def sparse(self) -> bool:
@@ -83,6 +90,12 @@ WORKLOADS = {
                               causal=False, qk_format="fp8", seed=4,
                               video=(18, 48, 80), sta_tile=(6, 8, 8),
                               sta_window=(3, 3, 5)),
+    # 5: the sequence sweep's longest single-GPU point, dense, x20 outliers;
+    # NVFP4 Q/K with FP8 P/V, and the all-FP8 variant. Drawn on the device.
+    "long_seq_128k_nvfp4": Workload("long_seq_128k_nvfp4", B=1, H=32, N=131072, d=128, causal=False,
+                                    qk_format="nvfp4", seed=5, outliers=True, device_draw=True),
+    "long_seq_128k_fp8": Workload("long_seq_128k_fp8", B=1, H=32, N=131072, d=128, causal=False,
+                                  qk_format="fp8", seed=5, outliers=True, device_draw=True),
 }
 
 
@@ -125,8 +138,9 @@ def video_tile_major_perm(grid: Tuple[int, int, int], tile: Tuple[int, int, int]
 
 def _video_bias(gen: torch.Generator, grid, d: int) -> torch.Tensor:
     T, Hs, W = grid
-    f = torch.randint(1, 3, (3, d), generator=gen).to(torch.float32)
-    phi = torch.rand(d, generator=gen) * (2 * math.pi)
+    dev = gen.device
+    f = torch.randint(1, 3, (3, d), generator=gen, device=dev).to(torch.float32).cpu()
+    phi = torch.rand(d, generator=gen, device=dev).cpu() * (2 * math.pi)
     t = torch.arange(T, dtype=torch.float32).view(T, 1, 1, 1) / T
     h = torch.arange(Hs, dtype=torch.float32).view(1, Hs, 1, 1) / Hs
     w = torch.arange(W, dtype=torch.float32).view(1, 1, W, 1) / W
@@ -135,34 +149,37 @@ def _video_bias(gen: torch.Generator, grid, d: int) -> torch.Tensor:
 
 
 def make_qkv(w: Workload, *, heads: Optional[int] = None, batch: Optional[int] = None,
-             N: Optional[int] = None, tile_major: bool = True):
-    """Return bf16 CPU tensors q, k, v of shape [B, H, N, d] for workload ``w``.
+             N: Optional[int] = None, tile_major: bool = True, device=None):
+    """Return bf16 tensors q, k, v of shape [B, H, N, d] for workload ``w``.
 
     ``heads``/``batch``/``N`` override the sizes for reduced parity cases; the
     seed and recipe stay the workload's. Sliding-tile workloads come in
     tile-major token order unless ``tile_major`` is False (raster order, as a
-    video model holds its tokens).
+    video model holds its tokens). ``device`` None draws from a CPU
+    generator and returns CPU tensors; a CUDA device draws from a CUDA
+    generator seeded the same way and returns tensors on that device.
     """
     B = w.B if batch is None else batch
     H = w.H if heads is None else heads
     n = w.N if N is None else N
     d = w.d
-    gen = torch.Generator().manual_seed(w.seed)
-    q = torch.randn(B, H, n, d, generator=gen)
-    k = torch.randn(B, H, n, d, generator=gen)
-    v = torch.randn(B, H, n, d, generator=gen)
+    dev = torch.device("cpu") if device is None else torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(w.seed)
+    q = torch.randn(B, H, n, d, generator=gen, device=dev)
+    k = torch.randn(B, H, n, d, generator=gen, device=dev)
+    v = torch.randn(B, H, n, d, generator=gen, device=dev)
     if w.outliers:
         for hh in range(H):
-            ch = torch.randperm(d, generator=gen)[:4]
+            ch = torch.randperm(d, generator=gen, device=dev)[:4]
             q[:, hh, :, ch] *= 20.0
             k[:, hh, :, ch] *= 20.0
     if w.video is not None and n == w.N:
-        bias = _video_bias(gen, w.video, d)
+        bias = _video_bias(gen, w.video, d).to(dev)
         q += bias
         k += bias
         v += bias
         if w.sta_tile is not None and tile_major:
-            perm = video_tile_major_perm(w.video, w.sta_tile)
+            perm = video_tile_major_perm(w.video, w.sta_tile).to(dev)
             q, k, v = q[:, :, perm], k[:, :, perm], v[:, :, perm]
     return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(),
             v.to(torch.bfloat16).contiguous())
