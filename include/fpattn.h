@@ -157,6 +157,32 @@ fpattn_status fpattn_quantize_fp8_group(const fpattn_tensor* x, const struct fpa
                                         int32_t* nonfinite_flag, fpattn_stream_t stream);
 
 /*
+ * Q, K and V of one attention call quantized together, in four launches
+ * (zero the accumulators, one amax pass over the three tensors, one
+ * conversion pass, one finalize) instead of four per tensor. The results are
+ * bit for bit those of the separate calls:
+ *   qk_dtype FPATTN_NVFP4: q, k as fpattn_quantize_nvfp4 (dynamic amax),
+ *     q_block_sf / k_block_sf fpattn_nvfp4_sf_bytes() each, q_scale /
+ *     k_scale one float each (s_t);
+ *   qk_dtype FPATTN_E4M3: q, k as fpattn_quantize_fp8(FPATTN_FP8_TILE128),
+ *     q_scale / k_scale B*H*ceil(N/128) floats, q_block_sf = k_block_sf =
+ *     NULL;
+ *   v as fpattn_quantize_fp8(FPATTN_FP8_CHANNEL): v_codes B*H*N*d bytes,
+ *     v_scales B*H*d floats.
+ * q, k, v: bf16 tensors of one shape. layout: NULL, or all three in raster
+ * order of a video (codes and per-tile scales come out tile-major, as from
+ * the _video calls). Errors as the separate calls; q, k, v of different
+ * shapes or a qk_dtype other than the two: FPATTN_ERR_INVALID_ARG /
+ * FPATTN_ERR_UNSUPPORTED. The Q/K scale outputs hold amax partial results
+ * until the last launch has run (stream order makes that invisible).
+ */
+fpattn_status fpattn_quantize_qkv(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                                  int32_t qk_dtype, const struct fpattn_video_layout_s* layout, uint8_t* q_codes,
+                                  uint8_t* q_block_sf, float* q_scale, uint8_t* k_codes, uint8_t* k_block_sf,
+                                  float* k_scale, uint8_t* v_codes, float* v_scales, int32_t* nonfinite_flag,
+                                  fpattn_stream_t stream);
+
+/*
  * Phase of denoising step t of num_steps (FPSAttention page, section 3.2):
  * with t1 = alpha1 * num_steps and t2 = alpha2 * num_steps (the page deploys
  * alpha1 = 0.2, alpha2 = 0.7), t <= t1 is early (coarse granularity, sparse
@@ -241,6 +267,19 @@ typedef struct {
   const int32_t* col_idx;  /* nnz entries */
   const int32_t* row_order;
 } fpattn_tile_mask_desc;
+
+/*
+ * HOST-only check of a tile mask held in HOST arrays (for instance before
+ * copying it to the device for fpattn_fwd), with no CUDA call. FPATTN_OK when
+ * row_ptr[0] = 0, row_ptr is non-decreasing with row_ptr[nblk] = nnz, every
+ * row's col_idx entries are strictly ascending and in [0, nblk), and
+ * row_order (may be NULL) is a permutation of 0 .. nblk-1; else
+ * FPATTN_ERR_INVALID_ARG. fpattn_fwd cannot read device arrays before its
+ * launch: given a mask that fails this check, it reads no memory outside the
+ * arrays and tensors, but its results are unspecified.
+ */
+fpattn_status fpattn_tile_mask_check(int32_t nblk, int32_t nnz, const int32_t* row_ptr, const int32_t* col_idx,
+                                     const int32_t* row_order);
 
 /*
  * 3D sliding-tile planner (FPSAttention page, section 2.2: query tile u

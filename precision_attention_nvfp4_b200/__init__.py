@@ -12,6 +12,9 @@ Public calls
                                   group_tiles tiles per scale
                                   (with video=VideoLayout: x in raster order,
                                   codes and scales in tile-major order)
+  quantize_qkv(q, k, v, fmt)   -> (q, k, v) quantized together: Q/K NVFP4 or
+                                  FP8 per tile, V FP8 per channel, in four
+                                  fused launches (same bits as the calls above)
   quantize_nvfp4_v(x)          -> Nvfp4VTensor: V in NVFP4 with 16-token
                                   blocks, channel-major (all-NVFP4 attention)
   sta_plan(grid, tile, window) -> StaPlan (host CSR over 128-token blocks)
@@ -36,9 +39,10 @@ import torch
 from . import _lib
 from ._lib import FpattnError
 
-__all__ = ["Nvfp4Tensor", "Nvfp4VTensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4",
+__all__ = ["Nvfp4Tensor", "Nvfp4VTensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_qkv",
            "quantize_nvfp4_v", "quantize_fp8", "sta_plan",
-           "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError"]
+           "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError",
+           "head_range"]
 
 
 def library() -> ctypes.CDLL:
@@ -171,11 +175,50 @@ def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
     return Fp8Tensor(codes, scales, granularity, (B, H, N, d))
 
 
+def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, qk_format: str = "nvfp4",
+                 nonfinite_flag: Optional[torch.Tensor] = None, video: Optional[VideoLayout] = None):
+    """Q and K (NVFP4, or FP8 per 128-token tile) and V (FP8 per channel) in
+    four fused launches; returns (q, k, v) quantized exactly as the separate
+    quantize_nvfp4 / quantize_fp8 calls would."""
+    B, H, N, d = _check_bf16(q)
+    if _check_bf16(k) != (B, H, N, d) or _check_bf16(v) != (B, H, N, d):
+        raise ValueError("q, k, v must have one shape")
+    lib = library()
+    dev = q.device
+    nblk = (N + 127) // 128
+    if qk_format == "nvfp4":
+        dt = _lib.NVFP4
+        qc, kc = (torch.empty((B, H, N, d // 2), dtype=torch.uint8, device=dev) for _ in range(2))
+        qsf, ksf = (torch.empty(lib.fpattn_nvfp4_sf_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+                    for _ in range(2))
+        qs, ks = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2))
+    elif qk_format == "fp8":
+        dt = _lib.E4M3
+        qc, kc = (torch.empty((B, H, N, d), dtype=torch.uint8, device=dev) for _ in range(2))
+        qsf = ksf = None
+        qs, ks = (torch.empty((B, H, nblk), dtype=torch.float32, device=dev) for _ in range(2))
+    else:
+        raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
+    vc = torch.empty((B, H, N, d), dtype=torch.uint8, device=dev)
+    vs = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    st = lib.fpattn_quantize_qkv(ctypes.byref(_desc(q, _lib.BF16, B, H, N, d)),
+                                 ctypes.byref(_desc(k, _lib.BF16, B, H, N, d)),
+                                 ctypes.byref(_desc(v, _lib.BF16, B, H, N, d)), dt, _video_ref(video),
+                                 qc.data_ptr(), _ptr(qsf), qs.data_ptr(), kc.data_ptr(), _ptr(ksf), ks.data_ptr(),
+                                 vc.data_ptr(), vs.data_ptr(), _ptr(nonfinite_flag), _stream())
+    _lib.check(st, "fpattn_quantize_qkv")
+    if qk_format == "nvfp4":
+        qq, kq = Nvfp4Tensor(qc, qsf, qs, (B, H, N, d)), Nvfp4Tensor(kc, ksf, ks, (B, H, N, d))
+    else:
+        qq, kq = Fp8Tensor(qc, qs, "tile128", (B, H, N, d)), Fp8Tensor(kc, ks, "tile128", (B, H, N, d))
+    return qq, kq, Fp8Tensor(vc, vs, "channel", (B, H, N, d))
+
+
 @dataclasses.dataclass
 class StaPlan:
     row_ptr: np.ndarray    # int32 [nblk + 1]
     col_idx: np.ndarray    # int32 [nnz]
-    row_order: np.ndarray  # int32 [nblk], longest rows first
+    row_order: Optional[np.ndarray]  # int32 [nblk], longest rows first, or None
 
     @property
     def nblk(self) -> int:
@@ -185,11 +228,25 @@ class StaPlan:
     def nnz(self) -> int:
         return len(self.col_idx)
 
+    def check(self) -> None:
+        """Raises FpattnError unless the CSR is well formed (fpattn_tile_mask_check)."""
+        rp = np.ascontiguousarray(self.row_ptr, dtype=np.int32)
+        ci = np.ascontiguousarray(self.col_idx, dtype=np.int32)
+        ro = None if self.row_order is None else np.ascontiguousarray(self.row_order, dtype=np.int32)
+        if len(rp) < 1 or (ro is not None and len(ro) != len(rp) - 1):
+            raise FpattnError(_lib.ERR_INVALID_ARG, "fpattn_tile_mask_check")
+        _lib.check(library().fpattn_tile_mask_check(len(rp) - 1, len(ci), rp.ctypes.data,
+                                                    ci.ctypes.data if len(ci) else None,
+                                                    None if ro is None else ro.ctypes.data),
+                   "fpattn_tile_mask_check")
+
     def to(self, device) -> "DeviceTileMask":
+        """Checks the mask on the host, then copies it to ``device``."""
+        self.check()
         return DeviceTileMask(self.nblk, self.nnz,
                               torch.from_numpy(self.row_ptr).to(device),
                               torch.from_numpy(self.col_idx).to(device),
-                              torch.from_numpy(self.row_order).to(device))
+                              None if self.row_order is None else torch.from_numpy(self.row_order).to(device))
 
 
 @dataclasses.dataclass
@@ -228,6 +285,50 @@ def step_phase(t: int, num_steps: int, alpha1: float = 0.2, alpha2: float = 0.7)
     return ph.value
 
 
+def _check_operands(q, k, v) -> None:
+    """Refuses, before any launch, operands the kernel would read past: q and
+    k both NVFP4 or both FP8 with per-tile scales, v FP8 with per-channel
+    scales or NVFP4 V, one shape [B, H, N, d] for all three, every buffer
+    sized for that shape and on one CUDA device."""
+    if isinstance(q, Nvfp4Tensor) and isinstance(k, Nvfp4Tensor):
+        pass
+    elif isinstance(q, Fp8Tensor) and isinstance(k, Fp8Tensor):
+        if q.granularity != "tile128" or k.granularity != "tile128":
+            raise ValueError("FP8 q and k need per-tile scales (granularity 'tile128' or 'group')")
+    else:
+        raise TypeError("q and k must both be Nvfp4Tensor or both Fp8Tensor")
+    if isinstance(v, Fp8Tensor):
+        if v.granularity != "channel":
+            raise ValueError("FP8 v needs per-channel scales (granularity 'channel')")
+    elif not isinstance(v, Nvfp4VTensor):
+        raise TypeError("v must be an Fp8Tensor (per channel) or an Nvfp4VTensor")
+    if not (tuple(q.shape) == tuple(k.shape) == tuple(v.shape)):
+        raise ValueError(f"q, k, v shapes differ: {q.shape}, {k.shape}, {v.shape}")
+    B, H, N, d = q.shape
+    nblk = (N + 127) // 128
+    dev = v.codes.device
+    for name, t in (("q", q), ("k", k)):
+        if isinstance(t, Nvfp4Tensor):
+            need = {"codes": B * H * N * d // 2, "block_sf": B * H * nblk * (d // 64) * 512, "tensor_scale": 1}
+        else:
+            need = {"codes": B * H * N * d, "scales": B * H * nblk}
+        _check_buffers(name, t, need, dev)
+    if isinstance(v, Nvfp4VTensor):
+        need = {"codes": B * H * d * 64 * nblk, "block_sf": B * H * nblk * 1024, "tensor_scale": 1}
+    else:
+        need = {"codes": B * H * N * d, "scales": B * H * d}
+    _check_buffers("v", v, need, dev)
+
+
+def _check_buffers(name, t, need, dev) -> None:
+    for field, n in need.items():
+        buf = getattr(t, field)
+        if not buf.is_cuda or buf.device != dev or not buf.is_contiguous():
+            raise ValueError(f"{name}.{field}: expected a contiguous tensor on {dev}")
+        if buf.numel() < n:
+            raise ValueError(f"{name}.{field}: {buf.numel()} elements, the shape {tuple(t.shape)} needs {n}")
+
+
 def attention_fwd(q, k, v, *, causal: bool = False, tile_mask: Optional[DeviceTileMask] = None,
                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, return_lse: bool = True,
@@ -241,25 +342,24 @@ def attention_fwd(q, k, v, *, causal: bool = False, tile_mask: Optional[DeviceTi
     order. ``rescale_threshold`` (tau, log2 units, 0..8) skips the O / l
     rescale until a row's max has grown by more than tau; 0 is exact.
     """
+    _check_operands(q, k, v)
     B, H, N, d = v.shape
     lib = library()
     if isinstance(v, Nvfp4VTensor):
-        vd, v_scale, v_sf = _desc(v.codes, _lib.NVFP4, B, H, N, d), v.tensor_scale.data_ptr(), v.block_sf.data_ptr()
+        vd, v_scale, v_sf = _desc(v.codes, _lib.NVFP4, *v.shape), v.tensor_scale.data_ptr(), v.block_sf.data_ptr()
     else:
-        vd, v_scale, v_sf = _desc(v.codes, _lib.E4M3, B, H, N, d), v.scales.data_ptr(), None
-    if isinstance(q, Nvfp4Tensor) and isinstance(k, Nvfp4Tensor):
-        qd = _desc(q.codes, _lib.NVFP4, B, H, N, d)
-        kd = _desc(k.codes, _lib.NVFP4, B, H, N, d)
+        vd, v_scale, v_sf = _desc(v.codes, _lib.E4M3, *v.shape), v.scales.data_ptr(), None
+    if isinstance(q, Nvfp4Tensor):
+        qd = _desc(q.codes, _lib.NVFP4, *q.shape)
+        kd = _desc(k.codes, _lib.NVFP4, *k.shape)
         sc = _lib.Scales(q.tensor_scale.data_ptr(), k.tensor_scale.data_ptr(), v_scale,
                          q.block_sf.data_ptr(), k.block_sf.data_ptr(), 1.0 / 448.0, softmax_scale,
                          rescale_threshold, v_sf)
-    elif isinstance(q, Fp8Tensor) and isinstance(k, Fp8Tensor):
-        qd = _desc(q.codes, _lib.E4M3, B, H, N, d)
-        kd = _desc(k.codes, _lib.E4M3, B, H, N, d)
+    else:
+        qd = _desc(q.codes, _lib.E4M3, *q.shape)
+        kd = _desc(k.codes, _lib.E4M3, *k.shape)
         sc = _lib.Scales(q.scales.data_ptr(), k.scales.data_ptr(), v_scale, None, None,
                          1.0 / 448.0, softmax_scale, rescale_threshold, v_sf)
-    else:
-        raise TypeError("q and k must both be Nvfp4Tensor or both Fp8Tensor")
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.codes.device)
     if lse is None and return_lse:
@@ -299,20 +399,20 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
         q = q.to(dev, non_blocking=True)
         k = k.to(dev, non_blocking=True)
         v = v.to(dev, non_blocking=True)
-    if qk_format == "nvfp4":
-        qq, kq = quantize_nvfp4(q, video=video), quantize_nvfp4(k, video=video)
-    elif qk_format == "fp8":
-        gran = "group" if qk_group_tiles > 1 else "tile128"
-        qq = quantize_fp8(q, gran, video=video, group_tiles=qk_group_tiles)
-        kq = quantize_fp8(k, gran, video=video, group_tiles=qk_group_tiles)
-    else:
+    if qk_format not in ("nvfp4", "fp8"):
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
-    if pv_format == "fp8":
-        vq = quantize_fp8(v, "channel", video=video)
-    elif pv_format == "nvfp4":
-        vq = quantize_nvfp4_v(v, video=video)
-    else:
+    if pv_format not in ("fp8", "nvfp4"):
         raise ValueError("pv_format must be 'fp8' or 'nvfp4'")
+    if pv_format == "fp8" and qk_group_tiles <= 1:
+        qq, kq, vq = quantize_qkv(q, k, v, qk_format, video=video)   # four fused launches
+    else:
+        if qk_format == "nvfp4":
+            qq, kq = quantize_nvfp4(q, video=video), quantize_nvfp4(k, video=video)
+        else:
+            gran = "group" if qk_group_tiles > 1 else "tile128"
+            qq = quantize_fp8(q, gran, video=video, group_tiles=qk_group_tiles)
+            kq = quantize_fp8(k, gran, video=video, group_tiles=qk_group_tiles)
+        vq = quantize_fp8(v, "channel", video=video) if pv_format == "fp8" else quantize_nvfp4_v(v, video=video)
     out, lse = attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
                              return_lse=return_lse, video=video, rescale_threshold=rescale_threshold)
     if host:
@@ -326,6 +426,19 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
         torch.cuda.current_stream().synchronize()
         return out_h, lse_h
     return out, lse
+
+
+def head_range(num_heads: int, world: int, rank: int) -> Tuple[int, int]:
+    """Rank ``rank``'s share [start, stop) of ``num_heads`` independent
+    (batch, head) problems split over ``world`` ranks: contiguous ranges in
+    rank order, the first ``num_heads % world`` ranks taking one more. The
+    flattened [B*H, N, d] view of a contiguous [B, H, N, d] tensor makes each
+    share one contiguous slice."""
+    if world < 1 or not 0 <= rank < world or num_heads < 0:
+        raise ValueError("need world >= 1, 0 <= rank < world, num_heads >= 0")
+    base, extra = divmod(num_heads, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
 
 
 def device_error(clear: bool = True) -> int:

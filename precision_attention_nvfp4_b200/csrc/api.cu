@@ -33,7 +33,8 @@ fpattn_status check_tensor(const fpattn_tensor* t, int dtype) {
   // keep every index of the kernels inside 32-bit block / item counters
   const long long bh = static_cast<long long>(t->B) * t->H;
   const long long nblk = (t->N + 127) / 128;
-  if (bh * nblk > (1ll << 30) || t->N > (1 << 28)) return FPATTN_ERR_UNSUPPORTED;
+  // (b, h) is the grid's y index in the quantize kernels: at most 65535
+  if (bh > 65535 || bh * nblk > (1ll << 30) || t->N > (1 << 28)) return FPATTN_ERR_UNSUPPORTED;
   if (!aligned16(t->data)) return FPATTN_ERR_ALIGNMENT;
   return FPATTN_OK;
 }
@@ -87,6 +88,35 @@ fpattn_status quantize_fp8(const fpattn_tensor* x, const fpattn_video_layout* la
     return from_cuda(
         fpattn::launch_quantize_fp8_channel(x->data, BH, x->N, x->d, codes, scales, nonfinite_flag, tmp, st));
   return FPATTN_ERR_INVALID_ARG;
+}
+
+fpattn_status quantize_qkv(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v, int32_t qk_dtype,
+                          const fpattn_video_layout* layout, uint8_t* q_codes, uint8_t* q_block_sf, float* q_scale,
+                          uint8_t* k_codes, uint8_t* k_block_sf, float* k_scale, uint8_t* v_codes,
+                          float* v_scales, int32_t* nonfinite_flag, fpattn_stream_t stream) {
+  fpattn_status s;
+  if ((s = check_tensor(q, FPATTN_BF16)) != FPATTN_OK) return s;
+  if ((s = check_tensor(k, FPATTN_BF16)) != FPATTN_OK) return s;
+  if ((s = check_tensor(v, FPATTN_BF16)) != FPATTN_OK) return s;
+  if (k->B != q->B || k->H != q->H || k->N != q->N || k->d != q->d || v->B != q->B || v->H != q->H ||
+      v->N != q->N || v->d != q->d)
+    return FPATTN_ERR_INVALID_ARG;
+  if (qk_dtype != FPATTN_NVFP4 && qk_dtype != FPATTN_E4M3) return FPATTN_ERR_UNSUPPORTED;
+  const bool fp4 = qk_dtype == FPATTN_NVFP4;
+  fpattn::VideoLayout vl;
+  fpattn::TokenMap tm;
+  if (layout && (s = check_layout(layout, q->N, &vl, &tm)) != FPATTN_OK) return s;
+  if (!q_codes || !k_codes || !v_codes || !q_scale || !k_scale || !v_scales) return FPATTN_ERR_INVALID_ARG;
+  if (fp4 ? (!q_block_sf || !k_block_sf) : (q_block_sf || k_block_sf)) return FPATTN_ERR_INVALID_ARG;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !aligned16(v_codes)) return FPATTN_ERR_ALIGNMENT;
+  if (fp4 && (!aligned16(q_block_sf) || !aligned16(k_block_sf))) return FPATTN_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+       reinterpret_cast<uintptr_t>(v_scales)) & 3u)
+    return FPATTN_ERR_ALIGNMENT;
+  return from_cuda(fpattn::launch_quantize_qkv(q->data, k->data, v->data, q->B * q->H, q->N, q->d, fp4, q_codes,
+                                               q_block_sf, q_scale, k_codes, k_block_sf, k_scale, v_codes,
+                                               v_scales, nonfinite_flag, layout ? &tm : nullptr,
+                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fpattn_status quantize_nvfp4_v(const fpattn_tensor* x, const fpattn_video_layout* layout, const float* static_amax,
@@ -170,6 +200,7 @@ fpattn_status fwd(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_t
   a.row_ptr = tile_mask ? tile_mask->row_ptr : nullptr;
   a.col_idx = tile_mask ? tile_mask->col_idx : nullptr;
   a.row_order = tile_mask ? tile_mask->row_order : nullptr;
+  a.nnz = tile_mask ? tile_mask->nnz : 0;
   a.B = q->B;
   a.H = q->H;
   a.N = q->N;
@@ -200,6 +231,15 @@ fpattn_status fpattn_quantize_nvfp4(const fpattn_tensor* x, const float* static_
 fpattn_status fpattn_quantize_fp8(const fpattn_tensor* x, int32_t granularity, uint8_t* codes, float* scales,
                                   int32_t* nonfinite_flag, fpattn_stream_t stream) {
   return quantize_fp8(x, nullptr, granularity, codes, scales, nonfinite_flag, stream);
+}
+
+fpattn_status fpattn_quantize_qkv(const fpattn_tensor* q, const fpattn_tensor* k, const fpattn_tensor* v,
+                                  int32_t qk_dtype, const fpattn_video_layout* layout, uint8_t* q_codes,
+                                  uint8_t* q_block_sf, float* q_scale, uint8_t* k_codes, uint8_t* k_block_sf,
+                                  float* k_scale, uint8_t* v_codes, float* v_scales, int32_t* nonfinite_flag,
+                                  fpattn_stream_t stream) {
+  return quantize_qkv(q, k, v, qk_dtype, layout, q_codes, q_block_sf, q_scale, k_codes, k_block_sf, k_scale,
+                      v_codes, v_scales, nonfinite_flag, stream);
 }
 
 fpattn_status fpattn_video_layout_check(const fpattn_video_layout* layout, int32_t N) {
@@ -319,6 +359,29 @@ fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, in
     return (row_ptr[x + 1] - row_ptr[x]) > (row_ptr[y + 1] - row_ptr[y]);
   });
   std::memcpy(row_order, order.data(), sizeof(int32_t) * nblk);
+  return FPATTN_OK;
+}
+
+fpattn_status fpattn_tile_mask_check(int32_t nblk, int32_t nnz, const int32_t* row_ptr, const int32_t* col_idx,
+                                     const int32_t* row_order) {
+  if (nblk <= 0 || nnz < 0 || !row_ptr || (nnz > 0 && !col_idx)) return FPATTN_ERR_INVALID_ARG;
+  if (row_ptr[0] != 0 || row_ptr[nblk] != nnz) return FPATTN_ERR_INVALID_ARG;
+  for (int32_t r = 0; r < nblk; ++r) {
+    const int32_t b = row_ptr[r], e = row_ptr[r + 1];
+    if (e < b || e > nnz) return FPATTN_ERR_INVALID_ARG;
+    for (int32_t i = b; i < e; ++i) {
+      if (col_idx[i] < 0 || col_idx[i] >= nblk) return FPATTN_ERR_INVALID_ARG;
+      if (i > b && col_idx[i] <= col_idx[i - 1]) return FPATTN_ERR_INVALID_ARG;
+    }
+  }
+  if (row_order) {
+    std::vector<char> seen(static_cast<size_t>(nblk), 0);
+    for (int32_t r = 0; r < nblk; ++r) {
+      const int32_t x = row_order[r];
+      if (x < 0 || x >= nblk || seen[x]) return FPATTN_ERR_INVALID_ARG;
+      seen[x] = 1;
+    }
+  }
   return FPATTN_OK;
 }
 

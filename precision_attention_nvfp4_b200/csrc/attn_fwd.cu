@@ -49,6 +49,7 @@
 // dependent launch) only after its prologue.
 // Work items are (batch*head, 128-query block); causal runs schedule the
 // longest query blocks first, tile-mask runs follow the mask's row order.
+#include <atomic>
 #include <cfloat>
 #include <cstdint>
 #include <cstdio>
@@ -67,7 +68,23 @@ __device__ int g_error_word = 0;
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kStages = 3;
+// Depth of the K/V shared-memory ring (and of the rings that follow it: O
+// rescale hand-off, O done).
+#ifndef FPATTN_KV_STAGES
+#define FPATTN_KV_STAGES 3
+#endif
+constexpr int kStages = FPATTN_KV_STAGES;
+// One thread issues both MMA kinds in a fixed interleave (else one thread each).
+#ifndef FPATTN_ONE_ISSUER
+#define FPATTN_ONE_ISSUER 0
+#endif
+constexpr bool kOneIssuer = FPATTN_ONE_ISSUER != 0;
+// Softmax exponentials taken against the previous reference max, before the
+// block's max is known (E4M3 P only).
+#ifndef FPATTN_SPECULATE
+#define FPATTN_SPECULATE 0
+#endif
+constexpr bool kSpeculate = FPATTN_SPECULATE != 0;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
@@ -76,7 +93,7 @@ constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
 enum : int {
   kErrQEmpty = 0x101, kErrKvEmpty = 0x102, kErrQFull = 0x201, kErrKFull = 0x202, kErrVFull = 0x203,
   kErrPFull = 0x204, kErrOReady = 0x205, kErrSFull = 0x301, kErrMax = 0x303, kErrFin = 0x304,
-  kErrAlpha = 0x305, kErrSFree = 0x306, kErrODone = 0x302, kErrDrain = 0x401
+  kErrAlpha = 0x305, kErrSFree = 0x306, kErrODone = 0x302, kErrPFree = 0x307, kErrDrain = 0x401
 };
 
 // FP4: Q, K in NVFP4 (else E4M3). PV4: P and V in NVFP4 and P V on the
@@ -100,14 +117,19 @@ struct Cfg {
   // polynomial (measured best: 3 next to the cheaper FP4 QK^T, 4 with FP8)
   static constexpr int kPolyPairs = FP4 ? 3 : 4;
   static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
-  // P buffers, 32 columns each (128 E4M3 keys). As many as K/V stages: the
-  // S of block g needs K stage g % kStages, which is refilled only after the
-  // PV of block g - kStages has completed, and that PV was the last reader of
-  // P buffer g % kPBufs. So a softmax thread that has seen S(g) may overwrite
-  // the buffer without a barrier of its own.
-  static constexpr int kPBufs = kStages;
+  // P buffers, 32 columns each (128 E4M3 keys), as many as K/V stages when
+  // tensor memory holds them: the S of block g needs K stage g % kStages,
+  // which is refilled only after the PV of block g - kStages has completed,
+  // and that PV was the last reader of P buffer g % kPBufs. So a softmax
+  // thread that has seen S(g) may overwrite the buffer without a barrier of
+  // its own. With fewer P buffers than stages (NVFP4 Q/K at four stages: the
+  // scale vectors take the columns of the fourth), the softmax waits for the
+  // PV of block g - kPBufs before writing P buffer g % kPBufs.
   static constexpr uint32_t kColP = 384;
   static constexpr uint32_t kPCols = PV4 ? 16 : 32;       // per P buffer: 128 keys of E2M1 or E4M3
+  static constexpr int kPBufs =
+      kColP + kPCols * kStages + (FP4 ? 3 * 4 * (D / 64) : 0) + (PV4 ? 32 : 0) <= 512 ? kStages : 3;
+  static constexpr bool kPWait = kPBufs < kStages;
   static constexpr uint32_t kColSFQ = kColP + kPCols * kPBufs;
   static constexpr uint32_t kSFCols = 4 * (D / 64);
   static constexpr uint32_t kColSFK = kColSFQ + kSFCols;  // + buf * kSFCols
@@ -115,6 +137,7 @@ struct Cfg {
   static constexpr uint32_t kColSFP = kColSFK + (FP4 ? 2 * kSFCols : 0);  // + (g & 1) * 8
   static constexpr uint32_t kColSFV = kColSFP + 16;                       // + (g & 1) * 8
   static_assert(!PV4 || kColSFV + 16 <= 512, "tensor memory columns");
+  static_assert(kColP + kPCols * kPBufs + (FP4 ? 3 * kSFCols : 0) <= 512, "tensor memory columns");
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQKTile;
@@ -141,6 +164,7 @@ struct Cfg {
   // Request at least this much so that a single CTA fits per SM (it takes
   // all 512 tensor-memory columns).
   static constexpr int kSmemRequest = (kBytes + 1024 > 120 * 1024 ? kBytes + 1024 : 120 * 1024);
+  static_assert(kSmemRequest <= 227 * 1024, "shared memory per CTA");
 };
 
 struct __align__(64) Params {
@@ -163,6 +187,7 @@ struct __align__(64) Params {
   const int32_t* col_idx;
   const int32_t* row_order;
   int N, nblk, BH, num_items;
+  int nnz;  // tile mask entries (sparse runs)
   int causal, sparse;
   float sm_scale_log2;
   float tau;           // conditional-rescale threshold, log2 units (0: exact running max)
@@ -182,11 +207,18 @@ __device__ __forceinline__ int sched_item(int r) {
                                   : static_cast<int>(blockIdx.x));
 }
 
+// The tile mask's arrays come from the caller: the host entry points check
+// them, and the kernel also keeps every index it derives from them in range
+// (a query block outside [0, nblk) is taken as block 0, a row's end is
+// clipped to nnz, a key block outside [0, nblk) is loaded as block 0 and
+// fully masked), so a malformed mask can give wrong results but never an
+// out-of-bounds access.
 __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, int& qb) {
   if (p.sparse) {
     const int r = item / p.BH;
     bh = item % p.BH;
     qb = p.row_order ? p.row_order[r] : r;
+    if (static_cast<unsigned>(qb) >= static_cast<unsigned>(p.nblk)) qb = 0;
   } else if (p.causal) {
     qb = p.nblk - 1 - item / p.BH;  // longest rows first
     bh = item % p.BH;
@@ -198,8 +230,9 @@ __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, 
 
 __device__ __forceinline__ KList key_list(const Params& p, int qb) {
   if (p.sparse) {
-    const int b = p.row_ptr[qb];
-    int e = p.row_ptr[qb + 1];
+    const int e0 = min(p.row_ptr[qb + 1], p.nnz);
+    const int b = max(0, min(p.row_ptr[qb], e0));
+    int e = e0;
     if (p.causal) {
       int n = b;
       while (n < e && p.col_idx[n] <= qb) ++n;
@@ -210,8 +243,11 @@ __device__ __forceinline__ KList key_list(const Params& p, int qb) {
   return {0, p.causal ? qb + 1 : p.nblk};
 }
 
+// Key block j of a query block's list; -1 for an entry outside [0, nblk).
 __device__ __forceinline__ int key_block(const Params& p, const KList& L, int j) {
-  return p.sparse ? p.col_idx[L.begin + j] : j;
+  if (!p.sparse) return j;
+  const int kb = p.col_idx[L.begin + j];
+  return static_cast<unsigned>(kb) < static_cast<unsigned>(p.nblk) ? kb : -1;
 }
 
 // Masks the scores of one 32-key chunk (keys key0..key0+31) that fall past
@@ -468,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           const int use = g / kStages;
           if (use > 0 && !(ok = mbar_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty)))
             break;
-          const int kb = key_block(p, L, j);
+          const int kb = max(key_block(p, L, j), 0);
           mbar_arrive_expect_tx(k_full + st, C::kQKTile + C::kSF);
           tma_load_3d_hint(smem + C::kOffK + st * C::kQKTile, &p.tm_k, k_full + st, 0, kb * 128, bh, keep);
           if (FP4)
@@ -486,73 +522,77 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ PV issuer
+  } else if (warp == 1 || (!kOneIssuer && warp == 2)) {
+    // ------------------------------------------------------- MMA issue
+    // Warp 1 issues O += P V, warp 2 issues S = Q K^T (one thread each);
+    // with kOneIssuer, warp 1 issues both in the fixed order S(0), S(1),
+    // PV(0), S(2), PV(1), S(3), ...: the S of block g + 2 follows the PV of
+    // block g on the in-order tensor pipe, so no S is queued ahead of a PV
+    // the softmax is waiting to see complete.
     if (lane == 0) {
       constexpr uint32_t kIdescPV = PV4 ? idesc_nvf4(128, D) : idesc_e4m3(128, D, true);
-      int g = 0;
-      bool ok = true;
-      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
-        int bh, qb;
-        decode_item(p, item, bh, qb);
-        const KList L = key_list(p, qb);
-        for (int j = 0; j < L.count; ++j, ++g) {
-          // O += P V once P is in TMEM, O has been rescaled and V has landed.
-          const int st = g % kStages;
-          const int pb = g % C::kPBufs;
-          if (!(ok = mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
-          if (!(ok = mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
-          if (!(ok = mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
-          tc_fence_after();
-          const uint64_t v_desc =
-              make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
-          if (PV4) {
-            // block scales of P (written by the softmax) and of V into tensor
-            // memory, then two K = 64 block-scaled MMAs with P from tensor memory
-            const uint32_t sb = (g & 1) * 8;
-#pragma unroll
-            for (int a = 0; a < 2; ++a) {
-              tmem_cp_32x128_warpx4(tmem + C::kColSFP + sb + 4 * a,
-                                    make_smem_desc(smem_u32(smem + C::kOffSFP + pb * C::kSFP + 512 * a), 128, 128, 0));
-              tmem_cp_32x128_warpx4(tmem + C::kColSFV + sb + 4 * a,
-                                    make_smem_desc(smem_u32(smem + C::kOffSFV + st * C::kSFV + 512 * a), 128, 128, 0));
-            }
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_nvf4_ts(tmem + C::kColO, tmem + C::kColP + pb * C::kPCols + 8 * kk, v_desc + 2 * kk, kIdescPV,
-                          tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
-                            v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(kv_empty + st);
-          mma_commit(o_done + st);
-          *consumed_cnt = g + 1;
-        }
-      }
-      // Drain: every issued MMA completes before tensor memory is released.
-      mma_commit(drain);
-      uint32_t drained = 0;
-      const unsigned long long t0 = globaltimer_ns();
-      while (!(drained = mbar_try_wait(smem_u32(drain), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-      }
-      if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------- S issuer
-    if (lane == 0) {
       constexpr uint32_t kIdescS = FP4 ? idesc_nvf4(128, 128) : idesc_e4m3(128, 128, false);
       const uint64_t q_desc = make_smem_desc(smem_u32(smem + C::kOffQ), 16, C::kQKSbo, C::kQKSwz);
-      int g = 0, it = 0;
-      bool ok = true;
-      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
-        int bh, qb;
-        decode_item(p, item, bh, qb);
-        const KList L = key_list(p, qb);
-        if (!(ok = mbar_wait(q_full, it & 1, abort_flag, &g_error_word, kErrQFull))) break;
+      // O += P V for block g (j-th block of its item) once P is in TMEM, O
+      // has been rescaled and V has landed.
+      auto issue_pv = [&](int g, int j) -> bool {
+        const int st = g % kStages;
+        const int pb = g % C::kPBufs;
+        if (!mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull)) return false;
+        if (!mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady)) return false;
+        if (!mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull)) return false;
+        tc_fence_after();
+        const uint64_t v_desc = make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
+        if (PV4) {
+          // block scales of P (written by the softmax) and of V into tensor
+          // memory, then two K = 64 block-scaled MMAs with P from tensor memory
+          const uint32_t sb = (g & 1) * 8;
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            tmem_cp_32x128_warpx4(tmem + C::kColSFP + sb + 4 * a,
+                                  make_smem_desc(smem_u32(smem + C::kOffSFP + pb * C::kSFP + 512 * a), 128, 128, 0));
+            tmem_cp_32x128_warpx4(tmem + C::kColSFV + sb + 4 * a,
+                                  make_smem_desc(smem_u32(smem + C::kOffSFV + st * C::kSFV + 512 * a), 128, 128, 0));
+          }
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_nvf4_ts(tmem + C::kColO, tmem + C::kColP + pb * C::kPCols + 8 * kk, v_desc + 2 * kk, kIdescPV,
+                        tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
+                          v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(kv_empty + st);
+        mma_commit(o_done + st);
+        *consumed_cnt = g + 1;
+        return true;
+      };
+      // S side: walks the same (item, key block) sequence. Q of an item is
+      // waited for before its first S; once its last S is issued, Q (and its
+      // scales) may be replaced. An item without key blocks still takes its
+      // Q phase.
+      int s_rnd = 0, s_it = 0, s_j = 0, s_g = 0, s_bh = 0, s_qb = 0;
+      int s_item = sched_item(0);
+      KList sL{0, 0};
+      if (s_item < p.num_items) {
+        decode_item(p, s_item, s_bh, s_qb);
+        sL = key_list(p, s_qb);
+      }
+      auto next_s_item = [&]() {
+        mma_commit(q_empty);  // all S of the item issued
+        ++s_it;
+        s_j = 0;
+        s_item = sched_item(++s_rnd);
+        if (s_item < p.num_items) {
+          decode_item(p, s_item, s_bh, s_qb);
+          sL = key_list(p, s_qb);
+        }
+      };
+      auto wait_q = [&]() -> bool {
+        if (!mbar_wait(q_full, s_it & 1, abort_flag, &g_error_word, kErrQFull)) return false;
         tc_fence_after();
         if (FP4) {
 #pragma unroll
@@ -560,43 +600,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tmem_cp_32x128_warpx4(tmem + C::kColSFQ + 4 * a,
                                   make_smem_desc(smem_u32(smem + C::kOffSFQ + 512 * a), 128, 128, 0));
         }
-        for (int j = 0; j < L.count; ++j, ++g) {
-          // S = Q K^T into buffer g % 2 once K has landed and the owner
-          // warpgroup has read the buffer's previous tile.
-          const int st = g % kStages;
-          const int buf = g & 1;
-          if (!(ok = mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
-          if (g >= 2 && !(ok = mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
-            break;
-          tc_fence_after();
-          const uint64_t k_desc =
-              make_smem_desc(smem_u32(smem + C::kOffK + st * C::kQKTile), 16, C::kQKSbo, C::kQKSwz);
-          const uint32_t s_tmem = tmem + buf * 128;
-          if (FP4) {
-            const uint32_t sfk = C::kColSFK + buf * C::kSFCols;
-#pragma unroll
-            for (int a = 0; a < D / 64; ++a)
-              tmem_cp_32x128_warpx4(tmem + sfk + 4 * a,
-                                    make_smem_desc(smem_u32(smem + C::kOffSFK + st * C::kSF + 512 * a), 128, 128, 0));
-#pragma unroll
-            for (int kk = 0; kk < C::kKSteps; ++kk)
-              mma_nvf4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, tmem + C::kColSFQ + 4 * kk,
-                          tmem + sfk + 4 * kk, kk > 0 ? 1u : 0u);
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < C::kKSteps; ++kk)
-              mma_f8f6f4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(s_full + buf);
-          mma_commit(kv_empty + st);
+        return true;
+      };
+      // Issues the next S of the sequence (none once it is exhausted).
+      auto issue_s = [&]() -> bool {
+        while (s_item < p.num_items && sL.count == 0) {
+          if (!wait_q()) return false;
+          next_s_item();
         }
-        if (!ok) break;
-        mma_commit(q_empty);  // all S of the item issued: Q (and its scales) may be replaced
+        if (s_item >= p.num_items) return true;
+        if (s_j == 0 && !wait_q()) return false;
+        // S = Q K^T into buffer g % 2 once K has landed and the softmax has
+        // read the buffer's previous tile.
+        const int g = s_g;
+        const int st = g % kStages;
+        const int buf = g & 1;
+        if (!mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull)) return false;
+        if (g >= 2 && !mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree))
+          return false;
+        tc_fence_after();
+        const uint64_t k_desc = make_smem_desc(smem_u32(smem + C::kOffK + st * C::kQKTile), 16, C::kQKSbo, C::kQKSwz);
+        const uint32_t s_tmem = tmem + buf * 128;
+        if (FP4) {
+          const uint32_t sfk = C::kColSFK + buf * C::kSFCols;
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a)
+            tmem_cp_32x128_warpx4(tmem + sfk + 4 * a,
+                                  make_smem_desc(smem_u32(smem + C::kOffSFK + st * C::kSF + 512 * a), 128, 128, 0));
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk)
+            mma_nvf4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, tmem + C::kColSFQ + 4 * kk,
+                        tmem + sfk + 4 * kk, kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk)
+            mma_f8f6f4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full + buf);
+        mma_commit(kv_empty + st);
+        ++s_g;
+        if (++s_j == sL.count) next_s_item();
+        return true;
+      };
+      bool ok = true;
+      if (kOneIssuer || warp == 1) {
+        if (kOneIssuer) ok = issue_s() && issue_s();
+        int g = 0;
+        for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
+          int bh, qb;
+          decode_item(p, item, bh, qb);
+          const KList L = key_list(p, qb);
+          for (int j = 0; j < L.count && ok; ++j, ++g) {
+            ok = issue_pv(g, j);
+            if (kOneIssuer && ok) ok = issue_s();
+          }
+        }
+      } else {
+        while (ok && s_item < p.num_items) ok = issue_s();
       }
-      mma_commit(drain + 1);
+      // Drain: every issued MMA completes before tensor memory is released.
+      uint64_t* dbar = drain + (warp == 1 ? 0 : 1);
+      mma_commit(dbar);
       uint32_t drained = 0;
       const unsigned long long t0 = globaltimer_ns();
-      while (!(drained = mbar_try_wait(smem_u32(drain + 1), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!(drained = mbar_try_wait(smem_u32(dbar), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
@@ -624,9 +691,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (FP4) c_fp4 = p.q_scale[0] * p.k_scale[0] * p.sm_scale_log2;
       else inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(bh) * p.nblk + qb];
       float l = 0.f, m_ref = -INFINITY;
+      // FP8 K scales are loaded one block ahead
+      float ks_next = (!FP4 && L.count > 0)
+                          ? __ldg(p.k_scale + static_cast<size_t>(bh) * p.nblk + max(key_block(p, L, 0), 0))
+                          : 1.f;
       for (int j = 0; j < L.count && ok; ++j, ++g) {
-        const int kb = key_block(p, L, j);
+        const int kb_raw = key_block(p, L, j);
+        const int kb = max(kb_raw, 0);
         const int buf = g & 1;
+        const float ks = ks_next;
+        if (!FP4 && j + 1 < L.count)
+          ks_next = __ldg(p.k_scale + static_cast<size_t>(bh) * p.nblk + max(key_block(p, L, j + 1), 0));
         // A failed wait raises the abort flag; the block then runs to its end
         // on whatever the buffers hold (every later wait returns at once) and
         // the loop stops after it.
@@ -643,9 +718,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         warp_arrive(s_free + buf);
         const int key0 = kb * 128 + 64 * w;
         const bool diag = p.causal && kb == qb;
-        if (diag || (kb + 1) * 128 > p.N) {
-          mask_chunk(r0, key0, qrow, diag, p.N);
-          mask_chunk(r1, key0 + 32, qrow, diag, p.N);
+        if (diag || (kb + 1) * 128 > p.N || kb_raw < 0) {
+          // an invalid mask entry masks every key of its block
+          const int lim = kb_raw < 0 ? 0 : p.N;
+          mask_chunk(r0, key0, qrow, diag, lim);
+          mask_chunk(r1, key0 + 32, qrow, diag, lim);
+        }
+        const float c = FP4 ? c_fp4 : inv_sq / ks;
+        const int pb = g % C::kPBufs;
+        if (C::kPWait && g >= C::kPBufs) {
+          // P buffer pb was last read by the PV of block g - kPBufs
+          const int gp = g - C::kPBufs;
+          ok = warp_wait(o_done + gp % kStages, (gp / kStages) & 1, abort_flag, &g_error_word, kErrPFree) && ok;
+          tc_fence_after();
+        }
+        // Speculation: once the row has a reference max, the exponentials are
+        // taken against it before this block's max is known, and taken again
+        // (below) only if the block moves the max of any row of the warp. A
+        // row whose max stays gets exactly the values of the plain order.
+        const bool spec = kSpeculate && !PV4 && __all_sync(0xffffffffu, m_ref != -INFINITY);
+        uint32_t pk0[8], pk1[8];
+        float psum = 0.f;
+        if (!PV4 && spec) {
+          const float nb = p.p_log2_scale - m_ref;
+          psum = exp_pack32<C::kPolyPairs>(r0, c, nb, pk0);
+          psum += exp_pack32<C::kPolyPairs>(r1, c, nb, pk1);
         }
         const float half_max = max32(r1, max32(r0, -INFINITY));
         // exchange the half maxima (tag g + 1; slots alternate by block parity)
@@ -656,7 +753,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                                      abort_flag, &g_error_word, kErrMax);
         ok = __all_sync(0xffffffffu, got) && ok;
         const float rawmax = w == 0 ? fmaxf(half_max, other_max) : fmaxf(other_max, half_max);
-        const float c = FP4 ? c_fp4 : inv_sq / p.k_scale[static_cast<size_t>(bh) * p.nblk + kb];
         // m_ref: reference max (-inf while every key so far is masked). It
         // moves to the running max only when that exceeds it by more than tau
         // (log2 units; tau = 0: the exact running max), and P then reaches at
@@ -680,26 +776,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // P = 2^(c s - m + log2 448) -> E4M3, this half's 16 columns of P
         // buffer g % kPBufs.
         const float nbias = p.p_log2_scale - m_use;
-        const int pb = g % C::kPBufs;
-        float psum;
         if (PV4) {
           // NVFP4 P: this half's 64 keys are one K = 64 step of the P V
           // product: 8 columns of E2M1 and 4 block scales, which go through
           // shared memory (in the tensor-core scale layout) to the PV issuer.
           const uint32_t p_addr = tmem + lane_off + C::kColP + pb * C::kPCols + 8 * w;
-          uint32_t pk0[4], pk1[4], sfw = 0u;
-          psum = exp_pack32_fp4<C::kPolyPairs>(r0, c, nbias, pk0, sfw, 0);
-          tmem_st4(p_addr, pk0);
-          psum += exp_pack32_fp4<C::kPolyPairs>(r1, c, nbias, pk1, sfw, 2);
-          tmem_st4(p_addr + 4, pk1);
+          uint32_t fq0[4], fq1[4], sfw = 0u;
+          psum = exp_pack32_fp4<C::kPolyPairs>(r0, c, nbias, fq0, sfw, 0);
+          tmem_st4(p_addr, fq0);
+          psum += exp_pack32_fp4<C::kPolyPairs>(r1, c, nbias, fq1, sfw, 2);
+          tmem_st4(p_addr + 4, fq1);
           reinterpret_cast<uint32_t*>(smem + C::kOffSFP + pb * C::kSFP + 512 * w)[(row & 31) * 4 + (row >> 5)] = sfw;
           fence_proxy_async_shared();
         } else {
           const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32 + 16 * w;
-          uint32_t pk0[8], pk1[8];
-          psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
+          if (!spec || __any_sync(0xffffffffu, m_new != m_prev)) {
+            psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
+            psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
+          }
           tmem_st8(p_addr, pk0);
-          psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
           tmem_st8(p_addr + 8, pk1);
         }
         l += psum;
@@ -942,16 +1037,6 @@ CUtensorMapSwizzle swizzle_for(int row_bytes) {
                           : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-int sm_count() {
-  static int n = [] {
-    int dev = 0, c = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
-    return c;
-  }();
-  return n;
-}
-
 // NVFP4 V, transposed: bytes [BH][D][nkb * 64] with box [1][D][64] (one
 // 128-key block of every channel), 64-byte swizzle.
 bool make_map_vt(CUtensorMap* m, const void* base, int D, int nkb, int BH) {
@@ -1002,17 +1087,25 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   p.num_items = BH * p.nblk;
   p.causal = a.causal ? 1 : 0;
   p.sparse = a.row_ptr ? 1 : 0;
+  p.nnz = a.nnz;
   p.sm_scale_log2 = a.softmax_scale * 1.4426950408889634f;
   p.tau = a.rescale_threshold;
   p.p_log2_scale = kLog2_448 - a.rescale_threshold;
-  static bool configured = false;
-  if (!configured) {
+  // The shared-memory opt-in is a per-device attribute of the kernel: set it
+  // once on each device this process launches on.
+  static std::atomic<unsigned long long> configured[(kMaxDevices + 63) / 64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  const unsigned long long bit = cacheable ? 1ull << (dev % 64) : 0ull;
+  if (!cacheable || !(configured[cacheable ? dev / 64 : 0].load(std::memory_order_acquire) & bit)) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, FP4, PV4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemRequest);
     if (e != cudaSuccess) return e;
-    configured = true;
+    if (cacheable) configured[dev / 64].fetch_or(bit, std::memory_order_acq_rel);
   }
-  const int grid = p.num_items < sm_count() ? p.num_items : sm_count();
+  const int sms = device_sm_count();
+  const int grid = p.num_items < sms ? p.num_items : sms;
   const cudaError_t e = launch_pdl(attn_fwd_kernel<D, FP4, PV4>, dim3(grid), dim3(kThreads), C::kSmemRequest, st, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

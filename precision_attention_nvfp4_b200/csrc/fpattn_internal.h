@@ -1,13 +1,39 @@
 // Internal host-side interfaces between the C ABI layer and the kernels.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "token_map.cuh"
 
+#ifndef FPATTN_MAX_DEVICES
+#define FPATTN_MAX_DEVICES 64
+#endif
+constexpr int kMaxDevices = FPATTN_MAX_DEVICES;
+
 namespace fpattn {
+
+// SM count of the current device, cached per device (a process may drive
+// several GPUs, one after another or from several threads).
+inline int device_sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= kMaxDevices) {
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+  }
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
 
 // tmap: NULL when x is already in the order the codes take; otherwise x is
 // read in raster order and the codes are written in tile-major order.
@@ -26,6 +52,13 @@ cudaError_t launch_quantize_fp8_channel(const void* x, int BH, int N, int d, uin
 cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const float* static_amax,
                                   uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
                                   const TokenMap* tmap, cudaStream_t st);
+
+// Q, K (NVFP4 when qk_fp4, else FP8 per 128-token tile) and V (FP8 per
+// channel) in four launches; results equal the separate launchers'.
+cudaError_t launch_quantize_qkv(const void* q, const void* k, const void* v, int BH, int N, int d, bool qk_fp4,
+                                uint8_t* q_codes, uint8_t* q_sf, float* q_scale, uint8_t* k_codes, uint8_t* k_sf,
+                                float* k_scale, uint8_t* v_codes, float* v_scales, int* nonfinite,
+                                const TokenMap* tmap, cudaStream_t st);
 
 // Video grid and tile of a tile-major token order.
 struct VideoLayout {
@@ -67,6 +100,7 @@ struct AttnArgs {
   const int32_t* row_ptr;  // tile mask CSR or null
   const int32_t* col_idx;
   const int32_t* row_order;
+  int nnz;  // entries of col_idx
   int B, H, N, d;
   bool qk_fp4;
   bool pv_fp4;  // P and V in NVFP4: v is transposed NVFP4 codes, v_scale its tensor scale

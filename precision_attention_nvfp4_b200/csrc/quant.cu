@@ -108,18 +108,16 @@ __device__ __forceinline__ uint2 quant8_e4m3(const uint4& v, float s) {
 // ---------------------------------------------------------------------------
 enum TileMode { kFused = 0, kAmaxOnly = 1, kConvert = 2 };
 
-template <int D, bool kMap, int kMode = kFused>
-__global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restrict__ x, int N,
-                                                            uint2* __restrict__ codes, float* __restrict__ scales,
-                                                            int* nonfinite, TokenMap tmap) {
-  griddep_wait();
+// Body of one CTA: tile `tile` of (b, h) = bh, ntiles tiles per (b, h).
+template <int D, bool kMap, int kMode>
+__device__ __forceinline__ void fp8_tile_body(const uint4* __restrict__ x, int N, uint2* __restrict__ codes,
+                                              float* __restrict__ scales, int* nonfinite, const TokenMap& tmap,
+                                              int tile, size_t bh, int ntiles) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int kChunks = 128 * kChunksPerRow;  // 16-byte chunks per full tile
   constexpr int kPer = kChunks / kThreads;
   __shared__ float red[kThreads / 32];
   __shared__ int src_row[kMap ? 128 : 1];
-  const int tile = blockIdx.x;
-  const size_t bh = blockIdx.y;
   const int rows = min(128, N - tile * 128);
   const size_t base = (bh * N + static_cast<size_t>(tile) * 128) * kChunksPerRow;
   if (kMap) {
@@ -139,22 +137,30 @@ __global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restr
   }
   float s;
   if (kMode == kConvert) {
-    s = scales[bh * gridDim.x + tile];
+    s = scales[bh * ntiles + tile];
   } else {
     if (bad && nonfinite) atomicExch(nonfinite, 1);
     const float a = block_max(m, red);
     if (kMode == kAmaxOnly) {
-      if (threadIdx.x == 0) scales[bh * gridDim.x + tile] = a;
+      if (threadIdx.x == 0) scales[bh * ntiles + tile] = a;
       return;
     }
     s = fp8_scale_from_amax(a);
-    if (threadIdx.x == 0) scales[bh * gridDim.x + tile] = s;
+    if (threadIdx.x == 0) scales[bh * ntiles + tile] = s;
   }
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int c = threadIdx.x + i * kThreads;
     if (c / kChunksPerRow < rows) codes[base + c] = quant8_e4m3(v[i], s);
   }
+}
+
+template <int D, bool kMap, int kMode = kFused>
+__global__ void __launch_bounds__(kThreads) fp8_tile_kernel(const uint4* __restrict__ x, int N,
+                                                            uint2* __restrict__ codes, float* __restrict__ scales,
+                                                            int* nonfinite, TokenMap tmap) {
+  griddep_wait();
+  fp8_tile_body<D, kMap, kMode>(x, N, codes, scales, nonfinite, tmap, blockIdx.x, blockIdx.y, gridDim.x);
   griddep_launch_dependents();
 }
 
@@ -185,15 +191,14 @@ __global__ void fp8_group_finalize_kernel(float* __restrict__ scales, int nblk, 
 // ---------------------------------------------------------------------------
 constexpr int kRowsPerCta = 256;
 
+// Body of one CTA: rows [256 bx, 256 bx + 256) of (b, h) = bh.
 template <int D>
-__global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4* __restrict__ x, int N,
-                                                                    float* __restrict__ amax, int* nonfinite) {
-  griddep_wait();
+__device__ __forceinline__ void fp8_channel_amax_body(const uint4* __restrict__ x, int N, float* __restrict__ amax,
+                                                      int* nonfinite, int bx, size_t bh) {
   constexpr int kCpr = D / 8;                 // chunks per row
   constexpr int kRowsPerIter = kThreads / kCpr;
   __shared__ float part[kRowsPerIter][D];
-  const size_t bh = blockIdx.y;
-  const int r0 = blockIdx.x * kRowsPerCta;
+  const int r0 = bx * kRowsPerCta;
   const int cg = threadIdx.x % kCpr;          // channel group of 8
   const int rr = threadIdx.x / kCpr;
   float m[8];
@@ -223,22 +228,27 @@ __global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4*
     for (int j = 0; j < kRowsPerIter; ++j) a = fmaxf(a, part[j][c]);
     atomicMax(reinterpret_cast<int*>(amax) + bh * D + c, __float_as_int(a));
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) fp8_channel_amax_kernel(const uint4* __restrict__ x, int N,
+                                                                    float* __restrict__ amax, int* nonfinite) {
+  griddep_wait();
+  fp8_channel_amax_body<D>(x, N, amax, nonfinite, blockIdx.x, blockIdx.y);
   griddep_launch_dependents();
 }
 
 // The amax pass is order-free, so only the conversion pass reads through the
 // token map (output row r, tile-major, from source row to_raster(r)).
 template <int D, bool kMap>
-__global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4* __restrict__ x, int N,
-                                                                     const float* __restrict__ amax,
-                                                                     uint2* __restrict__ codes, TokenMap tmap) {
-  griddep_wait();
+__device__ __forceinline__ void fp8_channel_quant_body(const uint4* __restrict__ x, int N,
+                                                       const float* __restrict__ amax, uint2* __restrict__ codes,
+                                                       const TokenMap& tmap, int bx, size_t bh) {
   constexpr int kCpr = D / 8;
   constexpr int kRowsPerIter = kThreads / kCpr;
   static_assert(kRowsPerCta == kThreads, "one source-row lookup per thread");
   __shared__ int src_row[kMap ? kRowsPerCta : 1];
-  const size_t bh = blockIdx.y;
-  const int r0 = blockIdx.x * kRowsPerCta;
+  const int r0 = bx * kRowsPerCta;
   const int cg = threadIdx.x % kCpr;
   const int rr = threadIdx.x / kCpr;
   const int rend = min(N, r0 + kRowsPerCta);
@@ -261,6 +271,14 @@ __global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4
           (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[6], s[6]), __fmul_rn(f[7], s[7]))) << 16);
     codes[idx] = o;
   }
+}
+
+template <int D, bool kMap>
+__global__ void __launch_bounds__(kThreads) fp8_channel_quant_kernel(const uint4* __restrict__ x, int N,
+                                                                     const float* __restrict__ amax,
+                                                                     uint2* __restrict__ codes, TokenMap tmap) {
+  griddep_wait();
+  fp8_channel_quant_body<D, kMap>(x, N, amax, codes, tmap, blockIdx.x, blockIdx.y);
   griddep_launch_dependents();
 }
 
@@ -282,14 +300,16 @@ __global__ void fp8_channel_finalize_kernel(float* __restrict__ s, int n) {
 //   (zero for the rows that pad N up to 128).
 // Pass 3: *tensor_scale = s_t.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __restrict__ x, size_t nchunks,
-                                                               float* __restrict__ amax_out, int* nonfinite) {
-  griddep_wait();
+// Body of CTA `block` of `nblocks` reducing |x| over nchunks 16-byte chunks
+// (grid-stride) into *amax_out.
+__device__ __forceinline__ void tensor_amax_body(const uint4* __restrict__ x, size_t nchunks,
+                                                 float* __restrict__ amax_out, int* nonfinite, int block,
+                                                 int nblocks) {
   __shared__ float red[kThreads / 32];
   float m = 0.f;
   bool bad = false;
-  const size_t stride = static_cast<size_t>(gridDim.x) * kThreads;
-  size_t c = blockIdx.x * static_cast<size_t>(kThreads) + threadIdx.x;
+  const size_t stride = static_cast<size_t>(nblocks) * kThreads;
+  size_t c = block * static_cast<size_t>(kThreads) + threadIdx.x;
   // four loads in flight per thread
   for (; c + 3 * stride < nchunks; c += 4 * stride) {
     const uint4 v0 = x[c], v1 = x[c + stride], v2 = x[c + 2 * stride], v3 = x[c + 3 * stride];
@@ -299,6 +319,12 @@ __global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __re
   if (bad && nonfinite) atomicExch(nonfinite, 1);
   m = block_max(m, red);
   if (threadIdx.x == 0) atomicMax(reinterpret_cast<int*>(amax_out), __float_as_int(m));
+}
+
+__global__ void __launch_bounds__(kThreads) tensor_amax_kernel(const uint4* __restrict__ x, size_t nchunks,
+                                                               float* __restrict__ amax_out, int* nonfinite) {
+  griddep_wait();
+  tensor_amax_body(x, nchunks, amax_out, nonfinite, blockIdx.x, gridDim.x);
   griddep_launch_dependents();
 }
 
@@ -315,17 +341,14 @@ __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
 // grid = (nblk * 128 / kRowsPerCta, B*H): rows are padded to 128 per (b, h),
 // and the padding rows only write zero scales.
 template <int D, bool kMap>
-__global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __restrict__ x, int N, int nblk,
-                                                               const float* __restrict__ amax_ptr,
-                                                               uint32_t* __restrict__ codes,
-                                                               uint8_t* __restrict__ sf, TokenMap tmap) {
-  griddep_wait();
+__device__ __forceinline__ void nvfp4_quant_body(const uint4* __restrict__ x, int N, int nblk,
+                                                 const float* __restrict__ amax_ptr, uint32_t* __restrict__ codes,
+                                                 uint8_t* __restrict__ sf, const TokenMap& tmap, int bx, int bh) {
   constexpr int kCpr = D / 8;                // 16-byte chunks per row
   constexpr int kRowsPerWarp = 128 / kCpr;   // 8 or 16
   constexpr int kGroups = D / 64;            // 512-byte scale groups per 128-row block
-  const int bh = blockIdx.y;
   const int lane = threadIdx.x & 31;
-  const int r0 = (blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp;
+  const int r0 = (bx * (kThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp;
   int src = 0;
   if (kMap && lane < kRowsPerWarp && r0 + lane < N) src = to_raster(tmap, r0 + lane);
   uint4 v[4];
@@ -366,6 +389,15 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __re
       sf[byte] = r < N ? static_cast<uint8_t>(sb) : 0u;
     }
   }
+}
+
+template <int D, bool kMap>
+__global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const uint4* __restrict__ x, int N, int nblk,
+                                                               const float* __restrict__ amax_ptr,
+                                                               uint32_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ sf, TokenMap tmap) {
+  griddep_wait();
+  nvfp4_quant_body<D, kMap>(x, N, nblk, amax_ptr, codes, sf, tmap, blockIdx.x, blockIdx.y);
   griddep_launch_dependents();
 }
 
@@ -445,6 +477,105 @@ __global__ void __launch_bounds__(D) nvfp4_tokens_quant_kernel(const uint32_t* _
   griddep_launch_dependents();
 }
 
+// ---------------------------------------------------------------------------
+// Q, K and V of one attention call in four launches: zero the accumulators,
+// one amax pass over all three tensors, one conversion pass, one finalize.
+// Each CTA runs the body of the stand-alone kernel for its share (the block
+// index picks the tensor), so the codes and scales are those of the separate
+// calls, bit for bit. With FP8 Q/K the per-tile quantization is one pass and
+// runs in the amax launch.
+// ---------------------------------------------------------------------------
+struct QkvParams {
+  const uint4* q;
+  const uint4* k;
+  const uint4* v;
+  int N, BH, nblk;
+  void* q_codes;       // NVFP4: packed E2M1 words; FP8: E4M3 bytes
+  void* k_codes;
+  uint8_t* q_sf;       // NVFP4 block scales (tensor-core layout)
+  uint8_t* k_sf;
+  float* q_scale;      // NVFP4: amax accumulator, then s_t; FP8: per-tile scales
+  float* k_scale;
+  uint2* v_codes;
+  float* v_scales;     // amax accumulators, then per-channel scales
+  int* nonfinite;
+  TokenMap tmap;
+  int amax_ctas;       // NVFP4: CTAs per tensor in the tensor-amax share
+  int vgx;             // channel passes: CTAs per (b, h) (256 rows each)
+  int qgx;             // NVFP4 conversion: CTAs per (b, h)
+};
+
+template <int D, bool kMap, bool kFp4>
+__global__ void __launch_bounds__(kThreads) qkv_amax_kernel(const __grid_constant__ QkvParams p) {
+  griddep_wait();
+  int b = blockIdx.x;
+  const int nqk = kFp4 ? p.amax_ctas : p.nblk * p.BH;  // CTAs of the Q share (and of the K share)
+  if (b < 2 * nqk) {
+    const bool isq = b < nqk;
+    const int bb = isq ? b : b - nqk;
+    if (kFp4) {
+      tensor_amax_body(isq ? p.q : p.k, static_cast<size_t>(p.BH) * p.N * (D / 8), isq ? p.q_scale : p.k_scale,
+                       p.nonfinite, bb, nqk);
+    } else {
+      fp8_tile_body<D, kMap, kFused>(isq ? p.q : p.k, p.N, static_cast<uint2*>(isq ? p.q_codes : p.k_codes),
+                                     isq ? p.q_scale : p.k_scale, p.nonfinite, p.tmap, bb % p.nblk, bb / p.nblk,
+                                     p.nblk);
+    }
+  } else {
+    b -= 2 * nqk;
+    fp8_channel_amax_body<D>(p.v, p.N, p.v_scales, p.nonfinite, b % p.vgx, b / p.vgx);
+  }
+  griddep_launch_dependents();
+}
+
+// V first, then K, then Q: the reverse of the amax pass, whose last reads are
+// the likeliest to be still in L2.
+template <int D, bool kMap, bool kFp4>
+__global__ void __launch_bounds__(kThreads) qkv_convert_kernel(const __grid_constant__ QkvParams p) {
+  griddep_wait();
+  int b = blockIdx.x;
+  const int nv = p.vgx * p.BH;
+  if (b < nv) {
+    fp8_channel_quant_body<D, kMap>(p.v, p.N, p.v_scales, p.v_codes, p.tmap, b % p.vgx, b / p.vgx);
+  } else if (kFp4) {
+    b -= nv;
+    const int nq = p.qgx * p.BH;
+    const bool isk = b < nq;
+    const int bb = isk ? b : b - nq;
+    nvfp4_quant_body<D, kMap>(isk ? p.k : p.q, p.N, p.nblk, isk ? p.k_scale : p.q_scale,
+                              static_cast<uint32_t*>(isk ? p.k_codes : p.q_codes), isk ? p.k_sf : p.q_sf, p.tmap,
+                              bb % p.qgx, bb / p.qgx);
+  }
+  griddep_launch_dependents();
+}
+
+// amax -> scale in place: s_t = A/2688 for NVFP4 Q and K (thread 0), 448/A
+// per V channel.
+template <bool kFp4>
+__global__ void qkv_finalize_kernel(float* __restrict__ q_scale, float* __restrict__ k_scale,
+                                    float* __restrict__ v_scales, int nv) {
+  griddep_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (kFp4 && i == 0) {
+    *q_scale = nvfp4_tensor_scale(*q_scale);
+    *k_scale = nvfp4_tensor_scale(*k_scale);
+  }
+  if (i < nv) v_scales[i] = fp8_scale_from_amax(v_scales[i]);
+  griddep_launch_dependents();
+}
+
+// Zeroes the accumulators of qkv_amax_kernel: a[0..na), b[0..nb), c[0..nc).
+__global__ void zero3_kernel(float* __restrict__ a, int na, float* __restrict__ b, int nb, float* __restrict__ c,
+                             int nc) {
+  griddep_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < na + nb + nc; i += gridDim.x * blockDim.x) {
+    if (i < na) a[i] = 0.f;
+    else if (i < na + nb) b[i - na] = 0.f;
+    else c[i - na - nb] = 0.f;
+  }
+  griddep_launch_dependents();
+}
+
 // Zeroes n floats (the amax accumulators), as a kernel so that it takes
 // part in the programmatic launch chain like every other step.
 __global__ void zero_kernel(float* __restrict__ p, int n) {
@@ -459,15 +590,7 @@ __global__ void nvfp4_finalize_kernel(const float* __restrict__ amax_ptr, float*
   griddep_launch_dependents();
 }
 
-inline int num_sms() {
-  static int sms = [] {
-    int dev = 0, n = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-  }();
-  return sms;
-}
+inline int num_sms() { return device_sm_count(); }
 
 }  // namespace
 
@@ -580,6 +703,58 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
   launch_pdl(kern, dim3(nblk * 128 / rows_per_cta, BH), dim3(kThreads), 0, st, static_cast<const uint4*>(x), N,
              nblk, amax_ptr, reinterpret_cast<uint32_t*>(codes), block_sf, tmap ? *tmap : TokenMap{});
   launch_pdl(nvfp4_finalize_kernel, dim3(1), dim3(32), 0, st, amax_ptr, tensor_scale);
+  return cudaGetLastError();
+}
+
+namespace {
+
+template <int D, bool kMap, bool kFp4>
+void launch_qkv(const QkvParams& p, cudaStream_t st) {
+  const int nv = p.BH * D;
+  launch_pdl(zero3_kernel, dim3((2 + nv + 255) / 256), dim3(256), 0, st, kFp4 ? p.q_scale : nullptr,
+             kFp4 ? 1 : 0, kFp4 ? p.k_scale : nullptr, kFp4 ? 1 : 0, p.v_scales, nv);
+  const int nqk = kFp4 ? p.amax_ctas : p.nblk * p.BH;
+  launch_pdl(qkv_amax_kernel<D, kMap, kFp4>, dim3(2 * nqk + p.vgx * p.BH), dim3(kThreads), 0, st, p);
+  launch_pdl(qkv_convert_kernel<D, kMap, kFp4>, dim3(p.vgx * p.BH + (kFp4 ? 2 * p.qgx * p.BH : 0)),
+             dim3(kThreads), 0, st, p);
+  launch_pdl(qkv_finalize_kernel<kFp4>, dim3((nv + 255) / 256), dim3(256), 0, st, p.q_scale, p.k_scale,
+             p.v_scales, nv);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_qkv(const void* q, const void* k, const void* v, int BH, int N, int d, bool qk_fp4,
+                                uint8_t* q_codes, uint8_t* q_sf, float* q_scale, uint8_t* k_codes, uint8_t* k_sf,
+                                float* k_scale, uint8_t* v_codes, float* v_scales, int* nonfinite,
+                                const TokenMap* tmap, cudaStream_t st) {
+  QkvParams p{};
+  p.q = static_cast<const uint4*>(q);
+  p.k = static_cast<const uint4*>(k);
+  p.v = static_cast<const uint4*>(v);
+  p.N = N;
+  p.BH = BH;
+  p.nblk = (N + 127) / 128;
+  p.q_codes = q_codes;
+  p.k_codes = k_codes;
+  p.q_sf = q_sf;
+  p.k_sf = k_sf;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_codes = reinterpret_cast<uint2*>(v_codes);
+  p.v_scales = v_scales;
+  p.nonfinite = nonfinite;
+  p.tmap = tmap ? *tmap : TokenMap{};
+  p.amax_ctas = num_sms() * 4;
+  p.vgx = (N + kRowsPerCta - 1) / kRowsPerCta;
+  p.qgx = p.nblk * 128 / ((kThreads / 32) * (128 / (d / 8)));
+  const bool map = tmap != nullptr;
+  if (d == 128) {
+    if (qk_fp4) map ? launch_qkv<128, true, true>(p, st) : launch_qkv<128, false, true>(p, st);
+    else map ? launch_qkv<128, true, false>(p, st) : launch_qkv<128, false, false>(p, st);
+  } else {
+    if (qk_fp4) map ? launch_qkv<64, true, true>(p, st) : launch_qkv<64, false, true>(p, st);
+    else map ? launch_qkv<64, true, false>(p, st) : launch_qkv<64, false, false>(p, st);
+  }
   return cudaGetLastError();
 }
 

@@ -269,3 +269,73 @@ def test_nvfp4_v_sizes_and_argument_errors(lib):
     sc_bad = _lib.Scales(p16, p16, p16, None, None, 1.0 / 448.0, 0.0, 0.0, p16 + 4)
     assert lib.fpattn_fwd(ctypes.byref(q), ctypes.byref(q), ctypes.byref(v4), ctypes.byref(sc_bad), None, 0, p16,
                           None, None) == _lib.ERR_ALIGNMENT
+
+
+def _mask_status(lib, row_ptr, col_idx, row_order=None, nblk=None):
+    rp = np.asarray(row_ptr, dtype=np.int32)
+    ci = np.asarray(col_idx, dtype=np.int32)
+    ro = None if row_order is None else np.asarray(row_order, dtype=np.int32)
+    n = len(rp) - 1 if nblk is None else nblk
+    return lib.fpattn_tile_mask_check(n, len(ci), rp.ctypes.data, ci.ctypes.data if len(ci) else None,
+                                      None if ro is None else ro.ctypes.data)
+
+
+def test_tile_mask_check_accepts_wellformed(lib):
+    assert _mask_status(lib, [0, 2, 2, 3], [0, 2, 1], [0, 2, 1]) == _lib.OK
+    assert _mask_status(lib, [0, 2, 2, 3], [0, 2, 1]) == _lib.OK        # row_order optional
+    plan = fp.sta_plan((3, 6, 10), (6, 8, 8), (3, 3, 5))
+    assert _mask_status(lib, plan.row_ptr, plan.col_idx, plan.row_order) == _lib.OK
+
+
+@pytest.mark.parametrize("row_ptr,col_idx,row_order", [
+    ([0, 2, 2, 3], [0, 3, 1], None),          # key block 3 >= nblk
+    ([0, 2, 2, 3], [0, -1, 1], None),         # negative key block
+    ([0, 2, 2, 3], [2, 0, 1], None),          # not ascending within a row
+    ([0, 2, 2, 3], [1, 1, 1], None),          # repeated entry
+    ([0, 2, 1, 3], [0, 2, 1], None),          # row_ptr decreasing
+    ([1, 2, 2, 3], [0, 2, 1], None),          # row_ptr[0] != 0
+    ([0, 2, 2, 4], [0, 2, 1], None),          # row_ptr[nblk] != nnz
+    ([0, 2, 2, 3], [0, 2, 1], [0, 0, 1]),     # row_order not a permutation
+    ([0, 2, 2, 3], [0, 2, 1], [0, 1, 3]),     # row_order out of range
+])
+def test_tile_mask_check_rejects_malformed(lib, row_ptr, col_idx, row_order):
+    assert _mask_status(lib, row_ptr, col_idx, row_order) == _lib.ERR_INVALID_ARG
+    # the Python mask refuses it before anything reaches a device
+    with pytest.raises(fp.FpattnError):
+        fp.StaPlan(np.asarray(row_ptr, np.int32), np.asarray(col_idx, np.int32),
+                   None if row_order is None else np.asarray(row_order, np.int32)).to("cpu")
+
+
+def test_attention_fwd_refuses_mismatched_operands():
+    """Operands the kernel would read past are refused in Python, before any
+    launch: shapes that differ, FP8 granularities swapped, q/k formats mixed,
+    buffers too small for the shape."""
+    import torch
+    B, H, N, d = 1, 2, 256, 128
+
+    def nv(n=N, h=H):
+        return fp.Nvfp4Tensor(torch.zeros(B, h, n, d // 2, dtype=torch.uint8),
+                              torch.zeros(B * h * ((n + 127) // 128) * 2 * 512, dtype=torch.uint8),
+                              torch.zeros(1), (B, h, n, d))
+
+    def f8(gran, n=N):
+        sc = torch.zeros(B, H, (n + 127) // 128) if gran == "tile128" else torch.zeros(B, H, d)
+        return fp.Fp8Tensor(torch.zeros(B, H, n, d, dtype=torch.uint8), sc, gran, (B, H, n, d))
+
+    with pytest.raises(ValueError, match="shapes differ"):
+        fp.attention_fwd(nv(), nv(n=128), f8("channel"))
+    with pytest.raises(ValueError, match="shapes differ"):
+        fp.attention_fwd(nv(h=1), nv(h=1), f8("channel"))
+    with pytest.raises(ValueError, match="per-channel"):
+        fp.attention_fwd(nv(), nv(), f8("tile128"))
+    with pytest.raises(ValueError, match="per-tile"):
+        fp.attention_fwd(f8("channel"), f8("channel"), f8("channel"))
+    with pytest.raises(TypeError):
+        fp.attention_fwd(nv(), f8("tile128"), f8("channel"))
+    short = nv()
+    short.block_sf = short.block_sf[:100]
+    with pytest.raises(ValueError):
+        fp.attention_fwd(short, nv(), f8("channel"))
+    # CPU buffers never reach the library
+    with pytest.raises(ValueError, match="contiguous tensor on"):
+        fp.attention_fwd(nv(), nv(), f8("channel"))

@@ -165,3 +165,67 @@ def test_workload_fp8_heads(name):
     sub = slice(0, 3)
     _check_fp8(q[:, sub].contiguous(), "tile128")
     _check_fp8(v[:, sub].contiguous(), "channel")
+
+
+# ---------------------------------------------- Q, K, V in four fused launches
+def _same_bits(a: torch.Tensor, b: torch.Tensor, what: str):
+    a, b = a.contiguous().view(torch.uint8).cpu(), b.contiguous().view(torch.uint8).cpu()
+    n = int((a != b).sum())
+    assert a.shape == b.shape and n == 0, f"{what}: {n} bytes differ"
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "fp8"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [128, 300, 1000])
+def test_quantize_qkv_equals_separate_calls(fmt, d, N):
+    """quantize_qkv (zero, one amax pass over Q, K and V, one conversion pass,
+    one finalize) gives bit for bit the codes and scales of the per-tensor
+    calls, which the tests above pin to the oracle."""
+    q = _rand((2, 3, N, d), 40 + N + d, outliers=True).cuda()
+    k = _rand((2, 3, N, d), 41 + N + d, scale=3.0).cuda()
+    v = _rand((2, 3, N, d), 42 + N + d, scale=0.5, outliers=True).cuda()
+    qq, kq, vq = fp.quantize_qkv(q, k, v, fmt)
+    if fmt == "nvfp4":
+        for got, ref in ((qq, fp.quantize_nvfp4(q)), (kq, fp.quantize_nvfp4(k))):
+            _same_bits(got.codes, ref.codes, "codes")
+            _same_bits(got.block_sf, ref.block_sf, "block scales")
+            _same_bits(got.tensor_scale, ref.tensor_scale, "tensor scale")
+    else:
+        for got, ref in ((qq, fp.quantize_fp8(q, "tile128")), (kq, fp.quantize_fp8(k, "tile128"))):
+            _same_bits(got.codes, ref.codes, "codes")
+            _same_bits(got.scales, ref.scales, "tile scales")
+    ref = fp.quantize_fp8(v, "channel")
+    _same_bits(vq.codes, ref.codes, "V codes")
+    _same_bits(vq.scales, ref.scales, "V channel scales")
+    torch.cuda.synchronize()
+
+
+def test_quantize_qkv_against_oracle_and_video_order():
+    """The fused call against the oracle directly (NVFP4 Q, FP8 V), and with a
+    raster-order video layout against the separate _video calls."""
+    x = _rand((1, 2, 300, 128), 77, outliers=True)
+    qq, _, vq = fp.quantize_qkv(x.cuda(), x.cuda(), x.cuda(), "nvfp4")
+    torch.cuda.synchronize()
+    codes, sb, s_t = quant.quantize_nvfp4(_f32(x))
+    assert qq.tensor_scale.cpu().numpy().view(np.uint32)[0] == np.float32(s_t).view(np.uint32)
+    assert np.array_equal(qq.codes.cpu().numpy(), codec.pack_e2m1(codes))
+    assert np.array_equal(qq.block_sf.cpu().numpy(), quant.nvfp4_sf_swizzle(sb.reshape(2, 300, 8), 300, 128).reshape(-1))
+    vc, vs = quant.quantize_fp8_channel(_f32(x))
+    assert np.array_equal(vq.codes.cpu().numpy(), vc)
+    assert np.array_equal(vq.scales.cpu().numpy().view(np.uint32), vs.view(np.uint32))
+    grid, tile = (4, 16, 16), (2, 8, 8)
+    video = fp.VideoLayout(grid, tile)
+    xs = [_rand((1, 2, 1024, 64), 80 + i, outliers=(i == 0)).cuda() for i in range(3)]
+    for fmt in ("nvfp4", "fp8"):
+        qq, kq, vq = fp.quantize_qkv(*xs, fmt, video=video)
+        if fmt == "nvfp4":
+            rq = fp.quantize_nvfp4(xs[0], video=video)
+            _same_bits(qq.codes, rq.codes, "video codes")
+            _same_bits(qq.block_sf, rq.block_sf, "video scales")
+        else:
+            rq = fp.quantize_fp8(xs[1], "tile128", video=video)
+            _same_bits(kq.codes, rq.codes, "video codes")
+            _same_bits(kq.scales, rq.scales, "video tile scales")
+        rv = fp.quantize_fp8(xs[2], "channel", video=video)
+        _same_bits(vq.codes, rv.codes, "video V codes")
+        _same_bits(vq.scales, rv.scales, "video V scales")
