@@ -520,11 +520,16 @@ def main():
     ms_step = ms_total / args.steps
     value = aggregate_value(flops, world, ms_step)
     peaks, peak_src = load_peaks()
-    # A kernel timed inside a seconds-long loop runs under the power cap for
-    # most of it: the sustained bf16 figure applies. A shorter timed region
-    # is a burst.
+    # The sustained bf16 figure was measured under the power cap at a lowered
+    # SM clock; it applies to a seconds-long timed region that itself ran
+    # capped or below the maximum clock. A short region, or one whose clock
+    # record shows the maximum clock and no power cap, takes the burst figure
+    # (measured at the maximum clock).
     timed_s = ms_total * 1e-3
-    sustained = timed_s >= 1.0 and "bf16_tflops_sustained" in peaks
+    capped = ("sw_power_cap" in clk.get("reasons", []) or
+              (clk.get("sm_mhz") is not None and clk.get("sm_max_mhz") and
+               clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"]))
+    sustained = timed_s >= 1.0 and capped and "bf16_tflops_sustained" in peaks
     bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
     # both MMAs do 2d flops per score: the peak is the harmonic mean of theirs
@@ -622,9 +627,11 @@ def main():
                          "frac": attn_tflops / peak, "frac_of_burst_peak": attn_tflops / peak_burst,
                          "traffic": profiled_traffic(w.name) if args.pv_format == "fp8" and
                          not args.rescale_threshold else None,
+                         "frac_of_sustained_peak": attn_tflops / (peak * peaks.get("bf16_tflops_sustained", bf16) / bf16),
                          "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} {bf16} "
-                                        f"(timed region {timed_s:.2f} s: "
-                                        f"{'>= 1 s, under the power cap' if sustained else '< 1 s, a burst'}) "
+                                        f"(timed region {timed_s:.2f} s, median SM clock {clk.get('sm_mhz')} MHz, "
+                                        f"{'power-capped or below max clock' if capped else 'max clock, no power cap'})"
+                                        f" "
                                         f"x nominal fp8 2x / fp4 4x; QK "
                                         f"{'fp4' if w.qk_format == 'nvfp4' else 'fp8'}, PV "
                                         f"{'fp4' if args.pv_format == 'nvfp4' else 'fp8'}, harmonic mean"},

@@ -113,6 +113,20 @@ fpattn_status fpattn_quantize_nvfp4(const fpattn_tensor* x, const float* static_
                                     int32_t* nonfinite_flag, fpattn_stream_t stream);
 
 /*
+ * The amax pass of fpattn_quantize_nvfp4 on its own (Blackwell FP4 practice
+ * page, section 1: the tensor scale comes from the largest magnitude): folds
+ * max|x| over the bf16 tensor x into the device float *amax, which is zeroed
+ * first unless accumulate != 0. Several calls on consecutive pieces of one
+ * tensor, the first with accumulate = 0 and the rest in stream order with
+ * accumulate = 1, leave the amax of the whole tensor; passed as static_amax
+ * to fpattn_quantize_nvfp4 on each piece it gives the codes and scales of
+ * the whole-tensor call (the tensor is quantized as its pieces arrive).
+ * nonfinite_flag as in fpattn_quantize_nvfp4. Errors as there.
+ */
+fpattn_status fpattn_tensor_amax(const fpattn_tensor* x, int32_t accumulate, float* amax, int32_t* nonfinite_flag,
+                                 fpattn_stream_t stream);
+
+/*
  * FP8 E4M3 quantization of a bf16 tensor (FPSAttention page, section 2.1:
  * X_hat = dequantize(FP8_convert(X * s_g)) / s_g; section 3.1: Q/K per block,
  * V per channel).

@@ -42,7 +42,7 @@ from ._lib import FpattnError
 __all__ = ["Nvfp4Tensor", "Nvfp4VTensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_qkv",
            "quantize_nvfp4_v", "quantize_fp8", "sta_plan",
            "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError",
-           "head_range"]
+           "head_range", "tensor_amax"]
 
 
 def library() -> ctypes.CDLL:
@@ -126,6 +126,20 @@ def quantize_nvfp4(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
                                              sf.data_ptr(), ts.data_ptr(), _ptr(nonfinite_flag), _stream())
     _lib.check(st, "fpattn_quantize_nvfp4" + ("_video" if video is not None else ""))
     return Nvfp4Tensor(codes, sf, ts, (B, H, N, d))
+
+
+def tensor_amax(x: torch.Tensor, out: Optional[torch.Tensor] = None, accumulate: bool = False,
+                nonfinite_flag: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """max|x| of a bf16 tensor folded into ``out`` (a device float32 [1],
+    zeroed first unless ``accumulate``): the amax pass of quantize_nvfp4, for
+    a tensor that arrives in pieces."""
+    B, H, N, d = _check_bf16(x)
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    st = library().fpattn_tensor_amax(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), 1 if accumulate else 0,
+                                      out.data_ptr(), _ptr(nonfinite_flag), _stream())
+    _lib.check(st, "fpattn_tensor_amax")
+    return out
 
 
 def quantize_nvfp4_v(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
@@ -389,16 +403,22 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
     NVFP4 and runs P V on the block-scaled FP4 tensor cores.
 
     CUDA inputs stay where they are. Host inputs (ideally pinned) are copied
-    to ``device`` (default cuda:0) on the current stream, and the output (and
-    lse) are copied back to host memory: into ``out_host`` / ``lse_host`` when
-    given (pinned buffers the caller reuses), else into new pinned tensors.
+    to ``device`` (default cuda:0) and the output (and lse) copied back to
+    host memory, into ``out_host`` / ``lse_host`` when given (pinned buffers
+    the caller reuses), else into new pinned tensors; the copies of one group
+    of heads overlap the kernels of another (see _attention_host), and the
+    call returns once the results are in host memory.
     """
-    host = not q.is_cuda
-    if host:
-        dev = torch.device(device or "cuda:0")
-        q = q.to(dev, non_blocking=True)
-        k = k.to(dev, non_blocking=True)
-        v = v.to(dev, non_blocking=True)
+    if qk_format not in ("nvfp4", "fp8"):
+        raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
+    if pv_format not in ("fp8", "nvfp4"):
+        raise ValueError("pv_format must be 'fp8' or 'nvfp4'")
+    if not q.is_cuda:
+        return _attention_host(q, k, v, qk_format=qk_format, causal=causal, tile_mask=tile_mask,
+                               softmax_scale=softmax_scale, return_lse=return_lse, device=device,
+                               out_host=out_host, lse_host=lse_host, video=video,
+                               rescale_threshold=rescale_threshold, qk_group_tiles=qk_group_tiles,
+                               pv_format=pv_format)
     if qk_format not in ("nvfp4", "fp8"):
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
     if pv_format not in ("fp8", "nvfp4"):
@@ -413,19 +433,104 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
             qq = quantize_fp8(q, gran, video=video, group_tiles=qk_group_tiles)
             kq = quantize_fp8(k, gran, video=video, group_tiles=qk_group_tiles)
         vq = quantize_fp8(v, "channel", video=video) if pv_format == "fp8" else quantize_nvfp4_v(v, video=video)
-    out, lse = attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
-                             return_lse=return_lse, video=video, rescale_threshold=rescale_threshold)
-    if host:
-        out_h = out_host if out_host is not None else torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        out_h.copy_(out, non_blocking=True)
-        lse_h = None
-        if lse is not None:
-            lse_h = lse_host if lse_host is not None else torch.empty(lse.shape, dtype=lse.dtype,
-                                                                      pin_memory=True)
-            lse_h.copy_(lse, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        return out_h, lse_h
-    return out, lse
+    return attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
+                         return_lse=return_lse, video=video, rescale_threshold=rescale_threshold)
+
+
+def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, return_lse, device, out_host,
+                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: int = 4):
+    """attention() for host inputs: the (batch, head) problems are split into
+    ``chunks`` contiguous groups, and the copies in, the kernels and the
+    copies out of different groups overlap on three streams. Q and K are
+    copied first: an NVFP4 tensor scale needs the amax over every head, so
+    their amax pass runs as each group lands, and each group is quantized
+    with the finished amax (the bits of the one-shot call). V is copied after
+    them, group by group, and each group's quantize + attention + copy back
+    starts as soon as its V has landed. With FP8 Q/K and V (no tensor-wide
+    amax) each group's Q, K, V are copied together."""
+    dev = torch.device(device or "cuda:0")
+    B, H, N, d = q.shape
+    if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
+        raise ValueError("q, k, v must have one shape")
+    BH = B * H
+    spans = [s for s in (head_range(BH, min(chunks, BH), r) for r in range(min(chunks, BH))) if s[1] > s[0]]
+    flat = [t.reshape(BH, N, d) for t in (q, k, v)]
+    cur = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    qd, kd, vd = (torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    out_d = torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev)
+    lse_d = torch.empty((BH, N), dtype=torch.float32, device=dev) if return_lse else None
+    out_h = out_host if out_host is not None else torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = None
+    if return_lse:
+        lse_h = lse_host if lse_host is not None else torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+    out_hf, lse_hf = out_h.view(BH, N, d), (lse_h.view(BH, N) if lse_h is not None else None)
+    s_in.wait_stream(cur)     # the device buffers were allocated on the current stream
+    ev_qk, ev_v = [torch.cuda.Event() for _ in spans], [torch.cuda.Event() for _ in spans]
+    # with no tensor-wide amax to wait for (FP8 Q/K and V), group i's Q, K, V
+    # are copied together so its kernels can start right after them
+    interleave = qk_format == "fp8" and pv_format == "fp8"
+    with torch.cuda.stream(s_in):
+        for i, (a, b) in enumerate(spans):
+            qd[a:b].copy_(flat[0][a:b], non_blocking=True)
+            kd[a:b].copy_(flat[1][a:b], non_blocking=True)
+            ev_qk[i].record(s_in)
+            if interleave:
+                vd[a:b].copy_(flat[2][a:b], non_blocking=True)
+                ev_v[i].record(s_in)
+        if not interleave:
+            for i, (a, b) in enumerate(spans):
+                vd[a:b].copy_(flat[2][a:b], non_blocking=True)
+                ev_v[i].record(s_in)
+
+    def part(t, a, b):
+        return t[a:b].view(1, b - a, N, d)
+
+    amax_q = amax_k = amax_v = None
+    if qk_format == "nvfp4":
+        amax_q, amax_k = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2))
+        for i, (a, b) in enumerate(spans):
+            cur.wait_event(ev_qk[i])
+            tensor_amax(part(qd, a, b), amax_q, accumulate=i > 0)
+            tensor_amax(part(kd, a, b), amax_k, accumulate=i > 0)
+    if pv_format == "nvfp4":
+        amax_v = torch.empty(1, dtype=torch.float32, device=dev)
+        for i, (a, b) in enumerate(spans):
+            cur.wait_event(ev_v[i])
+            tensor_amax(part(vd, a, b), amax_v, accumulate=i > 0)
+    s_out.wait_stream(cur)
+    for i, (a, b) in enumerate(spans):
+        cur.wait_event(ev_qk[i])
+        cur.wait_event(ev_v[i])
+        qc, kc, vc = part(qd, a, b), part(kd, a, b), part(vd, a, b)
+        if qk_format == "nvfp4":
+            qq, kq = quantize_nvfp4(qc, static_amax=amax_q, video=video), quantize_nvfp4(kc, static_amax=amax_k,
+                                                                                        video=video)
+        else:
+            gran = "group" if qk_group_tiles > 1 else "tile128"
+            qq = quantize_fp8(qc, gran, video=video, group_tiles=qk_group_tiles)
+            kq = quantize_fp8(kc, gran, video=video, group_tiles=qk_group_tiles)
+        if pv_format == "fp8":
+            vq = quantize_fp8(vc, "channel", video=video)
+        else:
+            vq = quantize_nvfp4_v(vc, static_amax=amax_v, video=video)
+        attention_fwd(qq, kq, vq, causal=causal, tile_mask=tile_mask, softmax_scale=softmax_scale,
+                      out=out_d[a:b].view(1, b - a, N, d),
+                      lse=None if lse_d is None else lse_d[a:b].view(1, b - a, N), return_lse=return_lse,
+                      video=video, rescale_threshold=rescale_threshold)
+        done = torch.cuda.Event()
+        done.record(cur)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            out_hf[a:b].copy_(out_d[a:b], non_blocking=True)
+            if lse_hf is not None:
+                lse_hf[a:b].copy_(lse_d[a:b], non_blocking=True)
+    cur.wait_stream(s_out)
+    for t in (qd, kd, vd, out_d) + ((lse_d,) if lse_d is not None else ()):
+        t.record_stream(s_in)
+        t.record_stream(s_out)
+    cur.synchronize()
+    return out_h, lse_h
 
 
 def head_range(num_heads: int, world: int, rank: int) -> Tuple[int, int]:

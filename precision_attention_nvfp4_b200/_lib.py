@@ -54,6 +54,8 @@ _SIGNATURES = {
                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "fpattn_quantize_qkv": (ctypes.c_int, [_P(Tensor), _P(Tensor), _P(Tensor), ctypes.c_int32, _P(VideoLayout)] +
                             [ctypes.c_void_p] * 10),
+    "fpattn_tensor_amax": (ctypes.c_int, [_P(Tensor), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p]),
     "fpattn_step_phase": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_double, ctypes.c_double,
                                          _P(ctypes.c_int32)]),
     "fpattn_sta_plan": (ctypes.c_int, [ctypes.c_int32] * 9 + [ctypes.c_void_p] * 3 +

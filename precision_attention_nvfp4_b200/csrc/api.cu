@@ -242,6 +242,16 @@ fpattn_status fpattn_quantize_qkv(const fpattn_tensor* q, const fpattn_tensor* k
                       v_codes, v_scales, nonfinite_flag, stream);
 }
 
+fpattn_status fpattn_tensor_amax(const fpattn_tensor* x, int32_t accumulate, float* amax, int32_t* nonfinite_flag,
+                                 fpattn_stream_t stream) {
+  fpattn_status s = check_tensor(x, FPATTN_BF16);
+  if (s != FPATTN_OK) return s;
+  if (!amax) return FPATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(amax) & 3u) return FPATTN_ERR_ALIGNMENT;
+  return from_cuda(fpattn::launch_tensor_amax_accum(x->data, x->B * x->H, x->N, x->d, accumulate != 0, amax,
+                                              nonfinite_flag, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fpattn_status fpattn_video_layout_check(const fpattn_video_layout* layout, int32_t N) {
   fpattn::VideoLayout vl;
   fpattn::TokenMap tm;

@@ -74,17 +74,6 @@ constexpr int kThreads = 512;
 #define FPATTN_KV_STAGES 3
 #endif
 constexpr int kStages = FPATTN_KV_STAGES;
-// One thread issues both MMA kinds in a fixed interleave (else one thread each).
-#ifndef FPATTN_ONE_ISSUER
-#define FPATTN_ONE_ISSUER 0
-#endif
-constexpr bool kOneIssuer = FPATTN_ONE_ISSUER != 0;
-// Softmax exponentials taken against the previous reference max, before the
-// block's max is known (E4M3 P only).
-#ifndef FPATTN_SPECULATE
-#define FPATTN_SPECULATE 0
-#endif
-constexpr bool kSpeculate = FPATTN_SPECULATE != 0;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
@@ -522,77 +511,73 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
       }
     }
-  } else if (warp == 1 || (!kOneIssuer && warp == 2)) {
-    // ------------------------------------------------------- MMA issue
-    // Warp 1 issues O += P V, warp 2 issues S = Q K^T (one thread each);
-    // with kOneIssuer, warp 1 issues both in the fixed order S(0), S(1),
-    // PV(0), S(2), PV(1), S(3), ...: the S of block g + 2 follows the PV of
-    // block g on the in-order tensor pipe, so no S is queued ahead of a PV
-    // the softmax is waiting to see complete.
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ PV issuer
     if (lane == 0) {
       constexpr uint32_t kIdescPV = PV4 ? idesc_nvf4(128, D) : idesc_e4m3(128, D, true);
+      int g = 0;
+      bool ok = true;
+      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
+        int bh, qb;
+        decode_item(p, item, bh, qb);
+        const KList L = key_list(p, qb);
+        for (int j = 0; j < L.count; ++j, ++g) {
+          // O += P V once P is in TMEM, O has been rescaled and V has landed.
+          const int st = g % kStages;
+          const int pb = g % C::kPBufs;
+          if (!(ok = mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
+          if (!(ok = mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
+          if (!(ok = mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
+          tc_fence_after();
+          const uint64_t v_desc =
+              make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
+          if (PV4) {
+            // block scales of P (written by the softmax) and of V into tensor
+            // memory, then two K = 64 block-scaled MMAs with P from tensor memory
+            const uint32_t sb = (g & 1) * 8;
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              tmem_cp_32x128_warpx4(tmem + C::kColSFP + sb + 4 * a,
+                                    make_smem_desc(smem_u32(smem + C::kOffSFP + pb * C::kSFP + 512 * a), 128, 128, 0));
+              tmem_cp_32x128_warpx4(tmem + C::kColSFV + sb + 4 * a,
+                                    make_smem_desc(smem_u32(smem + C::kOffSFV + st * C::kSFV + 512 * a), 128, 128, 0));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_nvf4_ts(tmem + C::kColO, tmem + C::kColP + pb * C::kPCols + 8 * kk, v_desc + 2 * kk, kIdescPV,
+                          tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
+                            v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(kv_empty + st);
+          mma_commit(o_done + st);
+          *consumed_cnt = g + 1;
+        }
+      }
+      // Drain: every issued MMA completes before tensor memory is released.
+      mma_commit(drain);
+      uint32_t drained = 0;
+      const unsigned long long t0 = globaltimer_ns();
+      while (!(drained = mbar_try_wait(smem_u32(drain), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+      if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- S issuer
+    if (lane == 0) {
       constexpr uint32_t kIdescS = FP4 ? idesc_nvf4(128, 128) : idesc_e4m3(128, 128, false);
       const uint64_t q_desc = make_smem_desc(smem_u32(smem + C::kOffQ), 16, C::kQKSbo, C::kQKSwz);
-      // O += P V for block g (j-th block of its item) once P is in TMEM, O
-      // has been rescaled and V has landed.
-      auto issue_pv = [&](int g, int j) -> bool {
-        const int st = g % kStages;
-        const int pb = g % C::kPBufs;
-        if (!mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull)) return false;
-        if (!mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady)) return false;
-        if (!mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull)) return false;
-        tc_fence_after();
-        const uint64_t v_desc = make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
-        if (PV4) {
-          // block scales of P (written by the softmax) and of V into tensor
-          // memory, then two K = 64 block-scaled MMAs with P from tensor memory
-          const uint32_t sb = (g & 1) * 8;
-#pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            tmem_cp_32x128_warpx4(tmem + C::kColSFP + sb + 4 * a,
-                                  make_smem_desc(smem_u32(smem + C::kOffSFP + pb * C::kSFP + 512 * a), 128, 128, 0));
-            tmem_cp_32x128_warpx4(tmem + C::kColSFV + sb + 4 * a,
-                                  make_smem_desc(smem_u32(smem + C::kOffSFV + st * C::kSFV + 512 * a), 128, 128, 0));
-          }
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_nvf4_ts(tmem + C::kColO, tmem + C::kColP + pb * C::kPCols + 8 * kk, v_desc + 2 * kk, kIdescPV,
-                        tmem + C::kColSFP + sb + 4 * kk, tmem + C::kColSFV + sb + 4 * kk,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8f6f4_ts(tmem + C::kColO, tmem + C::kColP + pb * 32 + 8 * kk,
-                          v_desc + static_cast<uint64_t>((kk * 32 * D) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(kv_empty + st);
-        mma_commit(o_done + st);
-        *consumed_cnt = g + 1;
-        return true;
-      };
-      // S side: walks the same (item, key block) sequence. Q of an item is
-      // waited for before its first S; once its last S is issued, Q (and its
-      // scales) may be replaced. An item without key blocks still takes its
-      // Q phase.
-      int s_rnd = 0, s_it = 0, s_j = 0, s_g = 0, s_bh = 0, s_qb = 0;
-      int s_item = sched_item(0);
-      KList sL{0, 0};
-      if (s_item < p.num_items) {
-        decode_item(p, s_item, s_bh, s_qb);
-        sL = key_list(p, s_qb);
-      }
-      auto next_s_item = [&]() {
-        mma_commit(q_empty);  // all S of the item issued
-        ++s_it;
-        s_j = 0;
-        s_item = sched_item(++s_rnd);
-        if (s_item < p.num_items) {
-          decode_item(p, s_item, s_bh, s_qb);
-          sL = key_list(p, s_qb);
-        }
-      };
-      auto wait_q = [&]() -> bool {
-        if (!mbar_wait(q_full, s_it & 1, abort_flag, &g_error_word, kErrQFull)) return false;
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+        int bh, qb;
+        decode_item(p, item, bh, qb);
+        const KList L = key_list(p, qb);
+        if (!(ok = mbar_wait(q_full, it & 1, abort_flag, &g_error_word, kErrQFull))) break;
         tc_fence_after();
         if (FP4) {
 #pragma unroll
@@ -600,70 +585,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tmem_cp_32x128_warpx4(tmem + C::kColSFQ + 4 * a,
                                   make_smem_desc(smem_u32(smem + C::kOffSFQ + 512 * a), 128, 128, 0));
         }
-        return true;
-      };
-      // Issues the next S of the sequence (none once it is exhausted).
-      auto issue_s = [&]() -> bool {
-        while (s_item < p.num_items && sL.count == 0) {
-          if (!wait_q()) return false;
-          next_s_item();
-        }
-        if (s_item >= p.num_items) return true;
-        if (s_j == 0 && !wait_q()) return false;
-        // S = Q K^T into buffer g % 2 once K has landed and the softmax has
-        // read the buffer's previous tile.
-        const int g = s_g;
-        const int st = g % kStages;
-        const int buf = g & 1;
-        if (!mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull)) return false;
-        if (g >= 2 && !mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree))
-          return false;
-        tc_fence_after();
-        const uint64_t k_desc = make_smem_desc(smem_u32(smem + C::kOffK + st * C::kQKTile), 16, C::kQKSbo, C::kQKSwz);
-        const uint32_t s_tmem = tmem + buf * 128;
-        if (FP4) {
-          const uint32_t sfk = C::kColSFK + buf * C::kSFCols;
+        for (int j = 0; j < L.count; ++j, ++g) {
+          // S = Q K^T into buffer g % 2 once K has landed and the owner
+          // warpgroup has read the buffer's previous tile.
+          const int st = g % kStages;
+          const int buf = g & 1;
+          if (!(ok = mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
+          if (g >= 2 && !(ok = mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
+            break;
+          tc_fence_after();
+          const uint64_t k_desc =
+              make_smem_desc(smem_u32(smem + C::kOffK + st * C::kQKTile), 16, C::kQKSbo, C::kQKSwz);
+          const uint32_t s_tmem = tmem + buf * 128;
+          if (FP4) {
+            const uint32_t sfk = C::kColSFK + buf * C::kSFCols;
 #pragma unroll
-          for (int a = 0; a < D / 64; ++a)
-            tmem_cp_32x128_warpx4(tmem + sfk + 4 * a,
-                                  make_smem_desc(smem_u32(smem + C::kOffSFK + st * C::kSF + 512 * a), 128, 128, 0));
+            for (int a = 0; a < D / 64; ++a)
+              tmem_cp_32x128_warpx4(tmem + sfk + 4 * a,
+                                    make_smem_desc(smem_u32(smem + C::kOffSFK + st * C::kSF + 512 * a), 128, 128, 0));
 #pragma unroll
-          for (int kk = 0; kk < C::kKSteps; ++kk)
-            mma_nvf4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, tmem + C::kColSFQ + 4 * kk,
-                        tmem + sfk + 4 * kk, kk > 0 ? 1u : 0u);
-        } else {
+            for (int kk = 0; kk < C::kKSteps; ++kk)
+              mma_nvf4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, tmem + C::kColSFQ + 4 * kk,
+                          tmem + sfk + 4 * kk, kk > 0 ? 1u : 0u);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < C::kKSteps; ++kk)
-            mma_f8f6f4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(s_full + buf);
-        mma_commit(kv_empty + st);
-        ++s_g;
-        if (++s_j == sL.count) next_s_item();
-        return true;
-      };
-      bool ok = true;
-      if (kOneIssuer || warp == 1) {
-        if (kOneIssuer) ok = issue_s() && issue_s();
-        int g = 0;
-        for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
-          int bh, qb;
-          decode_item(p, item, bh, qb);
-          const KList L = key_list(p, qb);
-          for (int j = 0; j < L.count && ok; ++j, ++g) {
-            ok = issue_pv(g, j);
-            if (kOneIssuer && ok) ok = issue_s();
+            for (int kk = 0; kk < C::kKSteps; ++kk)
+              mma_f8f6f4_ss(s_tmem, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
           }
+          mma_commit(s_full + buf);
+          mma_commit(kv_empty + st);
         }
-      } else {
-        while (ok && s_item < p.num_items) ok = issue_s();
+        if (!ok) break;
+        mma_commit(q_empty);  // all S of the item issued: Q (and its scales) may be replaced
       }
-      // Drain: every issued MMA completes before tensor memory is released.
-      uint64_t* dbar = drain + (warp == 1 ? 0 : 1);
-      mma_commit(dbar);
+      mma_commit(drain + 1);
       uint32_t drained = 0;
       const unsigned long long t0 = globaltimer_ns();
-      while (!(drained = mbar_try_wait(smem_u32(dbar), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!(drained = mbar_try_wait(smem_u32(drain + 1), 0)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
@@ -691,17 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (FP4) c_fp4 = p.q_scale[0] * p.k_scale[0] * p.sm_scale_log2;
       else inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(bh) * p.nblk + qb];
       float l = 0.f, m_ref = -INFINITY;
-      // FP8 K scales are loaded one block ahead
-      float ks_next = (!FP4 && L.count > 0)
-                          ? __ldg(p.k_scale + static_cast<size_t>(bh) * p.nblk + max(key_block(p, L, 0), 0))
-                          : 1.f;
       for (int j = 0; j < L.count && ok; ++j, ++g) {
         const int kb_raw = key_block(p, L, j);
         const int kb = max(kb_raw, 0);
         const int buf = g & 1;
-        const float ks = ks_next;
-        if (!FP4 && j + 1 < L.count)
-          ks_next = __ldg(p.k_scale + static_cast<size_t>(bh) * p.nblk + max(key_block(p, L, j + 1), 0));
         // A failed wait raises the abort flag; the block then runs to its end
         // on whatever the buffers hold (every later wait returns at once) and
         // the loop stops after it.
@@ -724,26 +675,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           mask_chunk(r0, key0, qrow, diag, lim);
           mask_chunk(r1, key0 + 32, qrow, diag, lim);
         }
-        const float c = FP4 ? c_fp4 : inv_sq / ks;
-        const int pb = g % C::kPBufs;
-        if (C::kPWait && g >= C::kPBufs) {
-          // P buffer pb was last read by the PV of block g - kPBufs
-          const int gp = g - C::kPBufs;
-          ok = warp_wait(o_done + gp % kStages, (gp / kStages) & 1, abort_flag, &g_error_word, kErrPFree) && ok;
-          tc_fence_after();
-        }
-        // Speculation: once the row has a reference max, the exponentials are
-        // taken against it before this block's max is known, and taken again
-        // (below) only if the block moves the max of any row of the warp. A
-        // row whose max stays gets exactly the values of the plain order.
-        const bool spec = kSpeculate && !PV4 && __all_sync(0xffffffffu, m_ref != -INFINITY);
-        uint32_t pk0[8], pk1[8];
-        float psum = 0.f;
-        if (!PV4 && spec) {
-          const float nb = p.p_log2_scale - m_ref;
-          psum = exp_pack32<C::kPolyPairs>(r0, c, nb, pk0);
-          psum += exp_pack32<C::kPolyPairs>(r1, c, nb, pk1);
-        }
         const float half_max = max32(r1, max32(r0, -INFINITY));
         // exchange the half maxima (tag g + 1; slots alternate by block parity)
         xs[(buf * 2 + w) * 128 + row] =
@@ -753,6 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                                      abort_flag, &g_error_word, kErrMax);
         ok = __all_sync(0xffffffffu, got) && ok;
         const float rawmax = w == 0 ? fmaxf(half_max, other_max) : fmaxf(other_max, half_max);
+        const float c = FP4 ? c_fp4 : inv_sq / p.k_scale[static_cast<size_t>(bh) * p.nblk + kb];
         // m_ref: reference max (-inf while every key so far is masked). It
         // moves to the running max only when that exceeds it by more than tau
         // (log2 units; tau = 0: the exact running max), and P then reaches at
@@ -776,25 +708,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // P = 2^(c s - m + log2 448) -> E4M3, this half's 16 columns of P
         // buffer g % kPBufs.
         const float nbias = p.p_log2_scale - m_use;
+        const int pb = g % C::kPBufs;
+        if (C::kPWait && g >= C::kPBufs) {
+          // P buffer pb was last read by the PV of block g - kPBufs
+          const int gp = g - C::kPBufs;
+          ok = warp_wait(o_done + gp % kStages, (gp / kStages) & 1, abort_flag, &g_error_word, kErrPFree) && ok;
+          tc_fence_after();
+        }
+        float psum;
         if (PV4) {
           // NVFP4 P: this half's 64 keys are one K = 64 step of the P V
           // product: 8 columns of E2M1 and 4 block scales, which go through
           // shared memory (in the tensor-core scale layout) to the PV issuer.
           const uint32_t p_addr = tmem + lane_off + C::kColP + pb * C::kPCols + 8 * w;
-          uint32_t fq0[4], fq1[4], sfw = 0u;
-          psum = exp_pack32_fp4<C::kPolyPairs>(r0, c, nbias, fq0, sfw, 0);
-          tmem_st4(p_addr, fq0);
-          psum += exp_pack32_fp4<C::kPolyPairs>(r1, c, nbias, fq1, sfw, 2);
-          tmem_st4(p_addr + 4, fq1);
+          uint32_t pk0[4], pk1[4], sfw = 0u;
+          psum = exp_pack32_fp4<C::kPolyPairs>(r0, c, nbias, pk0, sfw, 0);
+          tmem_st4(p_addr, pk0);
+          psum += exp_pack32_fp4<C::kPolyPairs>(r1, c, nbias, pk1, sfw, 2);
+          tmem_st4(p_addr + 4, pk1);
           reinterpret_cast<uint32_t*>(smem + C::kOffSFP + pb * C::kSFP + 512 * w)[(row & 31) * 4 + (row >> 5)] = sfw;
           fence_proxy_async_shared();
         } else {
           const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32 + 16 * w;
-          if (!spec || __any_sync(0xffffffffu, m_new != m_prev)) {
-            psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
-            psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
-          }
+          uint32_t pk0[8], pk1[8];
+          psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk0);
           tmem_st8(p_addr, pk0);
+          psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk1);
           tmem_st8(p_addr + 8, pk1);
         }
         l += psum;

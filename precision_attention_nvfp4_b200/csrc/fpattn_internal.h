@@ -53,6 +53,9 @@ cudaError_t launch_quantize_nvfp4(const void* x, int BH, int N, int d, const flo
                                   uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
                                   const TokenMap* tmap, cudaStream_t st);
 
+// max|x| folded into *amax (zeroed first unless accumulate).
+cudaError_t launch_tensor_amax_accum(const void* x, int BH, int N, int d, bool accumulate, float* amax, int* nonfinite,
+                               cudaStream_t st);
 // Q, K (NVFP4 when qk_fp4, else FP8 per 128-token tile) and V (FP8 per
 // channel) in four launches; results equal the separate launchers'.
 cudaError_t launch_quantize_qkv(const void* q, const void* k, const void* v, int BH, int N, int d, bool qk_fp4,

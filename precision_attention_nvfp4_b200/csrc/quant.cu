@@ -610,6 +610,15 @@ void launch_tensor_amax(const void* x, int BH, int N, int d, float* acc, int* no
 
 }  // namespace
 
+cudaError_t launch_tensor_amax_accum(const void* x, int BH, int N, int d, bool accumulate, float* amax, int* nonfinite,
+                               cudaStream_t st) {
+  if (!accumulate) launch_pdl(zero_kernel, dim3(1), dim3(32), 0, st, amax, 1);
+  const size_t nchunks = static_cast<size_t>(BH) * N * d / 8;
+  launch_pdl(tensor_amax_kernel, dim3(num_sms() * 8), dim3(kThreads), 0, st, static_cast<const uint4*>(x), nchunks,
+             amax, nonfinite);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_nvfp4_tokens(const void* x, int BH, int N, int d, const float* static_amax,
                                          uint8_t* codes, uint8_t* block_sf, float* tensor_scale, int* nonfinite,
                                          const TokenMap* tmap, cudaStream_t st) {
