@@ -295,6 +295,29 @@ def run_reference(args, w):
     return 0
 
 
+def choose_peak(peaks: dict, clk: dict, timed_s: float, qk: str, pv: str):
+    """Tensor peak of the attention kernel (TFLOP/s) for its MMA dtypes.
+
+    The measured bf16 figure times the nominal FP8 / FP4 ratios; both MMAs do
+    2d flops per score, so a mixed path takes the harmonic mean. The
+    sustained bf16 figure was measured under the power cap at a lowered SM
+    clock; it applies to a timed region of a second or more that itself ran
+    capped or below the maximum clock. A shorter region, or one whose clock
+    record shows the maximum clock and no power cap, takes the burst figure
+    (measured at the maximum clock). Returns (peak, burst peak, bf16 figure
+    used, sustained?, capped?)."""
+    capped = bool("sw_power_cap" in clk.get("reasons", []) or
+                  (clk.get("sm_mhz") is not None and clk.get("sm_max_mhz") and
+                   clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"]))
+    sustained = timed_s >= 1.0 and capped and "bf16_tflops_sustained" in peaks
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
+    p_qk = p4 if qk == "nvfp4" else p8
+    p_pv = p4 if pv == "nvfp4" else p8
+    peak = 2.0 / (1.0 / p_qk + 1.0 / p_pv)
+    return peak, peak * peaks["bf16_tflops"] / bf16, bf16, sustained, capped
+
+
 def rank_env():
     """(world, rank, local_rank) from the torchrun environment (1, 0, 0 if absent)."""
     return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
@@ -520,23 +543,8 @@ def main():
     ms_step = ms_total / args.steps
     value = aggregate_value(flops, world, ms_step)
     peaks, peak_src = load_peaks()
-    # The sustained bf16 figure was measured under the power cap at a lowered
-    # SM clock; it applies to a seconds-long timed region that itself ran
-    # capped or below the maximum clock. A short region, or one whose clock
-    # record shows the maximum clock and no power cap, takes the burst figure
-    # (measured at the maximum clock).
     timed_s = ms_total * 1e-3
-    capped = ("sw_power_cap" in clk.get("reasons", []) or
-              (clk.get("sm_mhz") is not None and clk.get("sm_max_mhz") and
-               clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"]))
-    sustained = timed_s >= 1.0 and capped and "bf16_tflops_sustained" in peaks
-    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    p8, p4 = bf16 * FP8_RATIO, bf16 * FP4_RATIO
-    # both MMAs do 2d flops per score: the peak is the harmonic mean of theirs
-    p_qk = p4 if w.qk_format == "nvfp4" else p8
-    p_pv = p4 if args.pv_format == "nvfp4" else p8
-    peak = 2.0 / (1.0 / p_qk + 1.0 / p_pv)
-    peak_burst = peak * peaks["bf16_tflops"] / bf16
+    peak, peak_burst, bf16, sustained, capped = choose_peak(peaks, clk, timed_s, w.qk_format, args.pv_format)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     quant_ms = ms_step - attn_ms
     quant_gbs = quant_bytes(w, args.pv_format) / (quant_ms * 1e-3) / 1e9

@@ -74,6 +74,36 @@ constexpr int kThreads = 512;
 #define FPATTN_KV_STAGES 3
 #endif
 constexpr int kStages = FPATTN_KV_STAGES;
+// Software-pipelined softmax for E4M3 P (the next block's tensor-memory
+// load and row max overlap this block's exponentials).
+#ifndef FPATTN_PIPELINED
+#define FPATTN_PIPELINED 0
+#endif
+constexpr bool kPipelined = FPATTN_PIPELINED != 0;
+// Per-warpgroup register budgets (setmaxnreg) of the 512-thread CTA, which
+// launches with 128 registers a thread: control warps, softmax warps,
+// correction warps. 128 * (56 + 96) + 256 * 176 = 64512 <= 65536.
+#ifndef FPATTN_REG_SPLIT
+#define FPATTN_REG_SPLIT 0
+#endif
+constexpr bool kRegSplit = FPATTN_REG_SPLIT != 0;
+constexpr uint32_t kRegsControl = 56, kRegsSoftmax = 176, kRegsCorrection = 96;
+static_assert(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax <= 65536, "register split");
+// Sleep (ns) between the polls of the single-thread roles' waits; 0 polls
+// with plain try_wait.
+#ifndef FPATTN_CTRL_SLEEP_NS
+#define FPATTN_CTRL_SLEEP_NS 0
+#endif
+// Warp that issues S = Q K^T (2, or 3, the otherwise idle warp).
+#ifndef FPATTN_S_WARP
+#define FPATTN_S_WARP 2
+#endif
+
+// Wait of a single-thread role (TMA producer, MMA issuers).
+__device__ __forceinline__ bool ctrl_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
+  if (FPATTN_CTRL_SLEEP_NS > 0) return mbar_wait_sleep(bar, parity, abort, err, code, FPATTN_CTRL_SLEEP_NS);
+  return mbar_wait(bar, parity, abort, err, code);
+}
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
@@ -387,6 +417,76 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
+// ---------------------------------------------------------------------------
+// Software-pipelined softmax (E4M3 P). A warp holds its half-row of the
+// current block's scores; while their exponentials run, it reads the next
+// block's scores from tensor memory and reduces them to their half-row max,
+// so the tensor-memory load and the max overlap the MUFU and FMA work.
+// ---------------------------------------------------------------------------
+struct SoftCtx {
+  const Params* p;
+  uint32_t tmem, lane_off;
+  int w, row;
+  uint64_t* s_full;
+  uint64_t* s_free;
+  uint64_t* p_full;
+  uint64_t* o_done;
+  uint64_t* a_bar;  // this quarter's ring
+  volatile unsigned long long* xs;
+  float* ax;
+  volatile int* abort_flag;
+};
+
+struct SoftItem {
+  KList L;
+  int bh, qb, qrow;
+  float c_fp4, inv_sq;  // score scale (log2 units): NVFP4 per tensor; FP8 per Q tile, / K tile scale
+  float l, m_ref;
+  bool ok;
+};
+
+// Waits for S(g) and starts the two loads of this warp's 64 scores.
+__device__ __forceinline__ void soft_issue_load(const SoftCtx& x, SoftItem& s, int g, uint32_t (&r0)[32],
+                                                uint32_t (&r1)[32]) {
+  const int buf = g & 1;
+  s.ok = warp_wait(x.s_full + buf, (g >> 1) & 1, x.abort_flag, &g_error_word, kErrSFull) && s.ok;
+  tc_fence_after();
+  const uint32_t a = x.tmem + x.lane_off + buf * 128 + 64 * x.w;
+  tmem_ld32(a, r0);
+  tmem_ld32(a + 32, r1);
+}
+
+// Completes the loads of S(g) (the j-th block of the item), releases the S
+// buffer, masks and returns the half-row max; c receives the block's scale.
+__device__ __forceinline__ float soft_finish_load(const SoftCtx& x, SoftItem& s, int j, int g, uint32_t (&r0)[32],
+                                                  uint32_t (&r1)[32], bool fp4, float ks, float& c) {
+  tmem_wait_ld(r0);
+  tmem_wait_ld(r1);
+  tc_fence_before();
+  warp_arrive(x.s_free + (g & 1));
+  const Params& p = *x.p;
+  const int kb_raw = key_block(p, s.L, j);
+  const int kb = max(kb_raw, 0);
+  const int key0 = kb * 128 + 64 * x.w;
+  const bool diag = p.causal && kb == s.qb;
+  if (diag || (kb + 1) * 128 > p.N || kb_raw < 0) {
+    // an invalid mask entry masks every key of its block
+    const int lim = kb_raw < 0 ? 0 : p.N;
+    mask_chunk(r0, key0, s.qrow, diag, lim);
+    mask_chunk(r1, key0 + 32, s.qrow, diag, lim);
+  }
+  c = fp4 ? s.c_fp4 : s.inv_sq / ks;
+  return max32(r1, max32(r0, -INFINITY));
+}
+
+// Publishes this half's max of block g for the partner warp (tag g + 1; the
+// slots alternate by block parity). The partner has read the slot's previous
+// value (block g - 2) before it published its own half of block g - 1, which
+// this warp has already read.
+__device__ __forceinline__ void soft_publish_max(const SoftCtx& x, int g, float hm) {
+  x.xs[((g & 1) * 2 + x.w) * 128 + x.row] = (static_cast<unsigned long long>(g + 1) << 32) | __float_as_uint(hm);
+}
+
 template <int D, bool FP4, bool PV4>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   using C = Cfg<D, FP4, PV4>;
@@ -470,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   // predecessor's results are read
   griddep_wait();
   if (warp < 4) {
+  if (kRegSplit && !PV4) reg_dealloc<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -481,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
-        if (it > 0) ok = mbar_wait(q_empty, (it - 1) & 1, abort_flag, &g_error_word, kErrQEmpty);
+        if (it > 0) ok = ctrl_wait(q_empty, (it - 1) & 1, abort_flag, &g_error_word, kErrQEmpty);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, C::kQKTile + C::kSF);
         tma_load_3d_hint(smem + C::kOffQ, &p.tm_q, q_full, 0, qb * 128, bh, stream);
@@ -491,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int j = 0; j < L.count; ++j, ++g) {
           const int st = g % kStages;
           const int use = g / kStages;
-          if (use > 0 && !(ok = mbar_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty)))
+          if (use > 0 && !(ok = ctrl_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty)))
             break;
           const int kb = max(key_block(p, L, j), 0);
           mbar_arrive_expect_tx(k_full + st, C::kQKTile + C::kSF);
@@ -525,9 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           // O += P V once P is in TMEM, O has been rescaled and V has landed.
           const int st = g % kStages;
           const int pb = g % C::kPBufs;
-          if (!(ok = mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
-          if (!(ok = mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
-          if (!(ok = mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
+          if (!(ok = ctrl_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
+          if (!(ok = ctrl_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
+          if (!(ok = ctrl_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
           tc_fence_after();
           const uint64_t v_desc =
               make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
@@ -566,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
-  } else if (warp == 2) {
+  } else if (warp == FPATTN_S_WARP) {
     // ------------------------------------------------------------- S issuer
     if (lane == 0) {
       constexpr uint32_t kIdescS = FP4 ? idesc_nvf4(128, 128) : idesc_e4m3(128, 128, false);
@@ -577,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
-        if (!(ok = mbar_wait(q_full, it & 1, abort_flag, &g_error_word, kErrQFull))) break;
+        if (!(ok = ctrl_wait(q_full, it & 1, abort_flag, &g_error_word, kErrQFull))) break;
         tc_fence_after();
         if (FP4) {
 #pragma unroll
@@ -590,8 +691,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           // warpgroup has read the buffer's previous tile.
           const int st = g % kStages;
           const int buf = g & 1;
-          if (!(ok = mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
-          if (g >= 2 && !(ok = mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
+          if (!(ok = ctrl_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
+          if (g >= 2 && !(ok = ctrl_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
             break;
           tc_fence_after();
           const uint64_t k_desc =
@@ -626,8 +727,120 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
   }
+  } else if (warp < 12 && kPipelined && !PV4) {
+    // ------------------------------------------------ softmax (pipelined)
+    // Warpgroup w takes keys 64w..64w+63 of every key block; thread (warp
+    // quarter q, lane t) owns query row 32q + t. The two halves' row maxima
+    // are exchanged per lane through tagged shared-memory words. Block g's
+    // scores sit in one register set while block g+1's are loaded into the
+    // other (the loop is unrolled by two so each set has fixed registers).
+    if (kRegSplit && !PV4) reg_alloc<kRegsSoftmax>();
+    SoftCtx x;
+    x.p = &p;
+    x.tmem = tmem;
+    x.w = (warp - 4) >> 2;
+    const int q4 = warp & 3;
+    x.row = q4 * 32 + lane;
+    x.lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    x.s_full = s_full;
+    x.s_free = s_free;
+    x.p_full = p_full;
+    x.o_done = o_done;
+    x.a_bar = a_bar + q4 * kStages;
+    x.xs = xs;
+    x.ax = ax;
+    x.abort_flag = abort_flag;
+    int g = 0, it = 0;
+    SoftItem s;
+    s.ok = true;
+    uint32_t a0[32], a1[32], b0[32], b1[32];
+    // One block: exchange the half maxima, rescale factor, exponentials of
+    // cur; the next block (if any) is loaded into nxt meanwhile.
+    auto step = [&](int j, uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t (&n0)[32], uint32_t (&n1)[32],
+                    float& hm, float& c) {
+      const int buf = g & 1;
+      // this block's half max was published when it was computed
+      float other;
+      const bool got = tagged_wait(x.xs + (buf * 2 + (x.w ^ 1)) * 128 + x.row, static_cast<uint32_t>(g + 1), other,
+                                   x.abort_flag, &g_error_word, kErrMax);
+      s.ok = __all_sync(0xffffffffu, got) && s.ok;
+      const float rawmax = x.w == 0 ? fmaxf(hm, other) : fmaxf(other, hm);
+      // reference max, rescale factor: as in the plain loop below
+      const float m_prev = s.m_ref;
+      const float cand = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
+      const float m_new = (m_prev == -INFINITY || cand - m_prev > p.tau) ? cand : m_prev;
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = m_prev == m_new ? 1.f : ex2_approx(m_prev - m_use);
+      if (x.w == (g & 1)) {
+        x.ax[(g % kStages) * 128 + x.row] = alpha;
+        warp_arrive(x.a_bar + g % kStages);
+      }
+      s.l *= alpha;
+      s.m_ref = m_new;
+      const float nbias = p.p_log2_scale - m_use;
+      const int pb = g % C::kPBufs;
+      if (C::kPWait && g >= C::kPBufs) {
+        // P buffer pb was last read by the PV of block g - kPBufs
+        const int gp = g - C::kPBufs;
+        s.ok = warp_wait(x.o_done + gp % kStages, (gp / kStages) & 1, x.abort_flag, &g_error_word, kErrPFree) && s.ok;
+        tc_fence_after();
+      }
+      const uint32_t p_addr = x.tmem + x.lane_off + C::kColP + pb * 32 + 16 * x.w;
+      uint32_t pk0[8], pk1[8];
+      float psum = exp_pack32<C::kPolyPairs>(c0, c, nbias, pk0);
+      tmem_st8(p_addr, pk0);
+      const bool more = j + 1 < s.L.count;
+      float ks = 1.f;
+      if (more) {
+        soft_issue_load(x, s, g + 1, n0, n1);
+        if (!FP4) ks = __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, j + 1), 0));
+      }
+      psum += exp_pack32<C::kPolyPairs>(c1, c, nbias, pk1);
+      if (more) {
+        hm = soft_finish_load(x, s, j + 1, g + 1, n0, n1, FP4, ks, c);
+        soft_publish_max(x, g + 1, hm);
+      }
+      tmem_st8(p_addr + 8, pk1);
+      s.l += psum;
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(x.p_full + pb);
+      ++g;
+    };
+    for (int rnd = 0, item = sched_item(0); item < p.num_items && s.ok; item = sched_item(++rnd), ++it) {
+      decode_item(p, item, s.bh, s.qb);
+      s.L = key_list(p, s.qb);
+      s.qrow = s.qb * 128 + x.row;
+      s.c_fp4 = 0.f;
+      s.inv_sq = 0.f;
+      if (FP4) s.c_fp4 = p.q_scale[0] * p.k_scale[0] * p.sm_scale_log2;
+      else s.inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(s.bh) * p.nblk + s.qb];
+      s.l = 0.f;
+      s.m_ref = -INFINITY;
+      if (s.L.count > 0) {
+        float hm, c;
+        soft_issue_load(x, s, g, a0, a1);
+        const float ks =
+            FP4 ? 1.f : __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, 0), 0));
+        hm = soft_finish_load(x, s, 0, g, a0, a1, FP4, ks, c);
+        soft_publish_max(x, g, hm);
+        for (int j = 0; j < s.L.count && s.ok; j += 2) {
+          step(j, a0, a1, b0, b1, hm, c);
+          if (j + 1 < s.L.count && s.ok) step(j + 1, b0, b1, a0, a1, hm, c);
+        }
+      }
+      if (!s.ok) break;
+      // per-item (l, m) of this warpgroup's half of the keys for the epilogue
+      if (it >= 2 && !(s.ok = warp_wait(fin_free + (it & 1), ((it >> 1) - 1) & 1, abort_flag, &g_error_word,
+                                        kErrFin)))
+        break;
+      fin[(((it & 1) * 2 + x.w) * 2 + 0) * 128 + x.row] = s.l;
+      fin[(((it & 1) * 2 + x.w) * 2 + 1) * 128 + x.row] = s.m_ref;
+      warp_arrive(fin_bar + (it & 1));
+    }
   } else if (warp < 12) {
     // ------------------------------------------------------------- softmax
+    if (kRegSplit && !PV4) reg_alloc<kRegsSoftmax>();
     // Both warpgroups work on every key block: warpgroup w takes keys
     // 64w..64w+63 of it. Thread (warp quarter q, lane t) owns query row
     // 32q + t; its 64 scores are read from tensor memory once and stay in
@@ -752,6 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
   } else {
     // ------------------------------------------------- correction, epilogue
+    if (kRegSplit && !PV4) reg_dealloc<kRegsCorrection>();
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t o_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::kColO;
@@ -1042,6 +1256,16 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
                                          C::kSmemRequest);
     if (e != cudaSuccess) return e;
     if (cacheable) configured[dev / 64].fetch_or(bit, std::memory_order_acq_rel);
+  }
+  if (kRegSplit && !PV4) {
+    // The per-warpgroup budgets add up to the 128 registers a thread the
+    // kernel must launch with; with fewer, the softmax warps' increase could
+    // never be granted, so such a build is refused instead of launched.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, FP4, PV4>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * kThreads < static_cast<int>(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax))
+      return cudaErrorInvalidConfiguration;
   }
   const int sms = device_sm_count();
   const int grid = p.num_items < sms ? p.num_items : sms;

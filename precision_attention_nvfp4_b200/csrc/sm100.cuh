@@ -111,6 +111,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// As mbar_wait, with a sleep of ns nanoseconds after each unsuccessful test:
+// for single-thread roles that share an SM sub-partition with busy warps.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort, int* err_word,
+                                                int code, unsigned ns) {
+  const uint32_t addr = smem_u32(bar);
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(addr, parity)) return true;
+    __nanosleep(ns);
+    if ((it & 15u) == 15u) {
+      if (*abort) return false;
+      const unsigned long long now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitTimeoutNs) {
+        atomicCAS(err_word, 0, code);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // As mbar_wait, but polls without suspending the thread: for the few waits on
 // the kernel's critical path, where the wake-up of a suspended thread costs
 // more than the issue slots the polling takes.

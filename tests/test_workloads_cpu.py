@@ -55,3 +55,49 @@ def test_quant_bytes_and_aggregate():
     assert bench.quant_bytes(v) == pytest.approx(2 * nv * 3 + nv * 5)
     # weak scaling: every rank does the per-rank flops in the (max over ranks) step time
     assert bench.aggregate_value(1e12, 4, 2.0) == pytest.approx(4 * 1e12 / 2e-3 / 1e12)
+
+
+def test_peak_choice_follows_the_clock_record():
+    peaks = {"bf16_tflops": 1655.8, "bf16_tflops_sustained": 1416.8, "hbm_gbs": 6538.3}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1357.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    # mixed NVFP4-QK + FP8-PV: harmonic mean of 4x and 2x the bf16 figure
+    peak, burst, bf16, sus, cap = bench.choose_peak(peaks, full, 5.0, "nvfp4", "fp8")
+    assert not sus and not cap and bf16 == 1655.8
+    assert peak == pytest.approx(2 / (1 / (4 * 1655.8) + 1 / (2 * 1655.8))) == pytest.approx(burst)
+    peak, burst, bf16, sus, cap = bench.choose_peak(peaks, capped, 5.0, "fp8", "fp8")
+    assert sus and cap and peak == pytest.approx(2 * 1416.8) and burst == pytest.approx(2 * 1655.8)
+    # a short region is a burst even when capped
+    peak, _, _, sus, _ = bench.choose_peak(peaks, capped, 0.2, "nvfp4", "nvfp4")
+    assert not sus and peak == pytest.approx(4 * 1655.8)
+
+
+def test_clock_sampler_keeps_the_timed_window():
+    cs = bench.ClockSampler(0)
+
+    class _P:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    cs.proc = _P()
+    line = "{sm}, 1965, 700.0, Active, Not Active, Not Active, Not Active, {cap}"
+    cs.samples = [(1.0, line.format(sm=1200, cap="Active")), (2.0, line.format(sm=1965, cap="Not Active")),
+                  (3.0, line.format(sm=1965, cap="Not Active")), (9.0, line.format(sm=900, cap="Active"))]
+    r = cs.stop(1.5, 3.5)
+    assert r["samples"] == 2 and r["sm_mhz"] == 1965.0 and r["reasons"] == [] and r["window"] == "timed region"
+    r = cs.stop(4.0, 4.01)     # no sample inside: all samples, said so
+    assert r["samples"] == 4 and "sw_power_cap" in r["reasons"] and r["window"].startswith("warm-up")
+
+
+def test_oracle_sample_rows_and_rate():
+    w = workloads.get("long_seq_128k_nvfp4")
+    rows = bench.sample_rows(w, [0, 1023])
+    assert [r[0] for r in rows] == [0, 1023 * 128] and all(8 <= len(r) <= 128 for r in rows)
+    small = workloads.get("llm_prefill_causal")
+    assert all(len(r) == 128 for r in bench.sample_rows(small, [0, 31]))
+    # rate: flops over attention time plus the rows' share of the quantization time
+    res = {"flops": 4e9, "attn_s": 1.0, "quant_s": 8.0, "done": [(0, np.arange(64)), (0, np.arange(64))]}
+    assert bench.oracle_rate(res, 1024) == pytest.approx(4e9 / (1.0 + 8.0 * 128 / 1024) / 1e12)
