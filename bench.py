@@ -345,6 +345,8 @@ def config_dict(w):
     if w.sparse:
         c["tokens"] = ("raster (time-major) bf16 in and out; the tile-major permutation runs inside the "
                        "quantize kernels and the attention epilogue")
+    if w != workloads.get(w.name):
+        c["reduced"] = f"B={w.B} H={w.H} instead of the workload's own (a profiler-sized case)"
     return c
 
 
@@ -440,7 +442,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_seq_128k_nvfp4", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=3, help="timed end-to-end calls (0: no e2e leg)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads (B=1) instead of its own B*H: a smaller "
+                         "case of the same kernels for profiler captures; the line says so in config")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--pv-format", default="fp8", choices=["fp8", "nvfp4"],
@@ -451,6 +456,8 @@ def main():
     if args.sweep:
         return run_sweep(args)
     w = workloads.get(args.workload)
+    if args.heads > 0:
+        w = w.scaled(B=1, H=args.heads)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -551,7 +558,7 @@ def main():
 
     # end to end through the public API: pinned host bf16 in, host bf16 out
     e2e = None
-    if rank == 0 or world > 1:
+    if args.e2e_steps > 0 and (rank == 0 or world > 1):
         qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
         out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
         lse_h = torch.empty(q_h.shape[:3], dtype=torch.float32, pin_memory=True)

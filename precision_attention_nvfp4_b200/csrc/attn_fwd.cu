@@ -70,25 +70,46 @@ namespace {
 constexpr int kThreads = 512;
 // Depth of the K/V shared-memory ring (and of the rings that follow it: O
 // rescale hand-off, O done).
+// 0 picks per configuration: 4 for FP8 Q/K with E4M3 P (four P buffers fit
+// in tensor memory), 3 otherwise (measured: a fourth stage with NVFP4 Q/K,
+// where the P buffers stay three, is slower).
 #ifndef FPATTN_KV_STAGES
-#define FPATTN_KV_STAGES 3
+#define FPATTN_KV_STAGES 0
 #endif
-constexpr int kStages = FPATTN_KV_STAGES;
+// Of every 16 exp2 pairs, how many take the FMA-pipe polynomial (the rest
+// take MUFU), with NVFP4 and with FP8 Q/K.
+#ifndef FPATTN_POLY_FP4
+#define FPATTN_POLY_FP4 3
+#endif
+#ifndef FPATTN_POLY_FP8
+#define FPATTN_POLY_FP8 4
+#endif
 // Software-pipelined softmax for E4M3 P (the next block's tensor-memory
 // load and row max overlap this block's exponentials).
 #ifndef FPATTN_PIPELINED
 #define FPATTN_PIPELINED 0
 #endif
 constexpr bool kPipelined = FPATTN_PIPELINED != 0;
+// 2: the two warpgroups order the next block's load and this block's
+// exponentials opposite ways (see the pipelined softmax).
+constexpr bool kStagger = FPATTN_PIPELINED == 2;
 // Per-warpgroup register budgets (setmaxnreg) of the 512-thread CTA, which
 // launches with 128 registers a thread: control warps, softmax warps,
 // correction warps. 128 * (56 + 96) + 256 * 176 = 64512 <= 65536.
 #ifndef FPATTN_REG_SPLIT
-#define FPATTN_REG_SPLIT 0
+#define FPATTN_REG_SPLIT 1
 #endif
 constexpr bool kRegSplit = FPATTN_REG_SPLIT != 0;
 constexpr uint32_t kRegsControl = 56, kRegsSoftmax = 176, kRegsCorrection = 96;
 static_assert(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax <= 65536, "register split");
+// Warp-wide waits test the phase once without blocking before they wait.
+#ifndef FPATTN_TEST_FIRST
+#define FPATTN_TEST_FIRST 0
+#endif
+constexpr bool kTestFirst = FPATTN_TEST_FIRST != 0;
+#ifndef FPATTN_CAUSAL_GROUP_MB
+#define FPATTN_CAUSAL_GROUP_MB 0
+#endif
 // Sleep (ns) between the polls of the single-thread roles' waits; 0 polls
 // with plain try_wait.
 #ifndef FPATTN_CTRL_SLEEP_NS
@@ -119,6 +140,8 @@ enum : int {
 // block-scaled FP4 tensor cores (else E4M3 P and V).
 template <int D, bool FP4, bool PV4>
 struct Cfg {
+  // depth of the K/V ring (and of the rings that follow it)
+  static constexpr int kStages = FPATTN_KV_STAGES > 0 ? FPATTN_KV_STAGES : (!FP4 && !PV4 ? 4 : 3);
   static constexpr int kQKRow = FP4 ? D / 2 : D;          // bytes per Q/K row
   static constexpr int kQKTile = 128 * kQKRow;            // bytes per 128-row Q/K tile
   // V tile of one 128-key block: E4M3 [128 keys][D], or NVFP4 transposed
@@ -134,7 +157,7 @@ struct Cfg {
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
   // of the 16 exp2 pairs of a 32-score chunk, how many take the FMA-pipe
   // polynomial (measured best: 3 next to the cheaper FP4 QK^T, 4 with FP8)
-  static constexpr int kPolyPairs = FP4 ? 3 : 4;
+  static constexpr int kPolyPairs = FP4 ? FPATTN_POLY_FP4 : FPATTN_POLY_FP8;
   static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
   // P buffers, 32 columns each (128 E4M3 keys), as many as K/V stages when
   // tensor memory holds them: the S of block g needs K stage g % kStages,
@@ -206,7 +229,8 @@ struct __align__(64) Params {
   const int32_t* col_idx;
   const int32_t* row_order;
   int N, nblk, BH, num_items;
-  int nnz;  // tile mask entries (sparse runs)
+  int nnz;     // tile mask entries (sparse runs)
+  int hgroup;  // causal runs: heads scheduled together (longest rows first within a group)
   int causal, sparse;
   float sm_scale_log2;
   float tau;           // conditional-rescale threshold, log2 units (0: exact running max)
@@ -239,8 +263,14 @@ __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, 
     qb = p.row_order ? p.row_order[r] : r;
     if (static_cast<unsigned>(qb) >= static_cast<unsigned>(p.nblk)) qb = 0;
   } else if (p.causal) {
-    qb = p.nblk - 1 - item / p.BH;  // longest rows first
-    bh = item % p.BH;
+    // longest rows first within groups of p.hgroup heads whose K/V fit in
+    // part of the L2; the groups follow one another
+    const int span = p.hgroup * p.nblk;  // items of a full group
+    const int grp = item / span;
+    const int r = item - grp * span;
+    const int gsz = min(p.hgroup, p.BH - grp * p.hgroup);
+    qb = p.nblk - 1 - r / gsz;
+    bh = grp * p.hgroup + r % gsz;
   } else {
     bh = item / p.nblk;             // one head's blocks together: K/V shared in L2
     qb = item % p.nblk;
@@ -383,6 +413,8 @@ __device__ __forceinline__ float exp_pack32_fp4(const uint32_t (&r)[32], float c
 // Every lane polls the barrier (one broadcast shared-memory access per poll),
 // so the warp never diverges around the wait.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
+  // a phase that has already completed is seen by one non-blocking test
+  if (kTestFirst && __all_sync(0xffffffffu, mbar_test_wait(smem_u32(bar), parity))) return true;
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err, code));
 }
 
@@ -490,6 +522,7 @@ __device__ __forceinline__ void soft_publish_max(const SoftCtx& x, int g, float 
 template <int D, bool FP4, bool PV4>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   using C = Cfg<D, FP4, PV4>;
+  constexpr int kStages = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -787,20 +820,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       const uint32_t p_addr = x.tmem + x.lane_off + C::kColP + pb * 32 + 16 * x.w;
       uint32_t pk0[8], pk1[8];
-      float psum = exp_pack32<C::kPolyPairs>(c0, c, nbias, pk0);
-      tmem_st8(p_addr, pk0);
       const bool more = j + 1 < s.L.count;
-      float ks = 1.f;
-      if (more) {
+      float psum;
+      float c_next = c, hm_next = hm;
+      // next block: load, reduce to the half max, publish
+      auto next = [&]() {
         soft_issue_load(x, s, g + 1, n0, n1);
-        if (!FP4) ks = __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, j + 1), 0));
+        const float ks =
+            FP4 ? 1.f : __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, j + 1), 0));
+        const float hn = soft_finish_load(x, s, j + 1, g + 1, n0, n1, FP4, ks, c_next);
+        soft_publish_max(x, g + 1, hn);
+        return hn;
+      };
+      if (kStagger) {
+        // Warpgroup 1 reads the next block first and exponentiates after;
+        // warpgroup 0 the other way round: on each SM sub-partition one warp
+        // runs its exponentials while the other waits on tensor memory.
+        if (x.w == 1 && more) hm_next = next();
+        psum = exp_pack32<C::kPolyPairs>(c0, c, nbias, pk0);
+        tmem_st8(p_addr, pk0);
+        psum += exp_pack32<C::kPolyPairs>(c1, c, nbias, pk1);
+        tmem_st8(p_addr + 8, pk1);
+        if (x.w == 0 && more) hm_next = next();
+      } else {
+        psum = exp_pack32<C::kPolyPairs>(c0, c, nbias, pk0);
+        tmem_st8(p_addr, pk0);
+        float ks = 1.f;
+        if (more) {
+          soft_issue_load(x, s, g + 1, n0, n1);
+          if (!FP4) ks = __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, j + 1), 0));
+        }
+        psum += exp_pack32<C::kPolyPairs>(c1, c, nbias, pk1);
+        if (more) {
+          hm_next = soft_finish_load(x, s, j + 1, g + 1, n0, n1, FP4, ks, c_next);
+          soft_publish_max(x, g + 1, hm_next);
+        }
+        tmem_st8(p_addr + 8, pk1);
       }
-      psum += exp_pack32<C::kPolyPairs>(c1, c, nbias, pk1);
-      if (more) {
-        hm = soft_finish_load(x, s, j + 1, g + 1, n0, n1, FP4, ks, c);
-        soft_publish_max(x, g + 1, hm);
-      }
-      tmem_st8(p_addr + 8, pk1);
+      hm = hm_next;
+      c = c_next;
       s.l += psum;
       tmem_wait_st();
       tc_fence_before();
@@ -1239,6 +1297,18 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   p.BH = BH;
   p.num_items = BH * p.nblk;
   p.causal = a.causal ? 1 : 0;
+  {
+    // Causal runs order the items longest row first; with every head in one
+    // group (the default), the same query block of all heads is in flight at
+    // once and all heads' K/V cycle through the L2. FPATTN_CAUSAL_GROUP_MB > 0
+    // groups the heads so that a group's K and V (codes and scales) take
+    // about that many MB of L2 (40 measured 5% slower on the LLM prefill).
+    const double kv_head = static_cast<double>(a.N) * (C::kQKRow + C::kSF / 128.0 + (PV4 ? D / 2.0 : D));
+    const double budget = FPATTN_CAUSAL_GROUP_MB * 1024.0 * 1024.0;
+    p.hgroup = budget > 0 ? static_cast<int>(budget / kv_head) : BH;
+    if (p.hgroup < 1) p.hgroup = 1;
+    if (p.hgroup > BH) p.hgroup = BH;
+  }
   p.sparse = a.row_ptr ? 1 : 0;
   p.nnz = a.nnz;
   p.sm_scale_log2 = a.softmax_scale * 1.4426950408889634f;
