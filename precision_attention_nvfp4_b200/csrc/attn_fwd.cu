@@ -21,13 +21,16 @@
 //
 // CTA organisation (persistent, one CTA per SM, 512 threads):
 //   warp 0        TMA producer: Q once per work item, K/V tiles into a
-//                 3-stage shared-memory ring (plus block scales)
+//                 shared-memory ring, 4 stages deep for FP8 Q/K with E4M3 P
+//                 and 3 otherwise (plus block scales)
 //   warp 1        tensor-memory allocator; issues O += P V (one thread)
 //   warp 2        issues S = Q K^T (one thread)
 //   warp 3        idle
 //   warps 4-7     softmax warpgroup 0: keys 0-63 of every key block
 //   warps 8-11    softmax warpgroup 1: keys 64-127 of every key block
 //   warps 12-15   O rescale (correction) and epilogue
+// The CTA launches with 128 registers a thread; the warpgroups then take
+// 56 (control), 176 (softmax) and 96 (correction) with setmaxnreg.
 // Thread (warp quarter q, lane t) of a softmax warpgroup owns query row
 // 32q + t and its warpgroup's 64 keys of the block, read from TMEM once into
 // registers. The two warps sharing a row quarter (and an SM sub-partition)
@@ -37,7 +40,8 @@
 // sum of its half; the epilogue adds the two.
 // Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32
 // 128x128, buffer = block parity), O at column 256 (d fp32 columns), a ring
-// of three P buffers (E4M3: 32 columns each; NVFP4: 16) at 384, then the
+// of P buffers (one per ring stage, three with NVFP4 Q/K; E4M3: 32 columns
+// each, NVFP4: 16) at 384, then the
 // NVFP4 scale vectors (Q, two K tiles; with PV4 also two each of P and V).
 // S and P having their own buffers lets the S of a block be issued as soon as
 // its buffer's previous tile has been read, independently of the PV of that
@@ -84,15 +88,6 @@ constexpr int kThreads = 512;
 #ifndef FPATTN_POLY_FP8
 #define FPATTN_POLY_FP8 4
 #endif
-// Software-pipelined softmax for E4M3 P (the next block's tensor-memory
-// load and row max overlap this block's exponentials).
-#ifndef FPATTN_PIPELINED
-#define FPATTN_PIPELINED 0
-#endif
-constexpr bool kPipelined = FPATTN_PIPELINED != 0;
-// 2: the two warpgroups order the next block's load and this block's
-// exponentials opposite ways (see the pipelined softmax).
-constexpr bool kStagger = FPATTN_PIPELINED == 2;
 // Per-warpgroup register budgets (setmaxnreg) of the 512-thread CTA, which
 // launches with 128 registers a thread: control warps, softmax warps,
 // correction warps. 128 * (56 + 96) + 256 * 176 = 64512 <= 65536.
@@ -102,6 +97,13 @@ constexpr bool kStagger = FPATTN_PIPELINED == 2;
 constexpr bool kRegSplit = FPATTN_REG_SPLIT != 0;
 constexpr uint32_t kRegsControl = 56, kRegsSoftmax = 176, kRegsCorrection = 96;
 static_assert(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax <= 65536, "register split");
+// Row-split softmax for E4M3 P: each softmax warp owns 16 rows and all 128
+// keys of a block (else each warpgroup owns 64 keys of all 128 rows and the
+// two exchange half-row maxima every block).
+#ifndef FPATTN_ROW_SPLIT
+#define FPATTN_ROW_SPLIT 1
+#endif
+constexpr bool kRowSplit = FPATTN_ROW_SPLIT != 0;
 // Warp-wide waits test the phase once without blocking before they wait.
 #ifndef FPATTN_TEST_FIRST
 #define FPATTN_TEST_FIRST 0
@@ -110,21 +112,6 @@ constexpr bool kTestFirst = FPATTN_TEST_FIRST != 0;
 #ifndef FPATTN_CAUSAL_GROUP_MB
 #define FPATTN_CAUSAL_GROUP_MB 0
 #endif
-// Sleep (ns) between the polls of the single-thread roles' waits; 0 polls
-// with plain try_wait.
-#ifndef FPATTN_CTRL_SLEEP_NS
-#define FPATTN_CTRL_SLEEP_NS 0
-#endif
-// Warp that issues S = Q K^T (2, or 3, the otherwise idle warp).
-#ifndef FPATTN_S_WARP
-#define FPATTN_S_WARP 2
-#endif
-
-// Wait of a single-thread role (TMA producer, MMA issuers).
-__device__ __forceinline__ bool ctrl_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
-  if (FPATTN_CTRL_SLEEP_NS > 0) return mbar_wait_sleep(bar, parity, abort, err, code, FPATTN_CTRL_SLEEP_NS);
-  return mbar_wait(bar, parity, abort, err, code);
-}
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
@@ -309,6 +296,28 @@ __device__ __forceinline__ void mask_chunk(uint32_t (&r)[32], int key0, int qrow
   }
 }
 
+// As mask_chunk for 32 scores of keys key0, key0 + 2, ..., key0 + 62.
+__device__ __forceinline__ void mask_chunk2(uint32_t (&r)[32], int key0, int qrow, bool causal_diag, int N) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int key = key0 + 2 * i;
+    if ((causal_diag && key > qrow) || key >= N) r[i] = 0xff800000u;  // -inf
+  }
+}
+
+// The two threads of a row (lanes t and t ^ 2 of the 16x64b pattern) hold
+// E4M3 P of keys 8j + {0, 2, 4, 6} (par 0) and 8j + {1, 3, 5, 7} (par 1) in
+// pk[j], byte by byte. Afterwards the par-0 thread holds P column 2j (keys
+// 8j .. 8j+3) and the par-1 thread column 2j + 1 (keys 8j+4 .. 8j+7), key
+// 4k + b in byte b.
+__device__ __forceinline__ void pair_columns(uint32_t (&pk)[8], int par) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, pk[j], 2);
+    pk[j] = par ? __byte_perm(pk[j], other, 0x3726) : __byte_perm(pk[j], other, 0x5140);
+  }
+}
+
 // Max of 32 scores: a tree of three-input max instructions.
 __device__ __forceinline__ float max32(const uint32_t (&r)[32], float m) {
   float a[4];
@@ -449,76 +458,6 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-// ---------------------------------------------------------------------------
-// Software-pipelined softmax (E4M3 P). A warp holds its half-row of the
-// current block's scores; while their exponentials run, it reads the next
-// block's scores from tensor memory and reduces them to their half-row max,
-// so the tensor-memory load and the max overlap the MUFU and FMA work.
-// ---------------------------------------------------------------------------
-struct SoftCtx {
-  const Params* p;
-  uint32_t tmem, lane_off;
-  int w, row;
-  uint64_t* s_full;
-  uint64_t* s_free;
-  uint64_t* p_full;
-  uint64_t* o_done;
-  uint64_t* a_bar;  // this quarter's ring
-  volatile unsigned long long* xs;
-  float* ax;
-  volatile int* abort_flag;
-};
-
-struct SoftItem {
-  KList L;
-  int bh, qb, qrow;
-  float c_fp4, inv_sq;  // score scale (log2 units): NVFP4 per tensor; FP8 per Q tile, / K tile scale
-  float l, m_ref;
-  bool ok;
-};
-
-// Waits for S(g) and starts the two loads of this warp's 64 scores.
-__device__ __forceinline__ void soft_issue_load(const SoftCtx& x, SoftItem& s, int g, uint32_t (&r0)[32],
-                                                uint32_t (&r1)[32]) {
-  const int buf = g & 1;
-  s.ok = warp_wait(x.s_full + buf, (g >> 1) & 1, x.abort_flag, &g_error_word, kErrSFull) && s.ok;
-  tc_fence_after();
-  const uint32_t a = x.tmem + x.lane_off + buf * 128 + 64 * x.w;
-  tmem_ld32(a, r0);
-  tmem_ld32(a + 32, r1);
-}
-
-// Completes the loads of S(g) (the j-th block of the item), releases the S
-// buffer, masks and returns the half-row max; c receives the block's scale.
-__device__ __forceinline__ float soft_finish_load(const SoftCtx& x, SoftItem& s, int j, int g, uint32_t (&r0)[32],
-                                                  uint32_t (&r1)[32], bool fp4, float ks, float& c) {
-  tmem_wait_ld(r0);
-  tmem_wait_ld(r1);
-  tc_fence_before();
-  warp_arrive(x.s_free + (g & 1));
-  const Params& p = *x.p;
-  const int kb_raw = key_block(p, s.L, j);
-  const int kb = max(kb_raw, 0);
-  const int key0 = kb * 128 + 64 * x.w;
-  const bool diag = p.causal && kb == s.qb;
-  if (diag || (kb + 1) * 128 > p.N || kb_raw < 0) {
-    // an invalid mask entry masks every key of its block
-    const int lim = kb_raw < 0 ? 0 : p.N;
-    mask_chunk(r0, key0, s.qrow, diag, lim);
-    mask_chunk(r1, key0 + 32, s.qrow, diag, lim);
-  }
-  c = fp4 ? s.c_fp4 : s.inv_sq / ks;
-  return max32(r1, max32(r0, -INFINITY));
-}
-
-// Publishes this half's max of block g for the partner warp (tag g + 1; the
-// slots alternate by block parity). The partner has read the slot's previous
-// value (block g - 2) before it published its own half of block g - 1, which
-// this warp has already read.
-__device__ __forceinline__ void soft_publish_max(const SoftCtx& x, int g, float hm) {
-  x.xs[((g & 1) * 2 + x.w) * 128 + x.row] = (static_cast<unsigned long long>(g + 1) << 32) | __float_as_uint(hm);
-}
-
 template <int D, bool FP4, bool PV4>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   using C = Cfg<D, FP4, PV4>;
@@ -579,7 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     for (int s = 0; s < kStages; ++s) mbar_init(o_done + s, 1);
     mbar_init(drain, 1);
     mbar_init(drain + 1, 1);
-    for (int i = 0; i < 4 * kStages; ++i) mbar_init(a_bar + i, 1);
+    // rescale factors: both warps of a quarter publish every block (row
+    // split), or the two warpgroups take turns (half-key loop)
+    for (int i = 0; i < 4 * kStages; ++i) mbar_init(a_bar + i, kRowSplit && !PV4 ? 2 : 1);
     *abort_flag = 0;
     *issued_cnt = 0;
     *consumed_cnt = 0;
@@ -615,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
-        if (it > 0) ok = ctrl_wait(q_empty, (it - 1) & 1, abort_flag, &g_error_word, kErrQEmpty);
+        if (it > 0) ok = mbar_wait(q_empty, (it - 1) & 1, abort_flag, &g_error_word, kErrQEmpty);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, C::kQKTile + C::kSF);
         tma_load_3d_hint(smem + C::kOffQ, &p.tm_q, q_full, 0, qb * 128, bh, stream);
@@ -625,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int j = 0; j < L.count; ++j, ++g) {
           const int st = g % kStages;
           const int use = g / kStages;
-          if (use > 0 && !(ok = ctrl_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty)))
+          if (use > 0 && !(ok = mbar_wait(kv_empty + st, (use - 1) & 1, abort_flag, &g_error_word, kErrKvEmpty)))
             break;
           const int kb = max(key_block(p, L, j), 0);
           mbar_arrive_expect_tx(k_full + st, C::kQKTile + C::kSF);
@@ -659,9 +600,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           // O += P V once P is in TMEM, O has been rescaled and V has landed.
           const int st = g % kStages;
           const int pb = g % C::kPBufs;
-          if (!(ok = ctrl_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
-          if (!(ok = ctrl_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
-          if (!(ok = ctrl_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
+          if (!(ok = mbar_wait(p_full + pb, (g / C::kPBufs) & 1, abort_flag, &g_error_word, kErrPFull))) break;
+          if (!(ok = mbar_wait(o_ready + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrOReady))) break;
+          if (!(ok = mbar_wait(v_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrVFull))) break;
           tc_fence_after();
           const uint64_t v_desc =
               make_smem_desc(smem_u32(smem + C::kOffV + st * C::kVTile), 16, C::kVSbo, C::kVSwz);
@@ -700,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
-  } else if (warp == FPATTN_S_WARP) {
+  } else if (warp == 2) {
     // ------------------------------------------------------------- S issuer
     if (lane == 0) {
       constexpr uint32_t kIdescS = FP4 ? idesc_nvf4(128, 128) : idesc_e4m3(128, 128, false);
@@ -711,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
-        if (!(ok = ctrl_wait(q_full, it & 1, abort_flag, &g_error_word, kErrQFull))) break;
+        if (!(ok = mbar_wait(q_full, it & 1, abort_flag, &g_error_word, kErrQFull))) break;
         tc_fence_after();
         if (FP4) {
 #pragma unroll
@@ -724,8 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           // warpgroup has read the buffer's previous tile.
           const int st = g % kStages;
           const int buf = g & 1;
-          if (!(ok = ctrl_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
-          if (g >= 2 && !(ok = ctrl_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
+          if (!(ok = mbar_wait(k_full + st, (g / kStages) & 1, abort_flag, &g_error_word, kErrKFull))) break;
+          if (g >= 2 && !(ok = mbar_wait(s_free + buf, ((g >> 1) - 1) & 1, abort_flag, &g_error_word, kErrSFree)))
             break;
           tc_fence_after();
           const uint64_t k_desc =
@@ -760,140 +701,114 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (!drained) atomicCAS(&g_error_word, 0, kErrDrain);
     }
   }
-  } else if (warp < 12 && kPipelined && !PV4) {
-    // ------------------------------------------------ softmax (pipelined)
-    // Warpgroup w takes keys 64w..64w+63 of every key block; thread (warp
-    // quarter q, lane t) owns query row 32q + t. The two halves' row maxima
-    // are exchanged per lane through tagged shared-memory words. Block g's
-    // scores sit in one register set while block g+1's are loaded into the
-    // other (the loop is unrolled by two so each set has fixed registers).
-    if (kRegSplit && !PV4) reg_alloc<kRegsSoftmax>();
-    SoftCtx x;
-    x.p = &p;
-    x.tmem = tmem;
-    x.w = (warp - 4) >> 2;
+  } else if (warp < 12 && kRowSplit && !PV4) {
+    // ------------------------------------------------ softmax (row split)
+    // Warp (warpgroup w, quarter q) owns rows 32q + 16w .. 32q + 16w + 15 of
+    // the query tile and all 128 keys of every block: thread t takes row
+    // 32q + 16w + t/4 + 8 (t & 1) and the keys of parity (t >> 1) & 1, 64
+    // scores read from tensor memory once (the 16x64b access pattern; the
+    // partner thread of the row is t ^ 2). The two threads of a row combine their maxima with
+    // one shuffle and keep partial row sums, so no warp waits on another: the
+    // two warps of an SM sub-partition run their blocks independently, and
+    // one's exponentials fill the other's latencies.
+    if (kRegSplit) reg_alloc<kRegsSoftmax>();
+    const int w = (warp - 4) >> 2;
     const int q4 = warp & 3;
-    x.row = q4 * 32 + lane;
-    x.lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    x.s_full = s_full;
-    x.s_free = s_free;
-    x.p_full = p_full;
-    x.o_done = o_done;
-    x.a_bar = a_bar + q4 * kStages;
-    x.xs = xs;
-    x.ax = ax;
-    x.abort_flag = abort_flag;
+    const int par = (lane >> 1) & 1;
+    const int row = q4 * 32 + w * 16 + (lane >> 2) + 8 * (lane & 1);
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32 + w * 16) << 16;
     int g = 0, it = 0;
-    SoftItem s;
-    s.ok = true;
-    uint32_t a0[32], a1[32], b0[32], b1[32];
-    // One block: exchange the half maxima, rescale factor, exponentials of
-    // cur; the next block (if any) is loaded into nxt meanwhile.
-    auto step = [&](int j, uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t (&n0)[32], uint32_t (&n1)[32],
-                    float& hm, float& c) {
-      const int buf = g & 1;
-      // this block's half max was published when it was computed
-      float other;
-      const bool got = tagged_wait(x.xs + (buf * 2 + (x.w ^ 1)) * 128 + x.row, static_cast<uint32_t>(g + 1), other,
-                                   x.abort_flag, &g_error_word, kErrMax);
-      s.ok = __all_sync(0xffffffffu, got) && s.ok;
-      const float rawmax = x.w == 0 ? fmaxf(hm, other) : fmaxf(other, hm);
-      // reference max, rescale factor: as in the plain loop below
-      const float m_prev = s.m_ref;
-      const float cand = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
-      const float m_new = (m_prev == -INFINITY || cand - m_prev > p.tau) ? cand : m_prev;
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = m_prev == m_new ? 1.f : ex2_approx(m_prev - m_use);
-      if (x.w == (g & 1)) {
-        x.ax[(g % kStages) * 128 + x.row] = alpha;
-        warp_arrive(x.a_bar + g % kStages);
-      }
-      s.l *= alpha;
-      s.m_ref = m_new;
-      const float nbias = p.p_log2_scale - m_use;
-      const int pb = g % C::kPBufs;
-      if (C::kPWait && g >= C::kPBufs) {
-        // P buffer pb was last read by the PV of block g - kPBufs
-        const int gp = g - C::kPBufs;
-        s.ok = warp_wait(x.o_done + gp % kStages, (gp / kStages) & 1, x.abort_flag, &g_error_word, kErrPFree) && s.ok;
+    bool ok = true;
+    for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+      int bh, qb;
+      decode_item(p, item, bh, qb);
+      const KList L = key_list(p, qb);
+      const int qrow = qb * 128 + row;
+      float c_fp4 = 0.f, inv_sq = 0.f;
+      if (FP4) c_fp4 = p.q_scale[0] * p.k_scale[0] * p.sm_scale_log2;
+      else inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(bh) * p.nblk + qb];
+      float l = 0.f, m_ref = -INFINITY;
+      // FP8 K tile scales are read one block ahead
+      float ks_next = (!FP4 && L.count > 0)
+                          ? __ldg(p.k_scale + static_cast<size_t>(bh) * p.nblk + max(key_block(p, L, 0), 0))
+                          : 1.f;
+      for (int j = 0; j < L.count && ok; ++j, ++g) {
+        const int kb_raw = key_block(p, L, j);
+        const int kb = max(kb_raw, 0);
+        const int buf = g & 1;
+        const float ks = ks_next;
+        if (!FP4 && j + 1 < L.count)
+          ks_next = __ldg(p.k_scale + static_cast<size_t>(bh) * p.nblk + max(key_block(p, L, j + 1), 0));
+        ok = warp_wait(s_full + buf, (g >> 1) & 1, abort_flag, &g_error_word, kErrSFull);
         tc_fence_after();
-      }
-      const uint32_t p_addr = x.tmem + x.lane_off + C::kColP + pb * 32 + 16 * x.w;
-      uint32_t pk0[8], pk1[8];
-      const bool more = j + 1 < s.L.count;
-      float psum;
-      float c_next = c, hm_next = hm;
-      // next block: load, reduce to the half max, publish
-      auto next = [&]() {
-        soft_issue_load(x, s, g + 1, n0, n1);
-        const float ks =
-            FP4 ? 1.f : __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, j + 1), 0));
-        const float hn = soft_finish_load(x, s, j + 1, g + 1, n0, n1, FP4, ks, c_next);
-        soft_publish_max(x, g + 1, hn);
-        return hn;
-      };
-      if (kStagger) {
-        // Warpgroup 1 reads the next block first and exponentiates after;
-        // warpgroup 0 the other way round: on each SM sub-partition one warp
-        // runs its exponentials while the other waits on tensor memory.
-        if (x.w == 1 && more) hm_next = next();
-        psum = exp_pack32<C::kPolyPairs>(c0, c, nbias, pk0);
-        tmem_st8(p_addr, pk0);
-        psum += exp_pack32<C::kPolyPairs>(c1, c, nbias, pk1);
-        tmem_st8(p_addr + 8, pk1);
-        if (x.w == 0 && more) hm_next = next();
-      } else {
-        psum = exp_pack32<C::kPolyPairs>(c0, c, nbias, pk0);
-        tmem_st8(p_addr, pk0);
-        float ks = 1.f;
-        if (more) {
-          soft_issue_load(x, s, g + 1, n0, n1);
-          if (!FP4) ks = __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, j + 1), 0));
+        uint32_t r0[32], r1[32];
+        const uint32_t s_addr = tmem + lane_off + buf * 128;
+        tmem_ld16x64b_x32(s_addr, r0);       // keys 2i + par
+        tmem_ld16x64b_x32(s_addr + 64, r1);  // keys 64 + 2i + par
+        tmem_wait_ld(r0);
+        tmem_wait_ld(r1);
+        tc_fence_before();
+        warp_arrive(s_free + buf);
+        const int key0 = kb * 128 + par;
+        const bool diag = p.causal && kb == qb;
+        if (diag || (kb + 1) * 128 > p.N || kb_raw < 0) {
+          // an invalid mask entry masks every key of its block
+          const int lim = kb_raw < 0 ? 0 : p.N;
+          mask_chunk2(r0, key0, qrow, diag, lim);
+          mask_chunk2(r1, key0 + 64, qrow, diag, lim);
         }
-        psum += exp_pack32<C::kPolyPairs>(c1, c, nbias, pk1);
-        if (more) {
-          hm_next = soft_finish_load(x, s, j + 1, g + 1, n0, n1, FP4, ks, c_next);
-          soft_publish_max(x, g + 1, hm_next);
+        const float own = max32(r1, max32(r0, -INFINITY));
+        const float rawmax = fmaxf(own, __shfl_xor_sync(0xffffffffu, own, 2));
+        const float c = FP4 ? c_fp4 : inv_sq / ks;
+        // reference max and rescale factor: as in the half-key loop below
+        const float m_prev = m_ref;
+        const float cand = rawmax == -INFINITY ? m_prev : fmaxf(m_prev, rawmax * c);
+        const float m_new = (m_prev == -INFINITY || cand - m_prev > p.tau) ? cand : m_prev;
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = m_prev == m_new ? 1.f : ex2_approx(m_prev - m_use);
+        // both warps of the quarter publish their 16 rows' factors every block
+        if (par == 0) ax[(g % kStages) * 128 + row] = alpha;
+        warp_arrive(a_bar + q4 * kStages + g % kStages);
+        l *= alpha;
+        m_ref = m_new;
+        const float nbias = p.p_log2_scale - m_use;
+        const int pb = g % C::kPBufs;
+        if (C::kPWait && g >= C::kPBufs) {
+          // P buffer pb was last read by the PV of block g - kPBufs
+          const int gp = g - C::kPBufs;
+          ok = warp_wait(o_done + gp % kStages, (gp / kStages) & 1, abort_flag, &g_error_word, kErrPFree) && ok;
+          tc_fence_after();
         }
-        tmem_st8(p_addr + 8, pk1);
+        // P: each thread packs its keys 8j + par + {0, 2, 4, 6}; the pair
+        // swaps halves so that the even thread holds P column 2j (keys
+        // 8j .. 8j + 3) and the odd one column 2j + 1, the columns the 16x64b
+        // store writes from them.
+        const uint32_t p_addr = tmem + lane_off + C::kColP + pb * 32;
+        uint32_t pk[8];
+        float psum = exp_pack32<C::kPolyPairs>(r0, c, nbias, pk);
+        pair_columns(pk, par);
+        tmem_st16x64b_x8(p_addr, pk);
+        psum += exp_pack32<C::kPolyPairs>(r1, c, nbias, pk);
+        pair_columns(pk, par);
+        tmem_st16x64b_x8(p_addr + 16, pk);
+        l += psum;
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(p_full + pb);
       }
-      hm = hm_next;
-      c = c_next;
-      s.l += psum;
-      tmem_wait_st();
-      tc_fence_before();
-      warp_arrive(x.p_full + pb);
-      ++g;
-    };
-    for (int rnd = 0, item = sched_item(0); item < p.num_items && s.ok; item = sched_item(++rnd), ++it) {
-      decode_item(p, item, s.bh, s.qb);
-      s.L = key_list(p, s.qb);
-      s.qrow = s.qb * 128 + x.row;
-      s.c_fp4 = 0.f;
-      s.inv_sq = 0.f;
-      if (FP4) s.c_fp4 = p.q_scale[0] * p.k_scale[0] * p.sm_scale_log2;
-      else s.inv_sq = p.sm_scale_log2 / p.q_scale[static_cast<size_t>(s.bh) * p.nblk + s.qb];
-      s.l = 0.f;
-      s.m_ref = -INFINITY;
-      if (s.L.count > 0) {
-        float hm, c;
-        soft_issue_load(x, s, g, a0, a1);
-        const float ks =
-            FP4 ? 1.f : __ldg(p.k_scale + static_cast<size_t>(s.bh) * p.nblk + max(key_block(p, s.L, 0), 0));
-        hm = soft_finish_load(x, s, 0, g, a0, a1, FP4, ks, c);
-        soft_publish_max(x, g, hm);
-        for (int j = 0; j < s.L.count && s.ok; j += 2) {
-          step(j, a0, a1, b0, b1, hm, c);
-          if (j + 1 < s.L.count && s.ok) step(j + 1, b0, b1, a0, a1, hm, c);
-        }
-      }
-      if (!s.ok) break;
-      // per-item (l, m) of this warpgroup's half of the keys for the epilogue
-      if (it >= 2 && !(s.ok = warp_wait(fin_free + (it & 1), ((it >> 1) - 1) & 1, abort_flag, &g_error_word,
-                                        kErrFin)))
+      if (!ok) break;
+      // per-item (l, m) of the row for the epilogue, in the first half's
+      // slot; the second half's slot is empty (l = 0)
+      const float lrow = l + __shfl_xor_sync(0xffffffffu, l, 2);
+      if (it >= 2 && !(ok = warp_wait(fin_free + (it & 1), ((it >> 1) - 1) & 1, abort_flag, &g_error_word,
+                                      kErrFin)))
         break;
-      fin[(((it & 1) * 2 + x.w) * 2 + 0) * 128 + x.row] = s.l;
-      fin[(((it & 1) * 2 + x.w) * 2 + 1) * 128 + x.row] = s.m_ref;
+      if (par == 0) {
+        fin[(((it & 1) * 2 + 0) * 2 + 0) * 128 + row] = lrow;
+        fin[(((it & 1) * 2 + 0) * 2 + 1) * 128 + row] = m_ref;
+        fin[(((it & 1) * 2 + 1) * 2 + 0) * 128 + row] = 0.f;
+        fin[(((it & 1) * 2 + 1) * 2 + 1) * 128 + row] = -INFINITY;
+      }
       warp_arrive(fin_bar + (it & 1));
     }
   } else if (warp < 12) {
