@@ -83,10 +83,10 @@ constexpr int kThreads = 512;
 // Of every 16 exp2 pairs, how many take the FMA-pipe polynomial (the rest
 // take MUFU), with NVFP4 and with FP8 Q/K.
 #ifndef FPATTN_POLY_FP4
-#define FPATTN_POLY_FP4 3
+#define FPATTN_POLY_FP4 5
 #endif
 #ifndef FPATTN_POLY_FP8
-#define FPATTN_POLY_FP8 4
+#define FPATTN_POLY_FP8 5
 #endif
 // Per-warpgroup register budgets (setmaxnreg) of the 512-thread CTA, which
 // launches with 128 registers a thread: control warps, softmax warps,
@@ -104,11 +104,6 @@ static_assert(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax <= 655
 #define FPATTN_ROW_SPLIT 1
 #endif
 constexpr bool kRowSplit = FPATTN_ROW_SPLIT != 0;
-// Warp-wide waits test the phase once without blocking before they wait.
-#ifndef FPATTN_TEST_FIRST
-#define FPATTN_TEST_FIRST 0
-#endif
-constexpr bool kTestFirst = FPATTN_TEST_FIRST != 0;
 #ifndef FPATTN_CAUSAL_GROUP_MB
 #define FPATTN_CAUSAL_GROUP_MB 0
 #endif
@@ -143,7 +138,7 @@ struct Cfg {
   static constexpr uint32_t kVSbo = PV4 ? 8 * 64 : 8 * D;
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
   // of the 16 exp2 pairs of a 32-score chunk, how many take the FMA-pipe
-  // polynomial (measured best: 3 next to the cheaper FP4 QK^T, 4 with FP8)
+  // polynomial (measured best with the row-split softmax: 5)
   static constexpr int kPolyPairs = FP4 ? FPATTN_POLY_FP4 : FPATTN_POLY_FP8;
   static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
   // P buffers, 32 columns each (128 E4M3 keys), as many as K/V stages when
@@ -422,8 +417,6 @@ __device__ __forceinline__ float exp_pack32_fp4(const uint32_t (&r)[32], float c
 // Every lane polls the barrier (one broadcast shared-memory access per poll),
 // so the warp never diverges around the wait.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
-  // a phase that has already completed is seen by one non-blocking test
-  if (kTestFirst && __all_sync(0xffffffffu, mbar_test_wait(smem_u32(bar), parity))) return true;
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err, code));
 }
 
