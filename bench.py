@@ -318,6 +318,25 @@ def choose_peak(peaks: dict, clk: dict, timed_s: float, qk: str, pv: str):
     return peak, peak * peaks["bf16_tflops"] / bf16, bf16, sustained, capped
 
 
+# Softmax cycles per 128x128 block and SM: MUFU 16,384 * 11/16 / 16 = 704
+# (5 of 16 exp2 pairs on the FMA-pipe polynomial), issue slots ~725 (about
+# 2,900 warp instructions at one a clock per sub-partition). The larger binds.
+SOFTMAX_CYCLES_PER_BLOCK = 725.0
+
+
+def alu_roofline(w: workloads.Workload, achieved_tflops: float, peaks: dict) -> dict:
+    """The attention kernel against its ALU-side bound: the exponentials of
+    a 128x128 block take SOFTMAX_CYCLES_PER_BLOCK cycles of an SM whatever d
+    is, so the bound in TFLOP/s is 4*128*128*d flops per block over that
+    time on every SM at the maximum clock."""
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    peak = 4.0 * 128 * 128 * w.d * 148 * mhz * 1e6 / SOFTMAX_CYCLES_PER_BLOCK / 1e12
+    return {"bound": "alu", "achieved": achieved_tflops, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved_tflops / peak,
+            "peak_source": f"derived: {SOFTMAX_CYCLES_PER_BLOCK:.0f} cycles of softmax work per 128x128 block "
+                           f"and SM (MUFU ex2 and issue counts), 148 SMs at {mhz:.0f} MHz"}
+
+
 def rank_env():
     """(world, rank, local_rank) from the torchrun environment (1, 0, 0 if absent)."""
     return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
@@ -650,6 +669,7 @@ def main():
                                         f"x nominal fp8 2x / fp4 4x; QK "
                                         f"{'fp4' if w.qk_format == 'nvfp4' else 'fp8'}, PV "
                                         f"{'fp4' if args.pv_format == 'nvfp4' else 'fp8'}, harmonic mean"},
+            "alu_roofline": alu_roofline(w, attn_tflops, peaks),
             "accuracy": accuracy, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk, "device_error": err,
         }

@@ -319,6 +319,39 @@ fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, in
                               size_t col_cap, int32_t* nblk_q_out, int32_t* nnz_out);
 
 /*
+ * HOST-only, no CUDA call: the schedule fpattn_fwd uses for a causal launch
+ * without a tile mask over bh = B*H (batch, head) problems of n tokens with
+ * head dimension d (64 or 128), Q/K in qk_dtype and V in pv_dtype
+ * (FPATTN_NVFP4 or FPATTN_E4M3), on a device with sm_count SMs.
+ *
+ * The kernel's work items are (head, 128-query block) pairs, taken longest
+ * row first (causal rows of later blocks attend more keys) and dealt to the
+ * *ctas persistent CTAs in a snake order (CTA 0..C-1 on even rounds, C-1..0
+ * on odd ones; position r*C + c or r*C + C-1-c). With every head in one
+ * group the same query block of all heads is in flight together, so the K/V
+ * of all heads pass through the L2 at once. The library therefore groups the
+ * heads so that one group's K and V bytes fit in a 32 MiB share of the L2,
+ * the groups following one another, and pads each group's positions to
+ * whole pairs of snake rounds so that every group is dealt evenly; a group
+ * size is used only when the padded schedule is modelled within 0.5% of the
+ * ungrouped one's balance. This is the library's own scheduling, not a step
+ * of the pages' method; results are identical either way.
+ *
+ * Outputs: *heads_per_group (= bh when not grouped), *group_positions
+ * (positions of a full group, items plus padding; bh*nblk when not grouped)
+ * and *positions (all positions of the launch). Position p of group
+ * p / group_positions holds an item when its offset in the group is below
+ * group_heads*nblk (group_heads = heads of that group); that item is head
+ * group*heads_per_group + offset % group_heads, query block
+ * nblk - 1 - offset / group_heads. Sizes out of fpattn_fwd's range give
+ * FPATTN_ERR_UNSUPPORTED; non-positive sizes, other dtypes or NULL outputs
+ * FPATTN_ERR_INVALID_ARG.
+ */
+fpattn_status fpattn_causal_plan(int64_t bh, int64_t n, int32_t d, int32_t qk_dtype, int32_t pv_dtype,
+                                 int32_t sm_count, int32_t* heads_per_group, int32_t* group_positions,
+                                 int32_t* positions, int32_t* ctas);
+
+/*
  * Fused quantized attention forward.
  *
  * q, k        both FPATTN_NVFP4 (QK^T on block-scaled FP4 tensor cores) or

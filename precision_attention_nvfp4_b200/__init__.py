@@ -42,7 +42,7 @@ from ._lib import FpattnError
 __all__ = ["Nvfp4Tensor", "Nvfp4VTensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_qkv",
            "quantize_nvfp4_v", "quantize_fp8", "sta_plan",
            "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError",
-           "head_range", "tensor_amax"]
+           "head_range", "tensor_amax", "causal_plan"]
 
 
 def library() -> ctypes.CDLL:
@@ -291,6 +291,20 @@ def sta_plan(tile_grid: Sequence[int], tile: Sequence[int], window: Sequence[int
     return StaPlan(row_ptr, col_idx[:nnz.value], row_order)
 
 
+def causal_plan(num_heads: int, N: int, d: int, qk_format: str = "nvfp4", pv_format: str = "fp8",
+                sm_count: int = 148) -> dict:
+    """Schedule of a causal attention launch over num_heads (batch, head)
+    problems (host-only): heads per group, schedule positions of a full group
+    and of the launch, and the CTA count. The heads are grouped so that one
+    group's K/V stay in L2; the output does not depend on it."""
+    fmt = {"nvfp4": 2, "fp8": 1, "e4m3": 1}
+    vals = [ctypes.c_int32(0) for _ in range(4)]
+    _lib.check(library().fpattn_causal_plan(int(num_heads), int(N), int(d), fmt[qk_format], fmt[pv_format],
+                                            int(sm_count), *(ctypes.byref(v) for v in vals)),
+               "fpattn_causal_plan")
+    return dict(zip(("heads_per_group", "group_positions", "positions", "ctas"), (v.value for v in vals)))
+
+
 def step_phase(t: int, num_steps: int, alpha1: float = 0.2, alpha2: float = 0.7) -> int:
     """Denoising phase of step t (1-based): 0 early, 1 middle, 2 late."""
     ph = ctypes.c_int32(0)
@@ -438,16 +452,18 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
 
 
 def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, return_lse, device, out_host,
-                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: int = 4):
+                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: int = 8):
     """attention() for host inputs: the (batch, head) problems are split into
     ``chunks`` contiguous groups, and the copies in, the kernels and the
     copies out of different groups overlap on three streams. Q and K are
     copied first: an NVFP4 tensor scale needs the amax over every head, so
-    their amax pass runs as each group lands, and each group is quantized
-    with the finished amax (the bits of the one-shot call). V is copied after
-    them, group by group, and each group's quantize + attention + copy back
-    starts as soon as its V has landed. With FP8 Q/K and V (no tensor-wide
-    amax) each group's Q, K, V are copied together."""
+    their amax pass runs as each group lands, and every group's Q and K are
+    quantized as soon as the amax is complete (the bits of the one-shot
+    call). V is copied after them, group by group, and each group's V
+    quantize + attention + copy back starts as soon as its V has landed; the
+    copies back then run while the rest of V comes in, so small groups keep
+    the tail after the last input byte short. With FP8 Q/K and V (no
+    tensor-wide amax) each group's Q, K, V are copied together."""
     dev = torch.device(device or "cuda:0")
     B, H, N, d = q.shape
     if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
@@ -499,17 +515,24 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
             cur.wait_event(ev_v[i])
             tensor_amax(part(vd, a, b), amax_v, accumulate=i > 0)
     s_out.wait_stream(cur)
+
+    def quantize_qk(i, a, b):
+        qc, kc = part(qd, a, b), part(kd, a, b)
+        if qk_format == "nvfp4":
+            return (quantize_nvfp4(qc, static_amax=amax_q, video=video),
+                    quantize_nvfp4(kc, static_amax=amax_k, video=video))
+        gran = "group" if qk_group_tiles > 1 else "tile128"
+        return (quantize_fp8(qc, gran, video=video, group_tiles=qk_group_tiles),
+                quantize_fp8(kc, gran, video=video, group_tiles=qk_group_tiles))
+
+    # with a tensor-wide Q/K amax every group's Q/K can be quantized as soon
+    # as the amax is done, ahead of the V copies; otherwise group by group
+    qk_ready = [quantize_qk(i, a, b) for i, (a, b) in enumerate(spans)] if qk_format == "nvfp4" else None
     for i, (a, b) in enumerate(spans):
         cur.wait_event(ev_qk[i])
         cur.wait_event(ev_v[i])
-        qc, kc, vc = part(qd, a, b), part(kd, a, b), part(vd, a, b)
-        if qk_format == "nvfp4":
-            qq, kq = quantize_nvfp4(qc, static_amax=amax_q, video=video), quantize_nvfp4(kc, static_amax=amax_k,
-                                                                                        video=video)
-        else:
-            gran = "group" if qk_group_tiles > 1 else "tile128"
-            qq = quantize_fp8(qc, gran, video=video, group_tiles=qk_group_tiles)
-            kq = quantize_fp8(kc, gran, video=video, group_tiles=qk_group_tiles)
+        qq, kq = qk_ready[i] if qk_ready is not None else quantize_qk(i, a, b)
+        vc = part(vd, a, b)
         if pv_format == "fp8":
             vq = quantize_fp8(vc, "channel", video=video)
         else:

@@ -303,6 +303,28 @@ fpattn_status fpattn_step_phase(int32_t t, int32_t num_steps, double alpha1, dou
   return FPATTN_OK;
 }
 
+fpattn_status fpattn_causal_plan(int64_t bh, int64_t n, int32_t d, int32_t qk_dtype, int32_t pv_dtype,
+                                 int32_t sm_count, int32_t* heads_per_group, int32_t* group_positions,
+                                 int32_t* positions, int32_t* ctas) {
+  if (!heads_per_group || !group_positions || !positions || !ctas) return FPATTN_ERR_INVALID_ARG;
+  if (bh <= 0 || n <= 0 || sm_count <= 0) return FPATTN_ERR_INVALID_ARG;
+  if ((qk_dtype != FPATTN_NVFP4 && qk_dtype != FPATTN_E4M3) || (pv_dtype != FPATTN_NVFP4 && pv_dtype != FPATTN_E4M3))
+    return FPATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FPATTN_ERR_UNSUPPORTED;
+  const long long nblk = (n + 127) / 128;
+  if (bh > 65535 || bh * nblk > (1ll << 30) || n > (1 << 28)) return FPATTN_ERR_UNSUPPORTED;
+  const int items = static_cast<int>(bh * nblk);
+  const int grid = items < sm_count ? items : sm_count;
+  int hg = 0, gs = 0, total = 0;
+  fpattn::causal_plan(static_cast<int>(bh), static_cast<int>(n), d, qk_dtype == FPATTN_NVFP4,
+                      pv_dtype == FPATTN_NVFP4, grid, &hg, &gs, &total);
+  *heads_per_group = hg;
+  *group_positions = gs;
+  *positions = total;
+  *ctas = grid;
+  return FPATTN_OK;
+}
+
 fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, int32_t th, int32_t tw, int32_t wt,
                               int32_t wh, int32_t ww, int32_t* row_ptr, int32_t* col_idx, int32_t* row_order,
                               size_t col_cap, int32_t* nblk_q_out, int32_t* nnz_out) {

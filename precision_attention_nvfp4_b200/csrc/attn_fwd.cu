@@ -53,7 +53,9 @@
 // dependent launch) only after its prologue.
 // Work items are (batch*head, 128-query block); causal runs schedule the
 // longest query blocks first, tile-mask runs follow the mask's row order.
+#include <algorithm>
 #include <atomic>
+#include <climits>
 #include <cfloat>
 #include <cstdint>
 #include <cstdio>
@@ -61,6 +63,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <mutex>
+#include <vector>
 
 #include "fpattn_internal.h"
 #include "sm100.cuh"
@@ -104,9 +108,6 @@ static_assert(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax <= 655
 #define FPATTN_ROW_SPLIT 1
 #endif
 constexpr bool kRowSplit = FPATTN_ROW_SPLIT != 0;
-#ifndef FPATTN_CAUSAL_GROUP_MB
-#define FPATTN_CAUSAL_GROUP_MB 0
-#endif
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_6 = 2.584962500721156f;    // log2(6)
@@ -210,9 +211,11 @@ struct __align__(64) Params {
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const int32_t* row_order;
-  int N, nblk, BH, num_items;
-  int nnz;     // tile mask entries (sparse runs)
-  int hgroup;  // causal runs: heads scheduled together (longest rows first within a group)
+  int N, nblk, BH;
+  int num_items;  // schedule positions: the items, plus the padding of causal head groups
+  int nnz;        // tile mask entries (sparse runs)
+  int hgroup;     // causal runs: heads scheduled together (longest rows first within a group)
+  int gspan;      // causal runs: schedule positions of a full group (items + padding)
   int causal, sparse;
   float sm_scale_log2;
   float tau;           // conditional-rescale threshold, log2 units (0: exact running max)
@@ -224,12 +227,31 @@ struct KList {
   int begin, count;
 };
 
-// Work item of this CTA in scheduling round r: a snake over the CTAs (forward
-// on even rounds, backward on odd ones) so that with items sorted longest
-// first every CTA gets a near-equal share.
+// Schedule position of this CTA in scheduling round r: a snake over the CTAs
+// (forward on even rounds, backward on odd ones) so that with items sorted
+// longest first every CTA gets a near-equal share.
 __device__ __forceinline__ int sched_item(int r) {
   return r * gridDim.x + ((r & 1) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
                                   : static_cast<int>(blockIdx.x));
+}
+
+// Whether schedule position `pos` holds an item. Only causal head groups are
+// padded: each group's items are followed by empty positions up to a whole
+// number of snake round pairs, so every group is spread evenly over the CTAs.
+__device__ __forceinline__ bool item_present(const Params& p, int pos) {
+  if (p.sparse || !p.causal) return true;
+  const int grp = pos / p.gspan;
+  const int gsz = min(p.hgroup, p.BH - grp * p.hgroup);
+  return pos - grp * p.gspan < gsz * p.nblk;
+}
+
+// First position at or after round `rnd` that holds an item (rnd advances to
+// its round), or a position >= p.num_items when there is none. A CTA's
+// positions grow with the round, so every role of the CTA walks the same list.
+__device__ __forceinline__ int next_item(const Params& p, int& rnd) {
+  int pos = sched_item(rnd);
+  while (pos < p.num_items && !item_present(p, pos)) pos = sched_item(++rnd);
+  return pos;
 }
 
 // The tile mask's arrays come from the caller: the host entry points check
@@ -246,10 +268,9 @@ __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, 
     if (static_cast<unsigned>(qb) >= static_cast<unsigned>(p.nblk)) qb = 0;
   } else if (p.causal) {
     // longest rows first within groups of p.hgroup heads whose K/V fit in
-    // part of the L2; the groups follow one another
-    const int span = p.hgroup * p.nblk;  // items of a full group
-    const int grp = item / span;
-    const int r = item - grp * span;
+    // part of the L2; the groups follow one another (item_present is true)
+    const int grp = item / p.gspan;
+    const int r = item - grp * p.gspan;
     const int gsz = min(p.hgroup, p.BH - grp * p.hgroup);
     qb = p.nblk - 1 - r / gsz;
     bh = grp * p.hgroup + r % gsz;
@@ -545,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
       int g = 0, it = 0;
       bool ok = true;
-      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+      for (int rnd = 0, item = next_item(p, rnd); item < p.num_items && ok; ++rnd, item = next_item(p, rnd), ++it) {
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
@@ -585,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       constexpr uint32_t kIdescPV = PV4 ? idesc_nvf4(128, D) : idesc_e4m3(128, D, true);
       int g = 0;
       bool ok = true;
-      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd)) {
+      for (int rnd = 0, item = next_item(p, rnd); item < p.num_items && ok; ++rnd, item = next_item(p, rnd)) {
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
@@ -641,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const uint64_t q_desc = make_smem_desc(smem_u32(smem + C::kOffQ), 16, C::kQKSbo, C::kQKSwz);
       int g = 0, it = 0;
       bool ok = true;
-      for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+      for (int rnd = 0, item = next_item(p, rnd); item < p.num_items && ok; ++rnd, item = next_item(p, rnd), ++it) {
         int bh, qb;
         decode_item(p, item, bh, qb);
         const KList L = key_list(p, qb);
@@ -712,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32 + w * 16) << 16;
     int g = 0, it = 0;
     bool ok = true;
-    for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+    for (int rnd = 0, item = next_item(p, rnd); item < p.num_items && ok; ++rnd, item = next_item(p, rnd), ++it) {
       int bh, qb;
       decode_item(p, item, bh, qb);
       const KList L = key_list(p, qb);
@@ -819,7 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     int g = 0, it = 0;
     bool ok = true;
-    for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+    for (int rnd = 0, item = next_item(p, rnd); item < p.num_items && ok; ++rnd, item = next_item(p, rnd), ++it) {
       int bh, qb;
       decode_item(p, item, bh, qb);
       const KList L = key_list(p, qb);
@@ -937,7 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t o_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::kColO;
     int g = 0, it = 0;
     bool ok = true;
-    for (int rnd = 0, item = sched_item(0); item < p.num_items && ok; item = sched_item(++rnd), ++it) {
+    for (int rnd = 0, item = next_item(p, rnd); item < p.num_items && ok; ++rnd, item = next_item(p, rnd), ++it) {
       int bh, qb;
       decode_item(p, item, bh, qb);
       const KList L = key_list(p, qb);
@@ -1205,19 +1226,12 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   p.BH = BH;
   p.num_items = BH * p.nblk;
   p.causal = a.causal ? 1 : 0;
-  {
-    // Causal runs order the items longest row first; with every head in one
-    // group (the default), the same query block of all heads is in flight at
-    // once and all heads' K/V cycle through the L2. FPATTN_CAUSAL_GROUP_MB > 0
-    // groups the heads so that a group's K and V (codes and scales) take
-    // about that many MB of L2 (40 measured 5% slower on the LLM prefill).
-    const double kv_head = static_cast<double>(a.N) * (C::kQKRow + C::kSF / 128.0 + (PV4 ? D / 2.0 : D));
-    const double budget = FPATTN_CAUSAL_GROUP_MB * 1024.0 * 1024.0;
-    p.hgroup = budget > 0 ? static_cast<int>(budget / kv_head) : BH;
-    if (p.hgroup < 1) p.hgroup = 1;
-    if (p.hgroup > BH) p.hgroup = BH;
-  }
   p.sparse = a.row_ptr ? 1 : 0;
+  const int sms = device_sm_count();
+  const int grid = p.num_items < sms ? p.num_items : sms;
+  p.hgroup = BH;
+  p.gspan = p.num_items;
+  if (p.causal && !p.sparse) causal_plan(BH, a.N, D, FP4, PV4, grid, &p.hgroup, &p.gspan, &p.num_items);
   p.nnz = a.nnz;
   p.sm_scale_log2 = a.softmax_scale * 1.4426950408889634f;
   p.tau = a.rescale_threshold;
@@ -1245,13 +1259,110 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
     if (fa.numRegs * kThreads < static_cast<int>(128 * (kRegsControl + kRegsCorrection) + 256 * kRegsSoftmax))
       return cudaErrorInvalidConfiguration;
   }
-  const int sms = device_sm_count();
-  const int grid = p.num_items < sms ? p.num_items : sms;
   const cudaError_t e = launch_pdl(attn_fwd_kernel<D, FP4, PV4>, dim3(grid), dim3(kThreads), C::kSmemRequest, st, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
+
+// L2 share for the K/V of one causal head group: 32 MiB of the 126 MB L2 (the
+// LLM prefill's 37-head groups read each K/V byte from DRAM once; with all
+// 128 heads in flight, five times).
+#ifndef FPATTN_CAUSAL_GROUP_MB
+#define FPATTN_CAUSAL_GROUP_MB 32
+#endif
+constexpr double kCausalGroupBytes = FPATTN_CAUSAL_GROUP_MB * 1024.0 * 1024.0;
+
+namespace {
+
+// Schedule positions of a causal head group of n items: rounded up to whole
+// pairs of snake rounds over `grid` CTAs.
+long long padded_span(long long n, int grid) {
+  const long long pair = 2LL * grid;
+  return (n + pair - 1) / pair * pair;
+}
+
+// Makespan of the causal snake schedule with heads in groups of g (padded
+// unless one group holds every head), in 128x128 blocks with one block of
+// per-item cost added; `load` is scratch for the per-CTA sums.
+double causal_makespan(int BH, int nblk, int g, int grid, std::vector<double>& load) {
+  load.assign(grid, 0.0);
+  long long pos = 0;
+  for (int g0 = 0; g0 < BH; g0 += g) {
+    const int gsz = std::min(g, BH - g0);
+    const long long n = static_cast<long long>(gsz) * nblk;
+    for (long long r = 0; r < n; ++r) {
+      const long long at = pos + r;
+      const long long rnd = at / grid;
+      const int c = static_cast<int>(at % grid);
+      load[(rnd & 1) ? grid - 1 - c : c] += static_cast<double>(nblk - r / gsz) + 1.0;
+    }
+    pos += g >= BH ? n : padded_span(n, grid);
+  }
+  return *std::max_element(load.begin(), load.end());
+}
+
+// Heads per group of the causal schedule. Longest rows first over all heads
+// puts the same query block of every head in flight at once, so the K/V of
+// all heads pass through the L2 together. Groups whose K and V (codes and
+// scales, kv_head bytes a head) fit in kCausalGroupBytes keep that
+// working set in L2; a group size is taken only if its padded schedule is
+// within 0.5% of the ungrouped one's balance (modelled on the host, once per
+// shape), else all heads form one group.
+int causal_head_group(int BH, int nblk, int grid, double kv_head) {
+  const double budget = kCausalGroupBytes;
+  if (budget <= 0.0 || kv_head <= 0.0) return BH;
+  const double fit = budget / kv_head;
+  if (fit >= BH) return BH;
+  const int gmax = fit < 1.0 ? 1 : static_cast<int>(fit);
+  struct Entry { int BH, nblk, grid, gmax, g; };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (e.BH == BH && e.nblk == nblk && e.grid == grid && e.gmax == gmax) return e.g;
+  }
+  std::vector<double> load;
+  const double base = causal_makespan(BH, nblk, BH, grid, load);
+  int best = BH;
+  double best_m = base * 1.005;
+  // at most 64 sizes, largest first; a smaller group must beat a larger one
+  // by 0.1% to be taken
+  for (int g = gmax, tried = 0; g >= 1 && tried < 64; --g, ++tried) {
+    const double m = causal_makespan(BH, nblk, g, grid, load);
+    if (m <= best_m && (best == BH || m < best_m * 0.999)) {
+      best = g;
+      best_m = m;
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 64) cache.erase(cache.begin());
+  cache.push_back(Entry{BH, nblk, grid, gmax, best});
+  return best;
+}
+
+}  // namespace
+
+void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, int* hgroup, int* gspan,
+                 int* num_items) {
+  const int nblk = (N + 127) / 128;
+  *hgroup = BH;
+  *gspan = BH * nblk;
+  *num_items = BH * nblk;
+  if (BH < 1 || nblk < 1 || grid < 1) return;
+  // K codes and block scales, V codes: the bytes of one head's keys
+  const double kv_head = static_cast<double>(N) * ((qk_fp4 ? D / 2.0 + D / 16.0 : D) + (pv_fp4 ? D / 2.0 : D));
+  const int g = causal_head_group(BH, nblk, grid, kv_head);
+  if (g >= BH) return;
+  const long long span = padded_span(static_cast<long long>(g) * nblk, grid);
+  const int rest = BH % g;
+  const long long total = (BH / g) * span + (rest ? padded_span(static_cast<long long>(rest) * nblk, grid) : 0);
+  if (total > INT_MAX / 2) return;  // keep positions in int range: one group, no padding
+  *hgroup = g;
+  *gspan = static_cast<int>(span);
+  *num_items = static_cast<int>(total);
+}
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {
   if (a.pv_fp4) {

@@ -119,6 +119,12 @@ struct AttnArgs {
 // unavailable, other errors as produced by the CUDA runtime.
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st);
 
+// Causal schedule of an attention launch over BH (batch, head) problems of N
+// tokens on `grid` CTAs: heads per group, schedule positions of a full group
+// and of the whole launch (items plus the padding of each group). Host only.
+void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, int* hgroup, int* gspan,
+                 int* num_items);
+
 // Device error word access (defined next to the kernels).
 cudaError_t read_device_error(cudaStream_t st, int clear, int* code);
 

@@ -1,0 +1,48 @@
+"""Causal launches whose heads the library schedules in L2-sized groups.
+
+Output and LSE start as NaN, so a (head, query block) item the grouped
+schedule failed to deal would stay NaN; sampled rows of the first head, a
+middle one and one in the partial last group are checked against the oracle.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import precision_attention_nvfp4_b200 as fp
+import workloads
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,H,N,fmt", [(4, 32, 4096, "nvfp4"), (16, 64, 2048, "nvfp4"), (8, 64, 2048, "fp8")])
+def test_grouped_causal_schedule_covers_every_item(B, H, N, fmt):
+    d = 128
+    plan = fp.causal_plan(B * H, N, d, fmt, "fp8", sm_count=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan["heads_per_group"] < B * H, plan  # the grouped path is the one under test
+    w = workloads.Workload("t", B=B, H=H, N=N, d=d, causal=True, qk_format=fmt, seed=21)
+    q, k, v = workloads.make_qkv(w)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    if fmt == "nvfp4":
+        qq, kq = fp.quantize_nvfp4(qc), fp.quantize_nvfp4(kc)
+    else:
+        qq, kq = fp.quantize_fp8(qc, "tile128"), fp.quantize_fp8(kc, "tile128")
+    vq = fp.quantize_fp8(vc, "channel")
+    out = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device="cuda")
+    fp.attention_fwd(qq, kq, vq, causal=True, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert fp.device_error() == 0
+    assert not torch.isnan(out).any().item()
+    assert not torch.isnan(lse).any().item()
+    G = plan["heads_per_group"]
+    heads = [0, (B * H) // 2, (B * H // G) * G if (B * H) % G else B * H - 1]
+    nblk = N // 128
+    rows = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in (0, nblk // 2, nblk - 1)])
+    o = out.float().cpu().numpy().reshape(B * H, N, d)
+    ls = lse.cpu().numpy().reshape(B * H, N)
+    qh, kh, vh = parity.oracle_operands(q, k, v, fmt, heads)
+    for i, bh in enumerate(heads):
+        res = parity.compare_attention(o[bh], ls[bh], qh[i], kh[i], vh[i], rows, causal=True)
+        parity.assert_close(res, f"{fmt} B{B} H{H} N{N} head {bh}")
