@@ -408,7 +408,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
               return_lse: bool = True, device: Optional[torch.device] = None,
               out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None,
               video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0,
-              qk_group_tiles: int = 1, pv_format: str = "fp8"):
+              qk_group_tiles: int = 1, pv_format: str = "fp8", host_chunks: Optional[int] = None):
     """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
 
     ``qk_group_tiles`` > 1 (FP8 Q/K only) shares one Q/K scale across that
@@ -421,7 +421,9 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
     host memory, into ``out_host`` / ``lse_host`` when given (pinned buffers
     the caller reuses), else into new pinned tensors; the copies of one group
     of heads overlap the kernels of another (see _attention_host), and the
-    call returns once the results are in host memory.
+    call returns once the results are in host memory. ``host_chunks`` sets
+    the number of head groups of that pipeline (default: about 8 MiB of V a
+    group, at most 16); the results do not depend on it.
     """
     if qk_format not in ("nvfp4", "fp8"):
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
@@ -432,7 +434,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
                                softmax_scale=softmax_scale, return_lse=return_lse, device=device,
                                out_host=out_host, lse_host=lse_host, video=video,
                                rescale_threshold=rescale_threshold, qk_group_tiles=qk_group_tiles,
-                               pv_format=pv_format)
+                               pv_format=pv_format, chunks=host_chunks)
     if qk_format not in ("nvfp4", "fp8"):
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
     if pv_format not in ("fp8", "nvfp4"):
@@ -452,7 +454,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
 
 
 def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, return_lse, device, out_host,
-                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: int = 8):
+                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: Optional[int] = None):
     """attention() for host inputs: the (batch, head) problems are split into
     ``chunks`` contiguous groups, and the copies in, the kernels and the
     copies out of different groups overlap on three streams. Q and K are
@@ -463,13 +465,19 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
     quantize + attention + copy back starts as soon as its V has landed; the
     copies back then run while the rest of V comes in, so small groups keep
     the tail after the last input byte short. With FP8 Q/K and V (no
-    tensor-wide amax) each group's Q, K, V are copied together."""
+    tensor-wide amax) each group's Q, K, V are copied together. By default a
+    group holds about 8 MiB of V (at most 16 groups): enough groups to keep
+    the tail short, few enough that the host's enqueue work stays hidden
+    behind the Q/K copies."""
     dev = torch.device(device or "cuda:0")
     B, H, N, d = q.shape
     if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
         raise ValueError("q, k, v must have one shape")
     BH = B * H
-    spans = [s for s in (head_range(BH, min(chunks, BH), r) for r in range(min(chunks, BH))) if s[1] > s[0]]
+    if chunks is None:
+        chunks = max(1, min(16, (BH * N * d * 2) >> 23))
+    chunks = max(1, min(int(chunks), BH))
+    spans = [s for s in (head_range(BH, chunks, r) for r in range(chunks)) if s[1] > s[0]]
     flat = [t.reshape(BH, N, d) for t in (q, k, v)]
     cur = torch.cuda.current_stream(dev)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)

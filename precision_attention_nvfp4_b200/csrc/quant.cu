@@ -256,20 +256,40 @@ __device__ __forceinline__ void fp8_channel_quant_body(const uint4* __restrict__
     if (r0 + static_cast<int>(threadIdx.x) < rend) src_row[threadIdx.x] = to_raster(tmap, r0 + threadIdx.x);
     __syncthreads();
   }
+  // four rows' loads are issued before any of them is converted, so that a
+  // thread keeps 64 bytes in flight
+  constexpr int kBatch = 4;
+  uint4 v[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int ru = r0 + rr + u * kRowsPerIter;
+    v[u] = ru < rend ? x[(bh * N + (kMap ? src_row[ru - r0] : ru)) * kCpr + cg] : make_uint4(0u, 0u, 0u, 0u);
+  }
   float s[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) s[i] = fp8_scale_from_amax(amax[bh * D + cg * 8 + i]);
-  for (int r = r0 + rr; r < rend; r += kRowsPerIter) {
-    const size_t idx = (bh * N + r) * kCpr + cg;
-    const uint4 v = kMap ? x[(bh * N + src_row[r - r0]) * kCpr + cg] : x[idx];
-    float f[8];
-    unpack8(v, f);
-    uint2 o;
-    o.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[0], s[0]), __fmul_rn(f[1], s[1]))) |
-          (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[2], s[2]), __fmul_rn(f[3], s[3]))) << 16);
-    o.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[4], s[4]), __fmul_rn(f[5], s[5]))) |
-          (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[6], s[6]), __fmul_rn(f[7], s[7]))) << 16);
-    codes[idx] = o;
+  for (int r = r0 + rr; r < rend; r += kBatch * kRowsPerIter) {
+    uint4 nxt[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int ru = r + (kBatch + u) * kRowsPerIter;
+      nxt[u] = ru < rend ? x[(bh * N + (kMap ? src_row[ru - r0] : ru)) * kCpr + cg] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int ru = r + u * kRowsPerIter;
+      if (ru < rend) {
+        float f[8];
+        unpack8(v[u], f);
+        uint2 o;
+        o.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[0], s[0]), __fmul_rn(f[1], s[1]))) |
+              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[2], s[2]), __fmul_rn(f[3], s[3]))) << 16);
+        o.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[4], s[4]), __fmul_rn(f[5], s[5]))) |
+              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(f[6], s[6]), __fmul_rn(f[7], s[7]))) << 16);
+        codes[(bh * N + ru) * kCpr + cg] = o;
+      }
+      v[u] = nxt[u];
+    }
   }
 }
 

@@ -1,8 +1,9 @@
 """attention() on host (pinned) inputs: the chunked pipeline that overlaps
 the copies with the kernels returns the same bits as the call on device
-inputs, for every format pair, for uneven groups of heads, with the
-sliding-tile mask on a raster-order video, and with the tensor-amax pass run
-piece by piece (the NVFP4 tensor scale of the whole tensor)."""
+inputs, for every format pair, for the default and for uneven groups of
+heads, with the sliding-tile mask on a raster-order video, and with the
+tensor-amax pass run piece by piece (the NVFP4 tensor scale of the whole
+tensor)."""
 import numpy as np
 import pytest
 import torch
@@ -19,13 +20,14 @@ def _pinned(*ts):
 
 @pytest.mark.parametrize("qk,pv", [("nvfp4", "fp8"), ("fp8", "fp8"), ("nvfp4", "nvfp4"), ("fp8", "nvfp4")])
 @pytest.mark.parametrize("causal", [False, True])
-def test_host_pipeline_equals_device_call(qk, pv, causal):
+@pytest.mark.parametrize("chunks", [None, 4])
+def test_host_pipeline_equals_device_call(qk, pv, causal, chunks):
     w = workloads.Workload("t", B=1, H=5, N=700, d=128, causal=causal, qk_format=qk, seed=31, outliers=True)
     q, k, v = workloads.make_qkv(w)
     ref_out, ref_lse = fp.attention(q.cuda(), k.cuda(), v.cuda(), qk_format=qk, causal=causal, pv_format=pv)
     torch.cuda.synchronize()
     qh, kh, vh = _pinned(q, k, v)
-    out, lse = fp.attention(qh, kh, vh, qk_format=qk, causal=causal, pv_format=pv)
+    out, lse = fp.attention(qh, kh, vh, qk_format=qk, causal=causal, pv_format=pv, host_chunks=chunks)
     assert not out.is_cuda and out.is_pinned()
     assert torch.equal(out.view(torch.int16), ref_out.cpu().view(torch.int16))
     assert torch.equal(lse.view(torch.int32), ref_lse.cpu().view(torch.int32))
@@ -45,7 +47,7 @@ def test_host_pipeline_video_sta_and_reused_buffers():
     lse_h = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)
     for _ in range(2):
         out, lse = fp.attention(qh, kh, vh, qk_format="fp8", tile_mask=mask, video=video, out_host=out_h,
-                                lse_host=lse_h)
+                                lse_host=lse_h, host_chunks=3)
         assert out.data_ptr() == out_h.data_ptr()
         assert torch.equal(out.view(torch.int16), ref_out.cpu().view(torch.int16))
         assert torch.equal(lse.view(torch.int32), ref_lse.cpu().view(torch.int32))
