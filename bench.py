@@ -599,6 +599,23 @@ def main():
         d2h = out_h.numel() * 2 + lse_h.numel() * 4
         e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        if w.qk_format == "nvfp4" and args.pv_format == "fp8":
+            # the static-amax form: a caller's Q/K amax (here the inputs' own,
+            # so the bits are those of the dynamic call) lets each group of
+            # heads be quantized as it lands
+            amax = (fp.tensor_amax(q), fp.tensor_amax(k))
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                fp.attention(qp, kp, vp, qk_format=w.qk_format, causal=w.causal, tile_mask=mask, out_host=out_h,
+                             lse_host=lse_h, video=video, rescale_threshold=args.rescale_threshold,
+                             pv_format=args.pv_format, qk_amax=amax)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            s_ms = rank_max(e0.elapsed_time(e1) / args.e2e_steps)
+            e2e["caller_amax"] = {"value": world * flops / (s_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                                  "ms_per_step": s_ms,
+                                  "note": "attention(..., qk_amax=(amax Q, amax K)) from the caller, same copies"}
 
     cpu, accuracy = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -322,34 +322,47 @@ fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, in
  * HOST-only, no CUDA call: the schedule fpattn_fwd uses for a causal launch
  * without a tile mask over bh = B*H (batch, head) problems of n tokens with
  * head dimension d (64 or 128), Q/K in qk_dtype and V in pv_dtype
- * (FPATTN_NVFP4 or FPATTN_E4M3), on a device with sm_count SMs.
+ * (FPATTN_NVFP4 or FPATTN_E4M3), on a device with sm_count SMs. This is the
+ * library's own scheduling, not a step of the pages' method: the results are
+ * the same under any schedule.
  *
- * The kernel's work items are (head, 128-query block) pairs, taken longest
- * row first (causal rows of later blocks attend more keys) and dealt to the
- * *ctas persistent CTAs in a snake order (CTA 0..C-1 on even rounds, C-1..0
- * on odd ones; position r*C + c or r*C + C-1-c). With every head in one
- * group the same query block of all heads is in flight together, so the K/V
- * of all heads pass through the L2 at once. The library therefore groups the
- * heads so that one group's K and V bytes fit in a 32 MiB share of the L2,
- * the groups following one another, and pads each group's positions to
- * whole pairs of snake rounds so that every group is dealt evenly; a group
- * size is used only when the padded schedule is modelled within 0.5% of the
- * ungrouped one's balance. This is the library's own scheduling, not a step
- * of the pages' method; results are identical either way.
+ * The kernel's work items are (head, 128-query block) pairs; a causal row of
+ * query block qb attends qb + 1 key blocks. *ctas persistent CTAs take them
+ * in one of two orders:
  *
- * Outputs: *heads_per_group (= bh when not grouped), *group_positions
- * (positions of a full group, items plus padding; bh*nblk when not grouped)
- * and *positions (all positions of the launch). Position p of group
- * p / group_positions holds an item when its offset in the group is below
- * group_heads*nblk (group_heads = heads of that group); that item is head
- * group*heads_per_group + offset % group_heads, query block
- * nblk - 1 - offset / group_heads. Sizes out of fpattn_fwd's range give
- * FPATTN_ERR_UNSUPPORTED; non-positive sizes, other dtypes or NULL outputs
- * FPATTN_ERR_INVALID_ARG.
+ * Longest first (*pairs_per_head = 0). Items are taken longest row first and
+ * dealt in a snake order (CTA 0..C-1 on even rounds, C-1..0 on odd ones:
+ * position r*C + c or r*C + C-1-c). Over all heads at once, the same query
+ * block of every head would be in flight together and the K/V of all heads
+ * would pass through the L2 at once, so the heads are grouped so that one
+ * group's K and V bytes fit in a 32 MiB share of the L2, the groups following
+ * one another, and each group's positions are padded to whole pairs of snake
+ * rounds so that every group is dealt evenly. A group size is used only when
+ * the padded schedule is modelled within 0.5% of the ungrouped one's balance.
+ * Position p of group p / group_positions holds an item when its offset in
+ * the group is below group_heads*nblk (group_heads = heads of that group);
+ * that item is head group*heads_per_group + offset % group_heads, query block
+ * nblk - 1 - offset / group_heads. Ungrouped: heads_per_group = bh and
+ * group_positions = bh*nblk.
+ *
+ * Pairs (*pairs_per_head = P = ceil(nblk/2) > 0), when no group size both
+ * fits and balances and the heads' K/V exceed four shares (the whole L2):
+ * pair j = h*P + i of
+ * head h holds query blocks nblk-1-i and i, which together always cover nblk
+ * + 1 key blocks, so pairs dealt round-robin (CTA c takes pairs c, c + C, ...)
+ * balance the CTAs, and the CTAs in flight work on a few consecutive heads.
+ * CTA c's round r is position 2*((r/2)*C + c) + r%2; position 2j is query
+ * block nblk-1-i of pair j and 2j+1 is block i, absent when both are the
+ * same block (the middle one of an odd nblk). Used only when modelled within
+ * 1.5% of the snake's balance.
+ *
+ * *positions receives the positions of the whole launch. Sizes out of
+ * fpattn_fwd's range give FPATTN_ERR_UNSUPPORTED; non-positive sizes, other
+ * dtypes or NULL outputs FPATTN_ERR_INVALID_ARG.
  */
 fpattn_status fpattn_causal_plan(int64_t bh, int64_t n, int32_t d, int32_t qk_dtype, int32_t pv_dtype,
                                  int32_t sm_count, int32_t* heads_per_group, int32_t* group_positions,
-                                 int32_t* positions, int32_t* ctas);
+                                 int32_t* pairs_per_head, int32_t* positions, int32_t* ctas);
 
 /*
  * Fused quantized attention forward.

@@ -294,15 +294,18 @@ def sta_plan(tile_grid: Sequence[int], tile: Sequence[int], window: Sequence[int
 def causal_plan(num_heads: int, N: int, d: int, qk_format: str = "nvfp4", pv_format: str = "fp8",
                 sm_count: int = 148) -> dict:
     """Schedule of a causal attention launch over num_heads (batch, head)
-    problems (host-only): heads per group, schedule positions of a full group
-    and of the launch, and the CTA count. The heads are grouped so that one
-    group's K/V stay in L2; the output does not depend on it."""
+    problems (host-only): heads per group and schedule positions of a full
+    group (longest-first order), pairs of query blocks per head (paired
+    order, else 0), all positions of the launch, and the CTA count. Either
+    order keeps the K/V in flight within the L2; the output does not depend
+    on it."""
     fmt = {"nvfp4": 2, "fp8": 1, "e4m3": 1}
-    vals = [ctypes.c_int32(0) for _ in range(4)]
+    vals = [ctypes.c_int32(0) for _ in range(5)]
     _lib.check(library().fpattn_causal_plan(int(num_heads), int(N), int(d), fmt[qk_format], fmt[pv_format],
                                             int(sm_count), *(ctypes.byref(v) for v in vals)),
                "fpattn_causal_plan")
-    return dict(zip(("heads_per_group", "group_positions", "positions", "ctas"), (v.value for v in vals)))
+    return dict(zip(("heads_per_group", "group_positions", "pairs_per_head", "positions", "ctas"),
+                    (v.value for v in vals)))
 
 
 def step_phase(t: int, num_steps: int, alpha1: float = 0.2, alpha2: float = 0.7) -> int:
@@ -408,7 +411,8 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
               return_lse: bool = True, device: Optional[torch.device] = None,
               out_host: Optional[torch.Tensor] = None, lse_host: Optional[torch.Tensor] = None,
               video: Optional[VideoLayout] = None, rescale_threshold: float = 0.0,
-              qk_group_tiles: int = 1, pv_format: str = "fp8", host_chunks: Optional[int] = None):
+              qk_group_tiles: int = 1, pv_format: str = "fp8", host_chunks: Optional[int] = None,
+              qk_amax: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
     """softmax(Q K^T * scale) V with quantized operands, from bf16 inputs.
 
     ``qk_group_tiles`` > 1 (FP8 Q/K only) shares one Q/K scale across that
@@ -424,26 +428,39 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
     call returns once the results are in host memory. ``host_chunks`` sets
     the number of head groups of that pipeline (default: about 8 MiB of V a
     group, at most 16); the results do not depend on it.
+
+    ``qk_amax`` (NVFP4 Q/K only): device float32 [1] tensors with the amax of
+    Q and of K, e.g. from calibration or ``tensor_amax``, used for the tensor
+    scales instead of the amax of these inputs (the static-amax form of the
+    NVFP4 recipe). With it, host inputs are quantized group by group as they
+    land, so the copies back start before all of Q and K are in.
     """
     if qk_format not in ("nvfp4", "fp8"):
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
     if pv_format not in ("fp8", "nvfp4"):
         raise ValueError("pv_format must be 'fp8' or 'nvfp4'")
+    if qk_amax is not None:
+        if qk_format != "nvfp4":
+            raise ValueError("qk_amax applies to NVFP4 Q/K only")
+        if len(qk_amax) != 2 or not all(isinstance(a, torch.Tensor) and a.is_cuda and a.dtype == torch.float32
+                                        and a.numel() >= 1 for a in qk_amax):
+            raise ValueError("qk_amax must be two CUDA float32 tensors (amax of Q, amax of K)")
     if not q.is_cuda:
         return _attention_host(q, k, v, qk_format=qk_format, causal=causal, tile_mask=tile_mask,
                                softmax_scale=softmax_scale, return_lse=return_lse, device=device,
                                out_host=out_host, lse_host=lse_host, video=video,
                                rescale_threshold=rescale_threshold, qk_group_tiles=qk_group_tiles,
-                               pv_format=pv_format, chunks=host_chunks)
+                               pv_format=pv_format, chunks=host_chunks, qk_amax=qk_amax)
     if qk_format not in ("nvfp4", "fp8"):
         raise ValueError("qk_format must be 'nvfp4' or 'fp8'")
     if pv_format not in ("fp8", "nvfp4"):
         raise ValueError("pv_format must be 'fp8' or 'nvfp4'")
-    if pv_format == "fp8" and qk_group_tiles <= 1:
+    if pv_format == "fp8" and qk_group_tiles <= 1 and qk_amax is None:
         qq, kq, vq = quantize_qkv(q, k, v, qk_format, video=video)   # four fused launches
     else:
         if qk_format == "nvfp4":
-            qq, kq = quantize_nvfp4(q, video=video), quantize_nvfp4(k, video=video)
+            aq, ak = qk_amax if qk_amax is not None else (None, None)
+            qq, kq = quantize_nvfp4(q, static_amax=aq, video=video), quantize_nvfp4(k, static_amax=ak, video=video)
         else:
             gran = "group" if qk_group_tiles > 1 else "tile128"
             qq = quantize_fp8(q, gran, video=video, group_tiles=qk_group_tiles)
@@ -454,7 +471,8 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
 
 
 def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, return_lse, device, out_host,
-                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: Optional[int] = None):
+                    lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: Optional[int] = None,
+                    qk_amax=None):
     """attention() for host inputs: the (batch, head) problems are split into
     ``chunks`` contiguous groups, and the copies in, the kernels and the
     copies out of different groups overlap on three streams. Q and K are
@@ -464,8 +482,9 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
     call). V is copied after them, group by group, and each group's V
     quantize + attention + copy back starts as soon as its V has landed; the
     copies back then run while the rest of V comes in, so small groups keep
-    the tail after the last input byte short. With FP8 Q/K and V (no
-    tensor-wide amax) each group's Q, K, V are copied together. By default a
+    the tail after the last input byte short. With FP8 Q/K and V, or a
+    caller's Q/K amax (no tensor-wide amax to wait for), each group's Q, K, V
+    are copied together and the group is quantized as it lands. By default a
     group holds about 8 MiB of V (at most 16 groups): enough groups to keep
     the tail short, few enough that the host's enqueue work stays hidden
     behind the Q/K copies."""
@@ -493,7 +512,7 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
     ev_qk, ev_v = [torch.cuda.Event() for _ in spans], [torch.cuda.Event() for _ in spans]
     # with no tensor-wide amax to wait for (FP8 Q/K and V), group i's Q, K, V
     # are copied together so its kernels can start right after them
-    interleave = qk_format == "fp8" and pv_format == "fp8"
+    interleave = pv_format == "fp8" and (qk_format == "fp8" or qk_amax is not None)
     with torch.cuda.stream(s_in):
         for i, (a, b) in enumerate(spans):
             qd[a:b].copy_(flat[0][a:b], non_blocking=True)
@@ -511,7 +530,9 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
         return t[a:b].view(1, b - a, N, d)
 
     amax_q = amax_k = amax_v = None
-    if qk_format == "nvfp4":
+    if qk_amax is not None:
+        amax_q, amax_k = (a.to(dev) for a in qk_amax)
+    elif qk_format == "nvfp4":
         amax_q, amax_k = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2))
         for i, (a, b) in enumerate(spans):
             cur.wait_event(ev_qk[i])
@@ -535,7 +556,8 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
 
     # with a tensor-wide Q/K amax every group's Q/K can be quantized as soon
     # as the amax is done, ahead of the V copies; otherwise group by group
-    qk_ready = [quantize_qk(i, a, b) for i, (a, b) in enumerate(spans)] if qk_format == "nvfp4" else None
+    qk_ready = ([quantize_qk(i, a, b) for i, (a, b) in enumerate(spans)]
+                if qk_format == "nvfp4" and qk_amax is None else None)
     for i, (a, b) in enumerate(spans):
         cur.wait_event(ev_qk[i])
         cur.wait_event(ev_v[i])

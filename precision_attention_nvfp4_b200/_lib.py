@@ -61,7 +61,7 @@ _SIGNATURES = {
     "fpattn_sta_plan": (ctypes.c_int, [ctypes.c_int32] * 9 + [ctypes.c_void_p] * 3 +
                         [ctypes.c_size_t, _P(ctypes.c_int32), _P(ctypes.c_int32)]),
     "fpattn_causal_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
-                                          ctypes.c_int32, ctypes.c_int32] + [_P(ctypes.c_int32)] * 4),
+                                          ctypes.c_int32, ctypes.c_int32] + [_P(ctypes.c_int32)] * 5),
     "fpattn_tile_mask_check": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                               ctypes.c_void_p]),
     "fpattn_fwd": (ctypes.c_int, [_P(Tensor), _P(Tensor), _P(Tensor), _P(Scales), _P(TileMask),

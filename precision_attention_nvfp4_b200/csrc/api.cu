@@ -305,8 +305,8 @@ fpattn_status fpattn_step_phase(int32_t t, int32_t num_steps, double alpha1, dou
 
 fpattn_status fpattn_causal_plan(int64_t bh, int64_t n, int32_t d, int32_t qk_dtype, int32_t pv_dtype,
                                  int32_t sm_count, int32_t* heads_per_group, int32_t* group_positions,
-                                 int32_t* positions, int32_t* ctas) {
-  if (!heads_per_group || !group_positions || !positions || !ctas) return FPATTN_ERR_INVALID_ARG;
+                                 int32_t* pairs_per_head, int32_t* positions, int32_t* ctas) {
+  if (!heads_per_group || !group_positions || !pairs_per_head || !positions || !ctas) return FPATTN_ERR_INVALID_ARG;
   if (bh <= 0 || n <= 0 || sm_count <= 0) return FPATTN_ERR_INVALID_ARG;
   if ((qk_dtype != FPATTN_NVFP4 && qk_dtype != FPATTN_E4M3) || (pv_dtype != FPATTN_NVFP4 && pv_dtype != FPATTN_E4M3))
     return FPATTN_ERR_INVALID_ARG;
@@ -315,12 +315,13 @@ fpattn_status fpattn_causal_plan(int64_t bh, int64_t n, int32_t d, int32_t qk_dt
   if (bh > 65535 || bh * nblk > (1ll << 30) || n > (1 << 28)) return FPATTN_ERR_UNSUPPORTED;
   const int items = static_cast<int>(bh * nblk);
   const int grid = items < sm_count ? items : sm_count;
-  int hg = 0, gs = 0, total = 0;
+  fpattn::CausalPlan cp;
   fpattn::causal_plan(static_cast<int>(bh), static_cast<int>(n), d, qk_dtype == FPATTN_NVFP4,
-                      pv_dtype == FPATTN_NVFP4, grid, &hg, &gs, &total);
-  *heads_per_group = hg;
-  *group_positions = gs;
-  *positions = total;
+                      pv_dtype == FPATTN_NVFP4, grid, &cp);
+  *heads_per_group = cp.hgroup;
+  *group_positions = cp.gspan;
+  *pairs_per_head = cp.hpairs;
+  *positions = cp.num_items;
   *ctas = grid;
   return FPATTN_OK;
 }

@@ -216,6 +216,7 @@ struct __align__(64) Params {
   int nnz;        // tile mask entries (sparse runs)
   int hgroup;     // causal runs: heads scheduled together (longest rows first within a group)
   int gspan;      // causal runs: schedule positions of a full group (items + padding)
+  int hpairs;     // causal runs in pairs (else 0): pairs of query blocks per head, ceil(nblk / 2)
   int causal, sparse;
   float sm_scale_log2;
   float tau;           // conditional-rescale threshold, log2 units (0: exact running max)
@@ -227,19 +228,26 @@ struct KList {
   int begin, count;
 };
 
-// Schedule position of this CTA in scheduling round r: a snake over the CTAs
-// (forward on even rounds, backward on odd ones) so that with items sorted
-// longest first every CTA gets a near-equal share.
-__device__ __forceinline__ int sched_item(int r) {
-  return r * gridDim.x + ((r & 1) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
-                                  : static_cast<int>(blockIdx.x));
+// Schedule position of this CTA in scheduling round r. Causal runs in pairs
+// (p.hpairs > 0): pair (r / 2) * C + CTA, its longer query block on even
+// rounds and its shorter one on odd rounds (position 2 * pair + r % 2); every
+// pair costs the same, so dealing them round-robin balances the CTAs. Else a
+// snake over the C CTAs (forward on even rounds, backward on odd ones), so
+// that with items sorted longest first every CTA gets a near-equal share.
+__device__ __forceinline__ int sched_item(const Params& p, int r) {
+  const int c = static_cast<int>(blockIdx.x), C = static_cast<int>(gridDim.x);
+  if (p.hpairs) return (((r >> 1) * C + c) << 1) | (r & 1);
+  return r * C + ((r & 1) ? C - 1 - c : c);
 }
 
-// Whether schedule position `pos` holds an item. Only causal head groups are
-// padded: each group's items are followed by empty positions up to a whole
-// number of snake round pairs, so every group is spread evenly over the CTAs.
+// Whether schedule position `pos` holds an item. In pairs, the middle block
+// of an odd count is its own partner, so its pair has no second item. Causal
+// head groups are padded: each group's items are followed by empty positions
+// up to a whole number of snake round pairs, so every group is spread evenly
+// over the CTAs.
 __device__ __forceinline__ bool item_present(const Params& p, int pos) {
   if (p.sparse || !p.causal) return true;
+  if (p.hpairs) return (pos & 1) == 0 || 2 * ((pos >> 1) % p.hpairs) + 1 != p.nblk;
   const int grp = pos / p.gspan;
   const int gsz = min(p.hgroup, p.BH - grp * p.hgroup);
   return pos - grp * p.gspan < gsz * p.nblk;
@@ -249,8 +257,8 @@ __device__ __forceinline__ bool item_present(const Params& p, int pos) {
 // its round), or a position >= p.num_items when there is none. A CTA's
 // positions grow with the round, so every role of the CTA walks the same list.
 __device__ __forceinline__ int next_item(const Params& p, int& rnd) {
-  int pos = sched_item(rnd);
-  while (pos < p.num_items && !item_present(p, pos)) pos = sched_item(++rnd);
+  int pos = sched_item(p, rnd);
+  while (pos < p.num_items && !item_present(p, pos)) pos = sched_item(p, ++rnd);
   return pos;
 }
 
@@ -266,6 +274,12 @@ __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, 
     bh = item % p.BH;
     qb = p.row_order ? p.row_order[r] : r;
     if (static_cast<unsigned>(qb) >= static_cast<unsigned>(p.nblk)) qb = 0;
+  } else if (p.hpairs) {
+    // pair j of head bh: query blocks nblk - 1 - i (even position) and i
+    const int j = item >> 1;
+    bh = j / p.hpairs;
+    const int i = j - bh * p.hpairs;
+    qb = (item & 1) ? i : p.nblk - 1 - i;
   } else if (p.causal) {
     // longest rows first within groups of p.hgroup heads whose K/V fit in
     // part of the L2; the groups follow one another (item_present is true)
@@ -1231,7 +1245,15 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   const int grid = p.num_items < sms ? p.num_items : sms;
   p.hgroup = BH;
   p.gspan = p.num_items;
-  if (p.causal && !p.sparse) causal_plan(BH, a.N, D, FP4, PV4, grid, &p.hgroup, &p.gspan, &p.num_items);
+  p.hpairs = 0;
+  if (p.causal && !p.sparse) {
+    CausalPlan cp;
+    causal_plan(BH, a.N, D, FP4, PV4, grid, &cp);
+    p.hgroup = cp.hgroup;
+    p.gspan = cp.gspan;
+    p.hpairs = cp.hpairs;
+    p.num_items = cp.num_items;
+  }
   p.nnz = a.nnz;
   p.sm_scale_log2 = a.softmax_scale * 1.4426950408889634f;
   p.tau = a.rescale_threshold;
@@ -1272,6 +1294,10 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
 #define FPATTN_CAUSAL_GROUP_MB 32
 #endif
 constexpr double kCausalGroupBytes = FPATTN_CAUSAL_GROUP_MB * 1024.0 * 1024.0;
+// 0 keeps every causal launch on the longest-first order
+#ifndef FPATTN_CAUSAL_PAIRS
+#define FPATTN_CAUSAL_PAIRS 1
+#endif
 
 namespace {
 
@@ -1344,24 +1370,54 @@ int causal_head_group(int BH, int nblk, int grid, double kv_head) {
 
 }  // namespace
 
-void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, int* hgroup, int* gspan,
-                 int* num_items) {
+// Paired order for the causal launch, if its modelled makespan is within
+// 1.5% of the ungrouped snake's; returns false (plan untouched) otherwise.
+static bool causal_pairs(int BH, int nblk, int grid, CausalPlan* plan) {
+  const int hp = (nblk + 1) / 2;
+  const long long pairs = static_cast<long long>(BH) * hp;
+  if (2 * pairs > INT_MAX / 2) return false;
+  std::vector<double> load;
+  const double base = causal_makespan(BH, nblk, BH, grid, load);
+  load.assign(grid, 0.0);
+  for (long long j = 0; j < pairs; ++j) {
+    const int i = static_cast<int>(j % hp);
+    const int lo = i, hi = nblk - 1 - i;
+    load[j % grid] += (hi + 2.0) + (hi != lo ? lo + 2.0 : 0.0);
+  }
+  if (*std::max_element(load.begin(), load.end()) > base * 1.015) return false;
+  plan->hpairs = hp;
+  plan->num_items = static_cast<int>(2 * pairs);
+  return true;
+}
+
+void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan) {
   const int nblk = (N + 127) / 128;
-  *hgroup = BH;
-  *gspan = BH * nblk;
-  *num_items = BH * nblk;
+  plan->hgroup = BH;
+  plan->gspan = BH * nblk;
+  plan->hpairs = 0;
+  plan->num_items = BH * nblk;
   if (BH < 1 || nblk < 1 || grid < 1) return;
   // K codes and block scales, V codes: the bytes of one head's keys
   const double kv_head = static_cast<double>(N) * ((qk_fp4 ? D / 2.0 + D / 16.0 : D) + (pv_fp4 ? D / 2.0 : D));
+  const bool over_l2 = BH * kv_head > 4 * kCausalGroupBytes;
+  if (FPATTN_CAUSAL_PAIRS == 2 && over_l2 && causal_pairs(BH, nblk, grid, plan)) return;
   const int g = causal_head_group(BH, nblk, grid, kv_head);
-  if (g >= BH) return;
-  const long long span = padded_span(static_cast<long long>(g) * nblk, grid);
-  const int rest = BH % g;
-  const long long total = (BH / g) * span + (rest ? padded_span(static_cast<long long>(rest) * nblk, grid) : 0);
-  if (total > INT_MAX / 2) return;  // keep positions in int range: one group, no padding
-  *hgroup = g;
-  *gspan = static_cast<int>(span);
-  *num_items = static_cast<int>(total);
+  if (g < BH) {
+    const long long span = padded_span(static_cast<long long>(g) * nblk, grid);
+    const int rest = BH % g;
+    const long long total = (BH / g) * span + (rest ? padded_span(static_cast<long long>(rest) * nblk, grid) : 0);
+    if (total > INT_MAX / 2) return;  // keep positions in int range: one group, no padding
+    plan->hgroup = g;
+    plan->gspan = static_cast<int>(span);
+    plan->num_items = static_cast<int>(total);
+    return;
+  }
+  // No group size both fits and balances (a head's K/V are large, or the
+  // groups leave ragged rounds). When the heads' K/V together exceed the
+  // whole L2 (four shares), pair the rows instead, head by head, so that the
+  // CTAs in flight share the K/V of a few heads. (Below that size the pairs
+  // measured ~3% slower than the snake: B2 H32 N8192 and B5 H8 N12123.)
+  if (FPATTN_CAUSAL_PAIRS && over_l2) causal_pairs(BH, nblk, grid, plan);
 }
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {

@@ -120,10 +120,14 @@ struct AttnArgs {
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st);
 
 // Causal schedule of an attention launch over BH (batch, head) problems of N
-// tokens on `grid` CTAs: heads per group, schedule positions of a full group
-// and of the whole launch (items plus the padding of each group). Host only.
-void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, int* hgroup, int* gspan,
-                 int* num_items);
+// tokens on `grid` CTAs. Either heads in groups (hgroup heads a group, gspan
+// positions a full group, items plus padding; hpairs = 0), or pairs of query
+// blocks head by head (hpairs pairs a head). num_items: all positions of the
+// launch. Host only.
+struct CausalPlan {
+  int hgroup, gspan, hpairs, num_items;
+};
+void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan);
 
 // Device error word access (defined next to the kernels).
 cudaError_t read_device_error(cudaStream_t st, int clear, int* code);

@@ -353,11 +353,11 @@ __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
 }
 
 // One warp per 128 consecutive 16-byte chunks (8 rows at D = 128, 16 at
-// D = 64): every load instruction covers 512 contiguous bytes. Lane i holds
-// chunks 32k + i; the two chunks of a 16-element block sit in adjacent
-// lanes, which combine their maxima with one shuffle and then take the same
-// scale decisions. Each lane writes the 4 code bytes of its chunk (a warp
-// store covers 128 contiguous bytes); even lanes write the block's scale byte.
+// D = 64), that is 64 16-element scale blocks: lane i takes blocks i and
+// i + 32, each whole (two adjacent chunks), so the scale of a block is worked
+// out once, by the lane that converts it. Each load instruction covers 1 KB
+// of contiguous rows; each lane writes the 8 code bytes of a block (a warp
+// store covers 256 contiguous bytes) and its scale byte.
 // grid = (nblk * 128 / kRowsPerCta, B*H): rows are padded to 128 per (b, h),
 // and the padding rows only write zero scales.
 template <int D, bool kMap>
@@ -365,49 +365,57 @@ __device__ __forceinline__ void nvfp4_quant_body(const uint4* __restrict__ x, in
                                                  const float* __restrict__ amax_ptr, uint32_t* __restrict__ codes,
                                                  uint8_t* __restrict__ sf, const TokenMap& tmap, int bx, int bh) {
   constexpr int kCpr = D / 8;                // 16-byte chunks per row
+  constexpr int kBpr = D / 16;               // 16-element scale blocks per row
   constexpr int kRowsPerWarp = 128 / kCpr;   // 8 or 16
   constexpr int kGroups = D / 64;            // 512-byte scale groups per 128-row block
   const int lane = threadIdx.x & 31;
   const int r0 = (bx * (kThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp;
   int src = 0;
   if (kMap && lane < kRowsPerWarp && r0 + lane < N) src = to_raster(tmap, r0 + lane);
-  uint4 v[4];
+  // lane takes blocks lane and lane + 32 of the warp's rows: each a whole
+  // 16-element scale block (two 16-byte chunks), all four loads issued first
+  uint4 v[2][2];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = 32 * k + lane;
-    const int rl = c / kCpr;
+  for (int k = 0; k < 2; ++k) {
+    const int blk = 32 * k + lane;
+    const int rl = blk / kBpr;
     const int srow = kMap ? __shfl_sync(0xffffffffu, src, rl) : r0 + rl;
-    v[k] = r0 + rl < N ? x[(static_cast<size_t>(bh) * N + srow) * kCpr + c % kCpr] : make_uint4(0u, 0u, 0u, 0u);
+    const size_t base = (static_cast<size_t>(bh) * N + srow) * kCpr + 2 * (blk % kBpr);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) v[k][h] = r0 + rl < N ? x[base + h] : make_uint4(0u, 0u, 0u, 0u);
   }
   const float s_t = nvfp4_tensor_scale(*amax_ptr);
   const float six_st = __fmul_rn(6.f, s_t);
+  uint2* codes2 = reinterpret_cast<uint2*>(codes);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = 32 * k + lane;
-    const int r = r0 + c / kCpr;
-    const int cc = c % kCpr;
-    float f[8];
-    unpack8(v[k], f);
+  for (int k = 0; k < 2; ++k) {
+    const int blk = 32 * k + lane;
+    const int r = r0 + blk / kBpr;
+    const int col = blk % kBpr;
+    float f[16];
+    unpack8(v[k][0], f);
+    unpack8(v[k][1], f + 8);
     float a = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(f[i]));
     const uint32_t sb = cvt_e4m3x2(__fdiv_rn(a, six_st), 0.f) & 0xFFu;
     const float den = __fmul_rn(e4m3_to_float(sb), s_t);
     const float inv = __fdiv_rn(1.f, den);
     const bool usable = (den != 0.f) && (fabsf(inv) <= FLT_MAX);
-    float y[8];
+    // an unusable scale (zero block, or 1/den not finite) gives zero codes,
+    // so the products need no select of their own
+    float y[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = usable ? __fmul_rn(f[i], inv) : 0.f;
-    if (r < N) codes[(static_cast<size_t>(bh) * N + r) * (D / 8) + cc] = usable ? cvt_e2m1x8(y) : 0u;
-    if ((lane & 1) == 0) {
-      // row r = 128 nb + 32 j + i, scale column col = 4 grp + s: byte
-      // 16 i + 4 j + s of the 512-byte group (bh, nb, grp)
-      const int col = cc >> 1, rr = r & 127;
-      const size_t byte = ((static_cast<size_t>(bh) * nblk + (r >> 7)) * kGroups + (col >> 2)) * 512 +
-                          16 * (rr & 31) + 4 * (rr >> 5) + (col & 3);
-      sf[byte] = r < N ? static_cast<uint8_t>(sb) : 0u;
-    }
+    for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(f[i], inv);
+    if (r < N)
+      codes2[(static_cast<size_t>(bh) * N + r) * kBpr + col] =
+          usable ? make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8)) : make_uint2(0u, 0u);
+    // row r = 128 nb + 32 j + i, scale column col = 4 grp + s: byte
+    // 16 i + 4 j + s of the 512-byte group (bh, nb, grp)
+    const int rr = r & 127;
+    const size_t byte = ((static_cast<size_t>(bh) * nblk + (r >> 7)) * kGroups + (col >> 2)) * 512 +
+                        16 * (rr & 31) + 4 * (rr >> 5) + (col & 3);
+    sf[byte] = r < N ? static_cast<uint8_t>(sb) : 0u;
   }
 }
 
@@ -548,10 +556,17 @@ __global__ void __launch_bounds__(kThreads) qkv_amax_kernel(const __grid_constan
   griddep_launch_dependents();
 }
 
+// Resident CTAs a SM the conversion kernel is compiled for: its loads are
+// issued before the arithmetic, so more warps keep more of them in flight.
+#ifndef FPATTN_CONVERT_CTAS
+#define FPATTN_CONVERT_CTAS 5
+#endif
+constexpr int kConvertCtasPerSm = FPATTN_CONVERT_CTAS;
+
 // V first, then K, then Q: the reverse of the amax pass, whose last reads are
 // the likeliest to be still in L2.
 template <int D, bool kMap, bool kFp4>
-__global__ void __launch_bounds__(kThreads) qkv_convert_kernel(const __grid_constant__ QkvParams p) {
+__global__ void __launch_bounds__(kThreads, kConvertCtasPerSm) qkv_convert_kernel(const __grid_constant__ QkvParams p) {
   griddep_wait();
   int b = blockIdx.x;
   const int nv = p.vgx * p.BH;

@@ -10,6 +10,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import precision_attention_nvfp4_b200 as fp
 from precision_attention_nvfp4_b200 import _lib
@@ -339,3 +340,16 @@ def test_attention_fwd_refuses_mismatched_operands():
     # CPU buffers never reach the library
     with pytest.raises(ValueError, match="contiguous tensor on"):
         fp.attention_fwd(nv(), nv(), f8("channel"))
+
+
+def test_attention_refuses_bad_qk_amax():
+    """A caller's Q/K amax is refused before any launch unless it is two CUDA
+    float32 tensors and Q/K are NVFP4."""
+    q = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    amax = (torch.ones(1), torch.ones(1))
+    with pytest.raises(ValueError):
+        fp.attention(q, q, q, qk_format="fp8", qk_amax=amax)
+    with pytest.raises(ValueError):
+        fp.attention(q, q, q, qk_amax=amax)          # host tensors
+    with pytest.raises(ValueError):
+        fp.attention(q, q, q, qk_amax=(amax[0],))    # one tensor

@@ -1,8 +1,11 @@
-"""Causal launches whose heads the library schedules in L2-sized groups.
+"""Causal launches in the library's L2-aware orders: heads in L2-sized
+groups, or pairs of query blocks head by head (even and odd block counts,
+a ragged tail).
 
-Output and LSE start as NaN, so a (head, query block) item the grouped
-schedule failed to deal would stay NaN; sampled rows of the first head, a
-middle one and one in the partial last group are checked against the oracle.
+Output and LSE start as NaN, so a (head, query block) item the schedule
+failed to deal would stay NaN; sampled rows (first, middle and last query
+blocks) of the first head, a middle one and one in the partial last group are
+checked against the oracle.
 """
 
 import numpy as np
@@ -16,11 +19,13 @@ import parity
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,H,N,fmt", [(4, 32, 4096, "nvfp4"), (16, 64, 2048, "nvfp4"), (8, 64, 2048, "fp8")])
-def test_grouped_causal_schedule_covers_every_item(B, H, N, fmt):
+@pytest.mark.parametrize("B,H,N,fmt", [(4, 32, 4096, "nvfp4"), (16, 64, 2048, "nvfp4"), (8, 64, 2048, "fp8"),
+                                        (4, 23, 6144, "fp8"), (10, 8, 12123, "nvfp4")])
+def test_causal_schedule_covers_every_item(B, H, N, fmt):
     d = 128
     plan = fp.causal_plan(B * H, N, d, fmt, "fp8", sm_count=torch.cuda.get_device_properties(0).multi_processor_count)
-    assert plan["heads_per_group"] < B * H, plan  # the grouped path is the one under test
+    # the grouped or the paired order is the one under test
+    assert plan["heads_per_group"] < B * H or plan["pairs_per_head"] > 0, plan
     w = workloads.Workload("t", B=B, H=H, N=N, d=d, causal=True, qk_format=fmt, seed=21)
     q, k, v = workloads.make_qkv(w)
     qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
@@ -38,8 +43,8 @@ def test_grouped_causal_schedule_covers_every_item(B, H, N, fmt):
     assert not torch.isnan(lse).any().item()
     G = plan["heads_per_group"]
     heads = [0, (B * H) // 2, (B * H // G) * G if (B * H) % G else B * H - 1]
-    nblk = N // 128
-    rows = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in (0, nblk // 2, nblk - 1)])
+    nblk = -(-N // 128)
+    rows = np.concatenate([np.arange(b * 128, min(N, b * 128 + 128)) for b in (0, nblk // 2, nblk - 1)])
     o = out.float().cpu().numpy().reshape(B * H, N, d)
     ls = lse.cpu().numpy().reshape(B * H, N)
     qh, kh, vh = parity.oracle_operands(q, k, v, fmt, heads)

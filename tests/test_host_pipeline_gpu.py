@@ -70,3 +70,25 @@ def test_tensor_amax_in_pieces_equals_whole():
     for f in ("codes", "block_sf", "tensor_scale"):
         assert torch.equal(getattr(whole, f).view(torch.uint8), getattr(parts, f).view(torch.uint8)), f
     np.testing.assert_equal(fp.tensor_amax(x).item(), 97.0)
+
+
+@pytest.mark.parametrize("scale", [1.0, 2.0])
+def test_host_pipeline_with_caller_amax(scale):
+    """A caller's Q/K amax (the static form of the NVFP4 recipe): the host
+    pipeline quantizes each group as it lands and returns the bits of the
+    device call with the same amax; with the true amax, those of the dynamic
+    call."""
+    w = workloads.Workload("t", B=2, H=3, N=520, d=128, causal=True, qk_format="nvfp4", seed=34, outliers=True)
+    q, k, v = workloads.make_qkv(w)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    amax = (fp.tensor_amax(qc) * scale, fp.tensor_amax(kc) * scale)
+    ref_out, ref_lse = fp.attention(qc, kc, vc, causal=True, qk_amax=amax)
+    if scale == 1.0:
+        dyn_out, _ = fp.attention(qc, kc, vc, causal=True)
+        assert torch.equal(dyn_out.view(torch.int16), ref_out.view(torch.int16))
+    torch.cuda.synchronize()
+    qh, kh, vh = _pinned(q, k, v)
+    out, lse = fp.attention(qh, kh, vh, causal=True, qk_amax=amax, host_chunks=4)
+    assert torch.equal(out.view(torch.int16), ref_out.cpu().view(torch.int16))
+    assert torch.equal(lse.view(torch.int32), ref_lse.cpu().view(torch.int32))
+    assert fp.device_error() == 0
