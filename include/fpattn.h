@@ -337,17 +337,19 @@ fpattn_status fpattn_sta_plan(int32_t nt, int32_t nh, int32_t nw, int32_t tt, in
  * would pass through the L2 at once, so the heads are grouped so that one
  * group's K and V bytes fit in a 32 MiB share of the L2, the groups following
  * one another, and each group's positions are padded to whole pairs of snake
- * rounds so that every group is dealt evenly. A group size is used only when
- * the padded schedule is modelled within 0.5% of the ungrouped one's balance.
+ * rounds so that every group is dealt evenly. Groups are used for NVFP4 Q/K
+ * with at most 32 query blocks (measured faster there; with FP8 Q/K slower),
+ * and a group size only when the padded schedule is modelled within 0.5% of
+ * the ungrouped one's balance.
  * Position p of group p / group_positions holds an item when its offset in
  * the group is below group_heads*nblk (group_heads = heads of that group);
  * that item is head group*heads_per_group + offset % group_heads, query block
  * nblk - 1 - offset / group_heads. Ungrouped: heads_per_group = bh and
  * group_positions = bh*nblk.
  *
- * Pairs (*pairs_per_head = P = ceil(nblk/2) > 0), when no group size both
- * fits and balances and the heads' K/V exceed four shares (the whole L2):
- * pair j = h*P + i of
+ * Pairs (*pairs_per_head = P = ceil(nblk/2) > 0), at d = 128 with at least
+ * 32 query blocks, no head groups, and the heads' K/V beyond four shares (the
+ * whole L2): pair j = h*P + i of
  * head h holds query blocks nblk-1-i and i, which together always cover nblk
  * + 1 key blocks, so pairs dealt round-robin (CTA c takes pairs c, c + C, ...)
  * balance the CTAs, and the CTAs in flight work on a few consecutive heads.

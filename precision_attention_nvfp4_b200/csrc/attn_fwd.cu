@@ -1390,6 +1390,15 @@ static bool causal_pairs(int BH, int nblk, int grid, CausalPlan* plan) {
   return true;
 }
 
+// Which order a causal launch takes, as measured on the sequence sweep
+// (B*H*N = 2^22 tokens, H = 32) against the plain longest-first snake:
+// - NVFP4 Q/K with at most 32 query blocks: L2-sized head groups (+3% to
+//   +8% at N <= 2048, neutral at 4096; LLM prefill reads its K/V once).
+//   With FP8 Q/K the groups were 5-12% slower at N = 1024-2048, so FP8 keeps
+//   the snake.
+// - d = 128 with at least 32 query blocks and K/V beyond the whole L2 (four
+//   shares): pairs (+8% to +23% from N = 4096 up). At d = 64 the pairs were
+//   1.5-2.5% slower, and with fewer blocks 7-23% slower.
 void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan) {
   const int nblk = (N + 127) / 128;
   plan->hgroup = BH;
@@ -1399,25 +1408,22 @@ void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, Causa
   if (BH < 1 || nblk < 1 || grid < 1) return;
   // K codes and block scales, V codes: the bytes of one head's keys
   const double kv_head = static_cast<double>(N) * ((qk_fp4 ? D / 2.0 + D / 16.0 : D) + (pv_fp4 ? D / 2.0 : D));
-  const bool over_l2 = BH * kv_head > 4 * kCausalGroupBytes;
-  if (FPATTN_CAUSAL_PAIRS == 2 && over_l2 && causal_pairs(BH, nblk, grid, plan)) return;
-  const int g = causal_head_group(BH, nblk, grid, kv_head);
-  if (g < BH) {
-    const long long span = padded_span(static_cast<long long>(g) * nblk, grid);
-    const int rest = BH % g;
-    const long long total = (BH / g) * span + (rest ? padded_span(static_cast<long long>(rest) * nblk, grid) : 0);
-    if (total > INT_MAX / 2) return;  // keep positions in int range: one group, no padding
-    plan->hgroup = g;
-    plan->gspan = static_cast<int>(span);
-    plan->num_items = static_cast<int>(total);
-    return;
+  if (qk_fp4 && nblk <= 32) {
+    const int g = causal_head_group(BH, nblk, grid, kv_head);
+    if (g < BH) {
+      const long long span = padded_span(static_cast<long long>(g) * nblk, grid);
+      const int rest = BH % g;
+      const long long total =
+          (BH / g) * span + (rest ? padded_span(static_cast<long long>(rest) * nblk, grid) : 0);
+      if (total > INT_MAX / 2) return;  // keep positions in int range: one group, no padding
+      plan->hgroup = g;
+      plan->gspan = static_cast<int>(span);
+      plan->num_items = static_cast<int>(total);
+      return;
+    }
   }
-  // No group size both fits and balances (a head's K/V are large, or the
-  // groups leave ragged rounds). When the heads' K/V together exceed the
-  // whole L2 (four shares), pair the rows instead, head by head, so that the
-  // CTAs in flight share the K/V of a few heads. (Below that size the pairs
-  // measured ~3% slower than the snake: B2 H32 N8192 and B5 H8 N12123.)
-  if (FPATTN_CAUSAL_PAIRS && over_l2) causal_pairs(BH, nblk, grid, plan);
+  if (FPATTN_CAUSAL_PAIRS && D == 128 && nblk >= 32 && BH * kv_head > 4 * kCausalGroupBytes)
+    causal_pairs(BH, nblk, grid, plan);
 }
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {

@@ -19,7 +19,7 @@ import parity
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,H,N,fmt", [(4, 32, 4096, "nvfp4"), (16, 64, 2048, "nvfp4"), (8, 64, 2048, "fp8"),
+@pytest.mark.parametrize("B,H,N,fmt", [(4, 32, 4096, "nvfp4"), (16, 64, 2048, "nvfp4"), (8, 64, 1024, "nvfp4"),
                                         (4, 23, 6144, "fp8"), (10, 8, 12123, "nvfp4")])
 def test_causal_schedule_covers_every_item(B, H, N, fmt):
     d = 128

@@ -48,7 +48,7 @@ def _kv_bytes(n, d, qk, pv):
 CASES = [  # (B*H, N, d, qk, pv)
     (128, 4096, 128, "nvfp4", "fp8"),    # LLM prefill
     (1024, 2048, 128, "nvfp4", "fp8"),   # a partial last group
-    (1024, 1024, 64, "fp8", "fp8"),
+    (1024, 1024, 64, "fp8", "fp8"),      # FP8: the snake, ungrouped
     (32, 131072, 128, "nvfp4", "fp8"),   # one head's K/V exceed the share: pairs
     (35, 300, 128, "nvfp4", "fp8"),      # fewer items than SMs
     (256, 16384, 128, "fp8", "fp8"),
@@ -80,8 +80,10 @@ def test_schedule_fits_the_share_and_keeps_the_balance(bh, n, d, qk, pv):
     kv = _kv_bytes(n, d, qk, pv)
     if bh * kv <= L2_SHARE:
         assert G == bh and P == 0  # everything fits already
-    if bh * kv <= 4 * L2_SHARE:
-        assert P == 0              # pairs only when the K/V exceed the whole L2
+    if bh * kv <= 4 * L2_SHARE or d != 128 or nblk < 32:
+        assert P == 0              # pairs only at d = 128, 32+ blocks, K/V beyond the whole L2
+    if qk != "nvfp4" or nblk > 32:
+        assert G == bh             # head groups only for NVFP4 Q/K with at most 32 blocks
     if P:
         assert G == bh and P == (nblk + 1) // 2 and plan["positions"] == 2 * bh * P
     elif G < bh:
