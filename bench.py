@@ -127,6 +127,13 @@ class ClockSampler:
             self.thread.start()
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # wait for the first sample (3 s at most) so that nvidia-smi's
+        # start-up falls before the warm-up: inside a short timed region it
+        # once coincided with steps ten times their usual length
+        t_end = time.time() + 3.0
+        while not self.samples and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:

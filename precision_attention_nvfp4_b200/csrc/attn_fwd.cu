@@ -270,8 +270,13 @@ __device__ __forceinline__ int next_item(const Params& p, int& rnd) {
 // out-of-bounds access.
 __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, int& qb) {
   if (p.sparse) {
-    const int r = item / p.BH;
-    bh = item % p.BH;
+    // one head's rows after another, each head's in the mask's row order
+    // (longest first): the CTAs in flight share the K/V windows of one or
+    // two heads (with every head's same row together, those of all heads
+    // passed through the L2 at once: 14.8 against 12.8 ms on the 40-head
+    // video workload)
+    const int r = item % p.nblk;
+    bh = item / p.nblk;
     qb = p.row_order ? p.row_order[r] : r;
     if (static_cast<unsigned>(qb) >= static_cast<unsigned>(p.nblk)) qb = 0;
   } else if (p.hpairs) {
@@ -1333,22 +1338,14 @@ double causal_makespan(int BH, int nblk, int g, int grid, std::vector<double>& l
 // all heads pass through the L2 together. Groups whose K and V (codes and
 // scales, kv_head bytes a head) fit in kCausalGroupBytes keep that
 // working set in L2; a group size is taken only if its padded schedule is
-// within 0.5% of the ungrouped one's balance (modelled on the host, once per
-// shape), else all heads form one group.
+// within 0.5% of the ungrouped one's balance (modelled on the host), else all
+// heads form one group.
 int causal_head_group(int BH, int nblk, int grid, double kv_head) {
   const double budget = kCausalGroupBytes;
   if (budget <= 0.0 || kv_head <= 0.0) return BH;
   const double fit = budget / kv_head;
   if (fit >= BH) return BH;
   const int gmax = fit < 1.0 ? 1 : static_cast<int>(fit);
-  struct Entry { int BH, nblk, grid, gmax, g; };
-  static std::mutex mu;
-  static std::vector<Entry> cache;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    for (const Entry& e : cache)
-      if (e.BH == BH && e.nblk == nblk && e.grid == grid && e.gmax == gmax) return e.g;
-  }
   std::vector<double> load;
   const double base = causal_makespan(BH, nblk, BH, grid, load);
   int best = BH;
@@ -1362,9 +1359,6 @@ int causal_head_group(int BH, int nblk, int grid, double kv_head) {
       best_m = m;
     }
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (cache.size() >= 64) cache.erase(cache.begin());
-  cache.push_back(Entry{BH, nblk, grid, gmax, best});
   return best;
 }
 
@@ -1399,7 +1393,7 @@ static bool causal_pairs(int BH, int nblk, int grid, CausalPlan* plan) {
 // - d = 128 with at least 32 query blocks and K/V beyond the whole L2 (four
 //   shares): pairs (+8% to +23% from N = 4096 up). At d = 64 the pairs were
 //   1.5-2.5% slower, and with fewer blocks 7-23% slower.
-void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan) {
+static void causal_plan_uncached(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan) {
   const int nblk = (N + 127) / 128;
   plan->hgroup = BH;
   plan->gspan = BH * nblk;
@@ -1424,6 +1418,30 @@ void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, Causa
   }
   if (FPATTN_CAUSAL_PAIRS && D == 128 && nblk >= 32 && BH * kv_head > 4 * kCausalGroupBytes)
     causal_pairs(BH, nblk, grid, plan);
+}
+
+// The plans of the last 64 shapes are kept: modelling one takes up to a few
+// milliseconds of host time, a launch of the same shape needs none.
+void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan) {
+  struct Entry {
+    int BH, N, D, flags, grid;
+    CausalPlan plan;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  const int flags = (qk_fp4 ? 1 : 0) | (pv_fp4 ? 2 : 0);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (e.BH == BH && e.N == N && e.D == D && e.flags == flags && e.grid == grid) {
+        *plan = e.plan;
+        return;
+      }
+  }
+  causal_plan_uncached(BH, N, D, qk_fp4, pv_fp4, grid, plan);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 64) cache.erase(cache.begin());
+  cache.push_back(Entry{BH, N, D, flags, grid, *plan});
 }
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {
