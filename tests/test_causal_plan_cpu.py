@@ -109,7 +109,7 @@ def test_pairs_keep_few_heads_in_flight():
     plan = fp.causal_plan(256, 16384, 128, "fp8", "fp8", sm_count=148)
     P, C = plan["pairs_per_head"], plan["ctas"]
     assert P == 64
-    j = np.arange(C)  # the pairs of round 0
+    j = np.arange(C)  # the pairs of the first scheduling round
     assert len(np.unique(j // P)) == 3
     assert np.all((128 - 1 - j % P) + 1 + (j % P) + 1 == 129)
 
