@@ -447,8 +447,16 @@ def run_sweep(args):
                     exec_flops = 4.0 * 128 * 128 * d * executed_block_pairs(w) * B * 32
                     peak = 2.0 / (1.0 / p4 + 1.0 / p8) if fmt == "nvfp4" else p8
                     tf = flops / (ms * 1e-3) / 1e12
+                    order = None
+                    if causal:
+                        plan = fp.causal_plan(B * 32, N, d, fmt, "fp8",
+                                              sm_count=torch.cuda.get_device_properties(0).multi_processor_count)
+                        order = ("pairs" if plan["pairs_per_head"] else
+                                 f"groups of {plan['heads_per_group']}" if plan["heads_per_group"] < B * 32
+                                 else "longest first")
                     print(json.dumps({
                         "sweep": True, "N": N, "B": B, "H": 32, "d": d, "causal": causal, "qk": fmt,
+                        "causal_order": order,
                         "attn_ms": ms, "tflops_dense_eq": tf,
                         "tflops_executed": exec_flops / (ms * 1e-3) / 1e12,
                         "frac_of_peak": tf / peak, "peak_tflops": peak,
