@@ -89,6 +89,15 @@ def executed_block_pairs(w: workloads.Workload) -> int:
     return nblk * (nblk + 1) // 2 if w.causal else nblk * nblk
 
 
+def quant_bytes_one_pass(w: workloads.Workload, pv_format: str = "fp8") -> float:
+    """The lower bound of the step's quantization bytes: every bf16 input read
+    once and every code and scale written once (the amax passes left out)."""
+    n = w.B * w.H * w.N * w.d
+    qk = 2 * n * ((2 + 0.5 + 1.0 / 16) if w.qk_format == "nvfp4" else (2 + 1))
+    v = n * ((2 + 0.5 + 1.0 / 16) if pv_format == "nvfp4" else (2 + 1))
+    return qk + v
+
+
 def quant_bytes(w: workloads.Workload, pv_format: str = "fp8") -> float:
     """Algorithmic HBM bytes of one step's quantization (two-pass amax)."""
     n = w.B * w.H * w.N * w.d
@@ -689,6 +698,7 @@ def main():
             "attn_tflops_dense_eq": w.dense_flops() / (attn_ms * 1e-3) / 1e12,
             "attn_tflops_executed": exec_flops / (attn_ms * 1e-3) / 1e12,
             "quant_ms": quant_ms, "quant_gbs": quant_gbs, "quant_frac_hbm": quant_gbs / peaks["hbm_gbs"],
+            "quant_one_pass_bound_ms": quant_bytes_one_pass(w, args.pv_format) / (peaks["hbm_gbs"] * 1e9) * 1e3,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "frac_of_burst_peak": attn_tflops / peak_burst,
                          "traffic": profiled_traffic(w.name) if args.pv_format == "fp8" and
