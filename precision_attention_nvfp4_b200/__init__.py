@@ -57,6 +57,19 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _aux(t: Optional[torch.Tensor], dev: torch.device, dtype: torch.dtype, n: int, name: str) -> Optional[int]:
+    """Device pointer of an optional buffer the kernels read or write (an
+    amax, a flag, an output), after checking that it is a contiguous tensor
+    of ``dtype`` on ``dev`` with at least ``n`` elements: anything else is
+    refused before a launch could touch it."""
+    if t is None:
+        return None
+    if (not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != dev or t.dtype != dtype
+            or not t.is_contiguous() or t.numel() < n):
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor on {dev} with at least {n} elements")
+    return t.data_ptr()
+
+
 def _desc(t: torch.Tensor, dtype: int, B: int, H: int, N: int, d: int) -> _lib.Tensor:
     return _lib.Tensor(t.data_ptr(), dtype, B, H, N, d)
 
@@ -118,12 +131,14 @@ def quantize_nvfp4(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None,
     sf = torch.empty(lib.fpattn_nvfp4_sf_bytes(B, H, N, d), dtype=torch.uint8, device=x.device)
     ts = torch.empty(1, dtype=torch.float32, device=x.device)
     xd = ctypes.byref(_desc(x, _lib.BF16, B, H, N, d))
+    amax_p = _aux(static_amax, x.device, torch.float32, 1, "static_amax")
+    flag_p = _aux(nonfinite_flag, x.device, torch.int32, 1, "nonfinite_flag")
     if video is None:
-        st = lib.fpattn_quantize_nvfp4(xd, _ptr(static_amax), codes.data_ptr(), sf.data_ptr(), ts.data_ptr(),
-                                       _ptr(nonfinite_flag), _stream())
+        st = lib.fpattn_quantize_nvfp4(xd, amax_p, codes.data_ptr(), sf.data_ptr(), ts.data_ptr(), flag_p,
+                                       _stream())
     else:
-        st = lib.fpattn_quantize_nvfp4_video(xd, _video_ref(video), _ptr(static_amax), codes.data_ptr(),
-                                             sf.data_ptr(), ts.data_ptr(), _ptr(nonfinite_flag), _stream())
+        st = lib.fpattn_quantize_nvfp4_video(xd, _video_ref(video), amax_p, codes.data_ptr(),
+                                             sf.data_ptr(), ts.data_ptr(), flag_p, _stream())
     _lib.check(st, "fpattn_quantize_nvfp4" + ("_video" if video is not None else ""))
     return Nvfp4Tensor(codes, sf, ts, (B, H, N, d))
 
@@ -136,8 +151,10 @@ def tensor_amax(x: torch.Tensor, out: Optional[torch.Tensor] = None, accumulate:
     B, H, N, d = _check_bf16(x)
     if out is None:
         out = torch.empty(1, dtype=torch.float32, device=x.device)
+    out_p = _aux(out, x.device, torch.float32, 1, "out")
+    flag_p = _aux(nonfinite_flag, x.device, torch.int32, 1, "nonfinite_flag")
     st = library().fpattn_tensor_amax(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), 1 if accumulate else 0,
-                                      out.data_ptr(), _ptr(nonfinite_flag), _stream())
+                                      out_p, flag_p, _stream())
     _lib.check(st, "fpattn_tensor_amax")
     return out
 
@@ -154,8 +171,9 @@ def quantize_nvfp4_v(x: torch.Tensor, static_amax: Optional[torch.Tensor] = None
     sf = torch.empty(sfb.value, dtype=torch.uint8, device=x.device)
     ts = torch.empty(1, dtype=torch.float32, device=x.device)
     st = lib.fpattn_quantize_nvfp4_v(ctypes.byref(_desc(x, _lib.BF16, B, H, N, d)), _video_ref(video),
-                                     _ptr(static_amax), codes.data_ptr(), sf.data_ptr(), ts.data_ptr(),
-                                     _ptr(nonfinite_flag), _stream())
+                                     _aux(static_amax, x.device, torch.float32, 1, "static_amax"), codes.data_ptr(),
+                                     sf.data_ptr(), ts.data_ptr(),
+                                     _aux(nonfinite_flag, x.device, torch.int32, 1, "nonfinite_flag"), _stream())
     _lib.check(st, "fpattn_quantize_nvfp4_v")
     return Nvfp4VTensor(codes, sf, ts, (B, H, N, d))
 
@@ -175,16 +193,17 @@ def quantize_fp8(x: torch.Tensor, granularity: str = "tile128",
     else:
         raise ValueError("granularity must be 'tile128', 'channel' or 'group'")
     xd = ctypes.byref(_desc(x, _lib.BF16, B, H, N, d))
+    flag_p = _aux(nonfinite_flag, x.device, torch.int32, 1, "nonfinite_flag")
     if g is None:
         st = lib.fpattn_quantize_fp8_group(xd, _video_ref(video), int(group_tiles), codes.data_ptr(),
-                                           scales.data_ptr(), _ptr(nonfinite_flag), _stream())
+                                           scales.data_ptr(), flag_p, _stream())
         _lib.check(st, "fpattn_quantize_fp8_group")
         return Fp8Tensor(codes, scales, "tile128", (B, H, N, d))
     if video is None:
-        st = lib.fpattn_quantize_fp8(xd, g, codes.data_ptr(), scales.data_ptr(), _ptr(nonfinite_flag), _stream())
+        st = lib.fpattn_quantize_fp8(xd, g, codes.data_ptr(), scales.data_ptr(), flag_p, _stream())
     else:
         st = lib.fpattn_quantize_fp8_video(xd, _video_ref(video), g, codes.data_ptr(), scales.data_ptr(),
-                                           _ptr(nonfinite_flag), _stream())
+                                           flag_p, _stream())
     _lib.check(st, "fpattn_quantize_fp8" + ("_video" if video is not None else ""))
     return Fp8Tensor(codes, scales, granularity, (B, H, N, d))
 
@@ -197,8 +216,11 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, qk_format: s
     B, H, N, d = _check_bf16(q)
     if _check_bf16(k) != (B, H, N, d) or _check_bf16(v) != (B, H, N, d):
         raise ValueError("q, k, v must have one shape")
+    if k.device != q.device or v.device != q.device:
+        raise ValueError("q, k, v must be on one device")
     lib = library()
     dev = q.device
+    flag_p = _aux(nonfinite_flag, dev, torch.int32, 1, "nonfinite_flag")
     nblk = (N + 127) // 128
     if qk_format == "nvfp4":
         dt = _lib.NVFP4
@@ -219,7 +241,7 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, qk_format: s
                                  ctypes.byref(_desc(k, _lib.BF16, B, H, N, d)),
                                  ctypes.byref(_desc(v, _lib.BF16, B, H, N, d)), dt, _video_ref(video),
                                  qc.data_ptr(), _ptr(qsf), qs.data_ptr(), kc.data_ptr(), _ptr(ksf), ks.data_ptr(),
-                                 vc.data_ptr(), vs.data_ptr(), _ptr(nonfinite_flag), _stream())
+                                 vc.data_ptr(), vs.data_ptr(), flag_p, _stream())
     _lib.check(st, "fpattn_quantize_qkv")
     if qk_format == "nvfp4":
         qq, kq = Nvfp4Tensor(qc, qsf, qs, (B, H, N, d)), Nvfp4Tensor(kc, ksf, ks, (B, H, N, d))
@@ -271,7 +293,13 @@ class DeviceTileMask:
     col_idx: torch.Tensor
     row_order: Optional[torch.Tensor]
 
-    def desc(self) -> _lib.TileMask:
+    def desc(self, dev: Optional[torch.device] = None) -> _lib.TileMask:
+        """The C descriptor; with ``dev``, after checking that the arrays are
+        int32 tensors on that device, sized as nblk and nnz say."""
+        if dev is not None:
+            _aux(self.row_ptr, dev, torch.int32, self.nblk + 1, "tile_mask.row_ptr")
+            _aux(self.col_idx, dev, torch.int32, self.nnz, "tile_mask.col_idx")
+            _aux(self.row_order, dev, torch.int32, self.nblk, "tile_mask.row_order")
         return _lib.TileMask(self.nblk, self.nnz, self.row_ptr.data_ptr(), self.col_idx.data_ptr(),
                              _ptr(self.row_order))
 
@@ -391,11 +419,15 @@ def attention_fwd(q, k, v, *, causal: bool = False, tile_mask: Optional[DeviceTi
         kd = _desc(k.codes, _lib.E4M3, *k.shape)
         sc = _lib.Scales(q.scales.data_ptr(), k.scales.data_ptr(), v_scale, None, None,
                          1.0 / 448.0, softmax_scale, rescale_threshold, v_sf)
+    dev = v.codes.device
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.codes.device)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     if lse is None and return_lse:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.codes.device)
-    mask = ctypes.byref(tile_mask.desc()) if tile_mask is not None else None
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    # the kernel writes every row of out and lse: a caller's buffers must hold them
+    _aux(out, dev, torch.bfloat16, B * H * N * d, "out")
+    _aux(lse, dev, torch.float32, B * H * N, "lse")
+    mask = ctypes.byref(tile_mask.desc(dev)) if tile_mask is not None else None
     if video is None:
         st = lib.fpattn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(sc), mask,
                             1 if causal else 0, out.data_ptr(), _ptr(lse), _stream())
