@@ -87,10 +87,10 @@ constexpr int kThreads = 512;
 // Of every 16 exp2 pairs, how many take the FMA-pipe polynomial (the rest
 // take MUFU), with NVFP4 and with FP8 Q/K.
 #ifndef FPATTN_POLY_FP4
-#define FPATTN_POLY_FP4 5
+#define FPATTN_POLY_FP4 4
 #endif
 #ifndef FPATTN_POLY_FP8
-#define FPATTN_POLY_FP8 5
+#define FPATTN_POLY_FP8 4
 #endif
 // Per-warpgroup register budgets (setmaxnreg) of the 512-thread CTA, which
 // launches with 128 registers a thread: control warps, softmax warps,
@@ -139,7 +139,8 @@ struct Cfg {
   static constexpr uint32_t kVSbo = PV4 ? 8 * 64 : 8 * D;
   static constexpr int kKSteps = FP4 ? D / 64 : D / 32;   // MMAs per S tile
   // of the 16 exp2 pairs of a 32-score chunk, how many take the FMA-pipe
-  // polynomial (measured best with the row-split softmax: 5)
+  // polynomial (measured best with the row-split softmax and the degree-4
+  // polynomial: 4; 3, 5 and 6 were 1-4% slower on the dense workloads)
   static constexpr int kPolyPairs = FP4 ? FPATTN_POLY_FP4 : FPATTN_POLY_FP8;
   static constexpr uint32_t kColO = 256;                  // O: d fp32 columns
   // P buffers, 32 columns each (128 E4M3 keys), as many as K/V stages when
