@@ -334,9 +334,12 @@ def choose_peak(peaks: dict, clk: dict, timed_s: float, qk: str, pv: str):
     return peak, peak * peaks["bf16_tflops"] / bf16, bf16, sustained, capped
 
 
-# Softmax cycles per 128x128 block and SM: MUFU 16,384 * 11/16 / 16 = 704
-# (5 of 16 exp2 pairs on the FMA-pipe polynomial), issue slots ~725 (about
-# 2,900 warp instructions at one a clock per sub-partition). The larger binds.
+# Softmax cycles per 128x128 block and SM, at the split of the exponentials
+# between MUFU and the FMA-pipe polynomial where the two balance (5 of 16 exp2
+# pairs on the polynomial): MUFU 16,384 * 11/16 / 16 = 704, issue slots ~725
+# (about 2,900 warp instructions of softmax work at one a clock per
+# sub-partition). The larger binds. This is a bound of the work, not of the
+# kernel's own split (4 of 16, which measured faster).
 SOFTMAX_CYCLES_PER_BLOCK = 725.0
 
 
