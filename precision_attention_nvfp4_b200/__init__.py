@@ -502,6 +502,19 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, qk_format: s
                          return_lse=return_lse, video=video, rescale_threshold=rescale_threshold)
 
 
+_COPY_STREAMS = {}
+
+
+def _copy_streams(dev: torch.device):
+    """The host pipeline's two copy streams of a device, created once: every
+    call orders them after the caller's stream itself, so reusing them adds
+    no dependency between calls beyond the caller's own stream order."""
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _COPY_STREAMS:
+        _COPY_STREAMS[key] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _COPY_STREAMS[key]
+
+
 def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, return_lse, device, out_host,
                     lse_host, video, rescale_threshold, qk_group_tiles, pv_format, chunks: Optional[int] = None,
                     qk_amax=None):
@@ -531,7 +544,7 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
     spans = [s for s in (head_range(BH, chunks, r) for r in range(chunks)) if s[1] > s[0]]
     flat = [t.reshape(BH, N, d) for t in (q, k, v)]
     cur = torch.cuda.current_stream(dev)
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_in, s_out = _copy_streams(dev)
     qd, kd, vd = (torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
     out_d = torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev)
     lse_d = torch.empty((BH, N), dtype=torch.float32, device=dev) if return_lse else None
