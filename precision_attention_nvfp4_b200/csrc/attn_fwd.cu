@@ -1351,9 +1351,12 @@ int causal_head_group(int BH, int nblk, int grid, double kv_head) {
   const double base = causal_makespan(BH, nblk, BH, grid, load);
   int best = BH;
   double best_m = base * 1.005;
-  // at most 64 sizes, largest first; a smaller group must beat a larger one
-  // by 0.1% to be taken
-  for (int g = gmax, tried = 0; g >= 1 && tried < 64; --g, ++tried) {
+  // at most 64 sizes, largest first, and about 2^21 modelled items in all
+  // (a few milliseconds of host time, once per shape); a smaller group must
+  // beat a larger one by 0.1% to be taken
+  const long long items = static_cast<long long>(BH) * nblk;
+  const int budget_sizes = static_cast<int>(std::max(1LL, std::min(64LL, (1LL << 21) / std::max(1LL, items))));
+  for (int g = gmax, tried = 0; g >= 1 && tried < budget_sizes; --g, ++tried) {
     const double m = causal_makespan(BH, nblk, g, grid, load);
     if (m <= best_m && (best == BH || m < best_m * 0.999)) {
       best = g;
