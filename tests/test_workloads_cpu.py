@@ -57,6 +57,23 @@ def test_quant_bytes_and_aggregate():
     assert bench.aggregate_value(1e12, 4, 2.0) == pytest.approx(4 * 1e12 / 2e-3 / 1e12)
 
 
+def test_one_pass_bound_and_alu_roofline():
+    w = workloads.get("llm_prefill_causal")
+    n = 4 * 32 * 4096 * 128
+    # every input read once, every code and scale written once
+    assert bench.quant_bytes_one_pass(w) == pytest.approx(2 * n * 2.5625 + n * 3)
+    assert bench.quant_bytes_one_pass(w, "nvfp4") == pytest.approx(3 * n * 2.5625)
+    v = workloads.get("video_dense_fp8")
+    nv = 1 * 40 * 75600 * 128
+    assert bench.quant_bytes_one_pass(v) == pytest.approx(3 * nv * 3)
+    # the ALU bound: 4*128*128*d flops per block over SOFTMAX_CYCLES_PER_BLOCK cycles on 148 SMs
+    r = bench.alu_roofline(w, 1000.0, {"sm_max_mhz": 1965.0})
+    expect = 4 * 128 * 128 * 128 * 148 * 1965e6 / bench.SOFTMAX_CYCLES_PER_BLOCK / 1e12
+    assert r["bound"] == "alu" and r["peak"] == pytest.approx(expect) and r["frac"] == pytest.approx(1000 / expect)
+    d64 = workloads.Workload("t", B=1, H=1, N=128, d=64, causal=False, qk_format="nvfp4", seed=0)
+    assert bench.alu_roofline(d64, 1.0, {"sm_max_mhz": 1965.0})["peak"] == pytest.approx(expect / 2)
+
+
 def test_peak_choice_follows_the_clock_record():
     peaks = {"bf16_tflops": 1655.8, "bf16_tflops_sustained": 1416.8, "hbm_gbs": 6538.3}
     full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
