@@ -52,14 +52,53 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def strip_comments(text: str) -> str:
+    """C++ source without its // and /* */ comments, trailing blanks and
+    empty lines (string and character literals are kept whole)."""
+    out, i, n, in_block = [], 0, len(text), False
+    line = []
+    while i < n:
+        c = text[i]
+        if in_block:
+            if text.startswith("*/", i):
+                in_block, i = False, i + 2
+            else:
+                if c == "\n":
+                    out.append("".join(line)); line = []
+                i += 1
+            continue
+        if text.startswith("//", i):
+            while i < n and text[i] != "\n":
+                i += 1
+            continue
+        if text.startswith("/*", i):
+            in_block, i = True, i + 2
+            continue
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            line.append(text[i:j + 1]); i = j + 1
+            continue
+        if c == "\n":
+            out.append("".join(line)); line = []
+        else:
+            line.append(c)
+        i += 1
+    out.append("".join(line))
+    return "\n".join(ln.rstrip() for ln in out if ln.strip())
+
+
 def kernel_source_hash() -> str:
-    """First 16 hex digits of sha256(attn_fwd.cu + sm100.cuh): ties a DRAM
-    traffic record to the kernel source it was captured on."""
+    """First 16 hex digits of sha256 over the code of attn_fwd.cu and
+    sm100.cuh (comments and blank lines removed): ties a DRAM traffic record
+    to the kernel code it was captured on, so that a change of wording in a
+    comment does not void it."""
     import hashlib
     h = hashlib.sha256()
     for src in ("attn_fwd.cu", "sm100.cuh"):
-        with open(os.path.join(ROOT, "precision_attention_nvfp4_b200", "csrc", src), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "precision_attention_nvfp4_b200", "csrc", src), encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -26,18 +26,19 @@
 //   warp 1        tensor-memory allocator; issues O += P V (one thread)
 //   warp 2        issues S = Q K^T (one thread)
 //   warp 3        idle
-//   warps 4-7     softmax warpgroup 0: keys 0-63 of every key block
-//   warps 8-11    softmax warpgroup 1: keys 64-127 of every key block
+//   warps 4-7     softmax warpgroup 0
+//   warps 8-11    softmax warpgroup 1
 //   warps 12-15   O rescale (correction) and epilogue
 // The CTA launches with 128 registers a thread; the warpgroups then take
 // 56 (control), 176 (softmax) and 96 (correction) with setmaxnreg.
-// Thread (warp quarter q, lane t) of a softmax warpgroup owns query row
-// 32q + t and its warpgroup's 64 keys of the block, read from TMEM once into
-// registers. The two warps sharing a row quarter (and an SM sub-partition)
-// work on the same block at the same time, so their exponentials keep the
-// MUFU and FMA pipes busy together; they exchange only their half-block row
-// maxima, per lane, through tagged shared-memory words. Each keeps the row
-// sum of its half; the epilogue adds the two.
+// With E4M3 P the softmax splits rows: the warp of warpgroup w and quarter q
+// owns rows 32q + 16w .. +15 and all 128 keys of every block, two threads a
+// row (the tensor-memory 16x64b pattern), so no warp waits on another within
+// a block. Its exponentials run 4 of every 16 pairs on an FMA-pipe
+// polynomial and the rest on MUFU. With NVFP4 P (PV4) the warpgroups split
+// keys instead: one row a thread, 64 keys a warpgroup, and the half-block row
+// maxima exchanged per lane through tagged shared-memory words; each keeps
+// the row sum of its half and the epilogue adds the two.
 // Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32
 // 128x128, buffer = block parity), O at column 256 (d fp32 columns), a ring
 // of P buffers (one per ring stage, three with NVFP4 Q/K; E4M3: 32 columns
@@ -51,8 +52,11 @@
 // K and V are loaded with an L2 evict-last policy, Q and the output with
 // evict-first. The kernel waits for its stream predecessor (programmatic
 // dependent launch) only after its prologue.
-// Work items are (batch*head, 128-query block); causal runs schedule the
-// longest query blocks first, tile-mask runs follow the mask's row order.
+// Work items are (batch*head, 128-query block), dealt to the CTAs in orders
+// that keep the K/V in flight within the L2: dense runs one head's query
+// blocks together; causal runs longest first in L2-sized head groups, or in
+// pairs of query blocks head by head (causal_plan); tile-mask runs one head
+// after another in the mask's row order.
 #include <algorithm>
 #include <atomic>
 #include <climits>

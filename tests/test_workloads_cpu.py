@@ -74,6 +74,14 @@ def test_one_pass_bound_and_alu_roofline():
     assert bench.alu_roofline(d64, 1.0, {"sm_max_mhz": 1965.0})["peak"] == pytest.approx(expect / 2)
 
 
+def test_code_hash_ignores_comments_only():
+    src = 'int a = 1; // note\n/* block\n note */ int b = 2;\n\nconst char* s = "// kept";\n'
+    reworded = 'int a = 1; // other words\n/* another\n block */ int b = 2;\nconst char* s = "// kept";  \n'
+    assert bench.strip_comments(src) == bench.strip_comments(reworded)
+    assert bench.strip_comments(src) != bench.strip_comments(src.replace("b = 2", "b = 3"))
+    assert '"// kept"' in bench.strip_comments(src)
+
+
 def test_peak_choice_follows_the_clock_record():
     peaks = {"bf16_tflops": 1655.8, "bf16_tflops_sustained": 1416.8, "hbm_gbs": 6538.3}
     full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
