@@ -1428,8 +1428,11 @@ static void causal_plan_uncached(int BH, int N, int D, bool qk_fp4, bool pv_fp4,
     causal_pairs(BH, nblk, grid, plan);
 }
 
-// The plans of the last 64 shapes are kept: modelling one takes up to a few
-// milliseconds of host time, a launch of the same shape needs none.
+// The plans of the last 64 shapes are kept: modelling one takes host time
+// (about 30 ns per modelled item: a few milliseconds for the head groups,
+// whose search is capped, and for the pairs linear in B*H*N/128, far below
+// the launch's own time, which grows with the square of N); a launch of the
+// same shape needs none.
 void causal_plan(int BH, int N, int D, bool qk_fp4, bool pv_fp4, int grid, CausalPlan* plan) {
   struct Entry {
     int BH, N, D, flags, grid;
