@@ -5,7 +5,9 @@ cross-rank steps are the barrier and the max-over-ranks timing reduction;
 both are exercised here, plus the whole-job aggregation, and the split of one
 seeded batch's heads over the ranks (head_range): every rank takes its
 contiguous share, and gathering the shares in rank order gives back the
-batch, every head once, in order.
+batch, every head once, in order. Splitting one batch needs one exchange for
+NVFP4 Q/K, the tensor amax (one float, max-reduced); with it every rank's
+share quantizes (oracle, on the CPU) exactly as the whole tensor would.
 """
 import datetime
 import os
@@ -109,3 +111,41 @@ def test_head_range_covers_each_head_once(n, world):
     assert all(spans[i][1] == spans[i + 1][0] for i in range(world - 1))
     sizes = [b - a for a, b in spans]
     assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+
+
+def _amax_worker(rank, world, port, q):
+    import numpy as np
+    from oracle import quant as oq
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = workloads.Workload("t", B=2, H=3, N=64, d=64, causal=False, qk_format="nvfp4", seed=22, outliers=True)
+        x, _, _ = workloads.make_qkv(w)
+        flat = x.reshape(w.B * w.H, w.N, w.d).float().numpy()
+        a, b = fp.head_range(w.B * w.H, world, rank)
+        # the one exchange a head-sharded batch needs: the NVFP4 tensor amax,
+        # one float per tensor, max-reduced over the ranks
+        local = torch.tensor([float(np.abs(flat[a:b]).max()) if b > a else 0.0])
+        dist.all_reduce(local, op=dist.ReduceOp.MAX)
+        codes, sf, st = oq.quantize_nvfp4(flat[a:b], static_amax=float(local))
+        whole_codes, whole_sf, whole_st = oq.quantize_nvfp4(flat)
+        q.put((rank, float(local) == float(np.abs(flat).max()), bool(np.array_equal(codes, whole_codes[a:b])),
+               bool(np.array_equal(sf, whole_sf[a:b])), float(st) == float(whole_st)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_nvfp4_amax_exchange_gives_the_whole_tensor_codes():
+    """Sharding one batch's heads over ranks: the max-reduced amax makes every
+    rank quantize its share exactly as the whole tensor would be quantized."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_amax_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert res == [(0, True, True, True, True), (1, True, True, True, True)]
