@@ -42,7 +42,7 @@ from ._lib import FpattnError
 __all__ = ["Nvfp4Tensor", "Nvfp4VTensor", "Fp8Tensor", "StaPlan", "VideoLayout", "quantize_nvfp4", "quantize_qkv",
            "quantize_nvfp4_v", "quantize_fp8", "sta_plan",
            "step_phase", "attention_fwd", "attention", "device_error", "library", "FpattnError",
-           "head_range", "tensor_amax", "causal_plan"]
+           "head_range", "tensor_amax", "causal_plan", "attention_sharded"]
 
 
 def library() -> ctypes.CDLL:
@@ -629,6 +629,33 @@ def _attention_host(q, k, v, *, qk_format, causal, tile_mask, softmax_scale, ret
         t.record_stream(s_out)
     cur.synchronize()
     return out_h, lse_h
+
+
+def attention_sharded(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, group=None,
+                      qk_format: str = "nvfp4", **kwargs):
+    """attention() on this rank's share of one batch's (batch, head)
+    problems (device bf16 [B_r, H_r, N, d], e.g. the heads head_range gives
+    the rank), with P and V in FP8. NVFP4 Q/K take their tensor scale from
+    the amax of the whole batch: the ranks' Q and K amax (two floats) are
+    max-reduced over ``group`` (torch.distributed) before quantizing, so every
+    share is quantized exactly as the whole batch would be. FP8 Q/K and V
+    have per-head scales and need no exchange. Every rank of the group must
+    call it, with its own share."""
+    import torch.distributed as dist
+    if kwargs.get("pv_format", "fp8") != "fp8":
+        raise ValueError("attention_sharded takes FP8 P/V (an NVFP4 V would need its tensor amax too)")
+    if qk_format != "nvfp4":
+        return attention(q, k, v, qk_format=qk_format, **kwargs)
+    _check_bf16(q)
+    _check_bf16(k)
+    amax = torch.cat([tensor_amax(q), tensor_amax(k)])
+    if dist.get_backend(group) == "gloo":
+        host = amax.cpu()
+        dist.all_reduce(host, op=dist.ReduceOp.MAX, group=group)
+        amax = host.to(q.device)
+    else:
+        dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    return attention(q, k, v, qk_format="nvfp4", qk_amax=(amax[0:1], amax[1:2]), **kwargs)
 
 
 def head_range(num_heads: int, world: int, rank: int) -> Tuple[int, int]:
